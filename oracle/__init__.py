@@ -1,0 +1,10 @@
+"""CPU oracle (numpy, float64 by default) for the TTT inner loop.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check in
+__graft_entry__ and by the benchmark's cpu_baseline / reference leg.  The
+product path never imports it, and it imports nothing from the product.
+"""
+from .ttt_oracle import *  # noqa: F401,F403
+from .ttt_oracle import (Model, make_model, prefill, prefill_sequence, scalar_kernels,  # noqa: F401
+                         scalar_kernels_ratio_form, chunk_update_closed, chunk_update_explicit,
+                         token_losses, token_gradients, unpack_blocks, pack_blocks)

@@ -1,0 +1,444 @@
+"""CPU oracle for the TTT-E2E inner loop with the E2-TTT closed-form chunk update.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, the smoke check in __graft_entry__ and
+the benchmark's cpu_baseline / reference leg may import or run this module.
+The product path (the CUDA library and its Python binding) never imports it
+and shares no code with it.
+
+What it computes, and where the pages define it
+-----------------------------------------------
+Pages cited by title:
+  [TTT-E2E]  "TTT-E2E：端到端测试时训练的长上下文语言建模"
+  [E2-TTT]   "Rethinking Expressivity and Efficiency in Test-Time Training"
+  [Review]   "NVIDIA开源TTT-E2E：128K上下文快2.7倍" (PaperDaily review)
+
+* The inner loop walks the sequence in chunks of b tokens; every token of a
+  chunk is predicted with the chunk-start weights and contributes its
+  next-token cross-entropy ([TTT-E2E] 内层循环：测试时训练; [E2-TTT]
+  高效的逐块更新机制, O^[r] = f_{W^[r-1]}(Q^[r])).
+* Only MLPs of the last blocks are updated; embedding, norms and attention
+  are frozen; an updated block may carry a frozen "static" MLP next to the
+  dynamic one ([Review] 元学习 section, dual-MLP paragraph).
+* Fast-weight MLP forms: GELU  y = W2 GELU(W1 x),  SwiGLU  y = W3 (SiLU(W1 x)
+  * (W2 x)), with a residual x + y ([E2-TTT] 快速权重网络实例化).  Reading: no
+  norm inside the block and no biases.
+* Frozen RMSNorm + LM head give the next-token loss ([TTT-E2E] 核心方法,
+  the loss l_t is next-token prediction).
+* G_t is the NEGATIVE gradient of token t's loss at the chunk-start weights;
+  the per-token recursion is M_t = beta_t M_{t-1} + eta_t G_t,
+  W_t = gamma_t W_{t-1} + M_t ([E2-TTT] 原始公式).
+* The chunk-end state follows Proposition 3.1 ([E2-TTT] 命题3.1):
+  M_C = btilde_0 M_0 + sum_t eta_t btilde_t G_t,
+  W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + sum_t eta_t btilde_t R_t G_t,
+  with suffix products btilde_t = prod_{i>t} beta_i, gtilde_t = prod_{i>t}
+  gamma_i and R_t = sum_{i>=t} gtilde_i / btilde_i.
+
+Readings where the pages leave a step open (each listed in the design doc):
+  * tokens[t] is the label of hidden row t (the caller pre-shifts);
+  * the reported chunk loss is the mean of the b token losses at chunk-start
+    weights, while the update uses the per-token gradients (a sum);
+  * RMSNorm: z = g * h / sqrt(mean(h^2) + eps), computed per row;
+  * GELU is the exact erf form; SiLU(x) = x sigmoid(x);
+  * the coefficients eta_t btilde_t R_t and btilde_0 R_1 are evaluated in the
+    division-free form the expanded equation of Proposition 3.1 gives
+    (sum over j of prod beta * gtilde_j), which equals the ratio form
+    wherever btilde > 0 and stays finite where a beta is 0.
+
+Parity pins (tests/test_oracle_*.py) tie every function here to something
+other than itself: exact-rational recursion, finite differences, torch
+autograd, closed forms of cross-entropy, the SGD reduction, resume and
+linearity.  No function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+from scipy.special import erf
+
+GELU = "gelu"
+SWIGLU = "swiglu"
+
+
+# ---------------------------------------------------------------------------
+# Elementwise functions ([E2-TTT] 快速权重网络实例化; [TTT-E2E] nn.GELU)
+# ---------------------------------------------------------------------------
+
+def gelu(x):
+    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def gelu_grad(x):
+    cdf = 0.5 * (1.0 + erf(x / math.sqrt(2.0)))
+    pdf = np.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+    return cdf + x * pdf
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def silu(x):
+    return x * sigmoid(x)
+
+
+def silu_grad(x):
+    s = sigmoid(x)
+    return s * (1.0 + x * (1.0 - s))
+
+
+# ---------------------------------------------------------------------------
+# Model description and weight packing
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Model:
+    """Frozen parts of the model plus the shapes of the fast weights.
+
+    lm_head E [V, d]; rms_gain g [d]; static[l] = list of the block's frozen
+    MLP matrices (same kind and shape as the dynamic MLP) or None.
+    """
+
+    d: int
+    hidden: int
+    vocab: int
+    n_blocks: int
+    mlp: str
+    rms_eps: float
+    lm_head: np.ndarray
+    rms_gain: np.ndarray
+    static: Optional[List[List[np.ndarray]]] = None
+
+    @property
+    def n_mats(self) -> int:
+        return 2 if self.mlp == GELU else 3
+
+    def mat_shapes(self) -> List[Tuple[int, int]]:
+        d, h = self.d, self.hidden
+        if self.mlp == GELU:
+            return [(h, d), (d, h)]
+        return [(h, d), (h, d), (d, h)]
+
+    def astype(self, dtype) -> "Model":
+        st = None
+        if self.static is not None:
+            st = [[m.astype(dtype) for m in blk] for blk in self.static]
+        return Model(self.d, self.hidden, self.vocab, self.n_blocks, self.mlp,
+                     self.rms_eps, self.lm_head.astype(dtype),
+                     self.rms_gain.astype(dtype), st)
+
+
+def unpack_blocks(flat: np.ndarray, n_blocks: int, shapes) -> List[List[np.ndarray]]:
+    """Flat [n_blocks][m] row-major matrices -> nested list (views)."""
+    out, off = [], 0
+    for _ in range(n_blocks):
+        blk = []
+        for (r, c) in shapes:
+            blk.append(flat[off:off + r * c].reshape(r, c))
+            off += r * c
+        out.append(blk)
+    assert off == flat.size, (off, flat.size)
+    return out
+
+
+def pack_blocks(blocks: List[List[np.ndarray]]) -> np.ndarray:
+    return np.concatenate([m.reshape(-1) for blk in blocks for m in blk])
+
+
+def make_model(d, hidden, vocab, n_blocks, mlp, rms_eps, lm_head, rms_gain,
+               static_w=None, dtype=np.float64) -> Model:
+    m = Model(d, hidden, vocab, n_blocks, mlp, rms_eps,
+              np.asarray(lm_head, dtype=dtype), np.asarray(rms_gain, dtype=dtype))
+    if static_w is not None:
+        m.static = unpack_blocks(np.asarray(static_w, dtype=dtype), n_blocks, m.mat_shapes())
+    return m
+
+
+# ---------------------------------------------------------------------------
+# Forward and per-token backward at fixed (chunk-start) weights
+# ---------------------------------------------------------------------------
+
+def mlp_forward(kind: str, mats: Sequence[np.ndarray], x: np.ndarray):
+    """y = MLP(x) for rows x [n, d]; returns (y, cache)."""
+    if kind == GELU:
+        W1, W2 = mats
+        U = x @ W1.T
+        A = gelu(U)
+        return A @ W2.T, (x, U, A)
+    W1, W2, W3 = mats
+    Ug = x @ W1.T
+    Uu = x @ W2.T
+    A = silu(Ug) * Uu
+    return A @ W3.T, (x, Ug, Uu, A)
+
+
+def mlp_backward(kind: str, mats, cache, d_out: np.ndarray):
+    """Backward of y = MLP(x) given dL/dy rows.
+
+    Returns (dL/dx through the MLP branch only, per-matrix factor pairs) where
+    the per-token gradient of matrix j is outer(L_j[t], R_j[t]).
+    """
+    if kind == GELU:
+        W1, W2 = mats
+        x, U, A = cache
+        dA = d_out @ W2
+        dU = dA * gelu_grad(U)
+        return dU @ W1, [(dU, x), (d_out, A)]
+    W1, W2, W3 = mats
+    x, Ug, Uu, A = cache
+    dA = d_out @ W3
+    dUg = dA * Uu * silu_grad(Ug)
+    dUu = dA * silu(Ug)
+    return dUg @ W1 + dUu @ W2, [(dUg, x), (dUu, x), (d_out, A)]
+
+
+def chunk_forward(model: Model, W: List[List[np.ndarray]], X: np.ndarray, y: np.ndarray):
+    """Per-token losses l_t at weights W for rows X [n, d] with labels y [n].
+
+    Block l applies h <- h + S_l(h) (if a static MLP exists), then
+    h <- h + D_l(h); then z = RMSNorm(h), logits = z E^T,
+    l_t = logsumexp(logits_t) - logits_t[y_t].
+    """
+    caches = []
+    h = X
+    for l in range(model.n_blocks):
+        if model.static is not None:
+            out, c = mlp_forward(model.mlp, model.static[l], h)
+            caches.append(("static", l, c))
+            h = h + out
+        out, c = mlp_forward(model.mlp, W[l], h)
+        caches.append(("dynamic", l, c))
+        h = h + out
+    ms = np.mean(h * h, axis=1)
+    r = 1.0 / np.sqrt(ms + model.rms_eps)
+    z = h * r[:, None] * model.rms_gain[None, :]
+    logits = z @ model.lm_head.T
+    mx = logits.max(axis=1)
+    lse = mx + np.log(np.sum(np.exp(logits - mx[:, None]), axis=1))
+    rows = np.arange(X.shape[0])
+    loss = lse - logits[rows, y]
+    return loss, (caches, h, r, logits, lse)
+
+
+def chunk_backward(model: Model, W, y, fwd):
+    """Per-token gradient factors of every dynamic matrix.
+
+    Returns grads[l][j] = (L, R) with dl_t/dW_{l,j} = outer(L[t], R[t]).
+    Each token's loss depends only on its own row, so one batched backward of
+    sum_t l_t yields every per-token gradient ([E2-TTT] 单次反向传播的链式法则分解).
+    """
+    caches, h, r, logits, lse = fwd
+    n = h.shape[0]
+    p = np.exp(logits - lse[:, None])
+    p[np.arange(n), y] -= 1.0                       # dl/dlogits
+    dz = p @ model.lm_head                          # dl/dz
+    gdz = dz * model.rms_gain[None, :]
+    d = model.d
+    dot = np.sum(gdz * h, axis=1)
+    dh = gdz * r[:, None] - h * (r ** 3 * dot / d)[:, None]   # RMSNorm backward
+
+    grads: List[List] = [None] * model.n_blocks
+    for kind, l, cache in reversed(caches):
+        mats = model.static[l] if kind == "static" else W[l]
+        dx_branch, pairs = mlp_backward(model.mlp, mats, cache, dh)
+        if kind == "dynamic":
+            grads[l] = pairs
+        dh = dh + dx_branch                         # residual
+    return grads
+
+
+# ---------------------------------------------------------------------------
+# Scalar kernels ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1)
+# ---------------------------------------------------------------------------
+
+def suffix_products(v: np.ndarray) -> np.ndarray:
+    """out[t] = prod_{i=t+1}^{C} v_i for t = 0..C (1-indexed v), out[C] = 1."""
+    C = v.shape[0]
+    out = np.ones(C + 1, dtype=np.float64)
+    for t in range(C - 1, -1, -1):
+        out[t] = out[t + 1] * float(v[t])
+    return out
+
+
+def scalar_kernels(eta, beta, gamma):
+    """Coefficients of Proposition 3.1 for one chunk of length C.
+
+    Inputs are the chunk's eta, beta, gamma (0-based arrays; entry k is token
+    t = k + 1).  Returns (K_W [C], K_M [C], gtilde_0, btilde_0, c_M) with
+      K_M_t = eta_t btilde_t,
+      K_W_t = eta_t btilde_t R_t = eta_t sum_{j=t}^{C} (prod_{i=t+1}^{j} beta_i) gtilde_j,
+      c_M   = btilde_0 R_1       = sum_{j=1}^{C} (prod_{i=1}^{j} beta_i) gtilde_j,
+    i.e. the gradient and momentum terms of the expanded chunk-end equation
+    (the one printed just before the definitions of btilde, gtilde, R).
+    Evaluated in float64.
+    """
+    eta = np.asarray(eta, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    gamma = np.asarray(gamma, dtype=np.float64)
+    C = eta.shape[0]
+    bt = suffix_products(beta)    # bt[k] = btilde_k, k = 0..C
+    gt = suffix_products(gamma)   # gt[k] = gtilde_k
+    KM = eta * bt[1:]
+    KW = np.empty(C, dtype=np.float64)
+    for k in range(C):            # token t = k+1
+        # prod_{i=t+1}^{j} beta_i for j = t..C  ->  cumprod of beta[k+1:], with 1 for j = t
+        run = np.concatenate(([1.0], np.cumprod(beta[k + 1:])))
+        KW[k] = eta[k] * np.sum(run * gt[k + 1:])
+    run0 = np.cumprod(beta)       # prod_{i=1}^{j} beta_i, j = 1..C
+    cM = float(np.sum(run0 * gt[1:]))
+    return KW, KM, float(gt[0]), float(bt[0]), cM
+
+
+def scalar_kernels_ratio_form(eta, beta, gamma):
+    """The same coefficients through R_t = sum_{i>=t} gtilde_i / btilde_i.
+
+    This is the form printed in the definitions; it divides by btilde and is
+    only defined where every btilde_i > 0.  Kept for the pins.
+    """
+    eta = np.asarray(eta, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    gamma = np.asarray(gamma, dtype=np.float64)
+    C = eta.shape[0]
+    bt = suffix_products(beta)
+    gt = suffix_products(gamma)
+    R = np.array([np.sum(gt[t:C + 1] / bt[t:C + 1]) for t in range(1, C + 1)])  # R_1..R_C
+    KW = eta * bt[1:] * R
+    KM = eta * bt[1:]
+    return KW, KM, float(gt[0]), float(bt[0]), float(bt[0] * R[0])
+
+
+# ---------------------------------------------------------------------------
+# Chunk update: closed form (Prop. 3.1 / Algorithm 1) and explicit recursion
+# ---------------------------------------------------------------------------
+
+def chunk_update_closed(W, M, grads, eta, beta, gamma):
+    """Algorithm 1 lines 2 and 4-7: aggregate with K_W and K_M, then
+    W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + dW and M_C = btilde_0 M_0 + dM.
+
+    G_t = -outer(L[t], R[t]), so sum_t K_t G_t = -(K * L)^T R.
+    """
+    KW, KM, g0, b0, cM = scalar_kernels(eta, beta, gamma)
+    dt = W[0][0].dtype
+    KW = KW.astype(dt)
+    KM = KM.astype(dt)
+    newW, newM = [], []
+    for l in range(len(W)):
+        bw, bm = [], []
+        for j in range(len(W[l])):
+            Lf, Rf = grads[l][j]
+            dW = -((Lf * KW[:, None]).T @ Rf)
+            dM = -((Lf * KM[:, None]).T @ Rf)
+            bw.append((dt.type(g0) * W[l][j] + dt.type(cM) * M[l][j] + dW).astype(dt))
+            bm.append((dt.type(b0) * M[l][j] + dM).astype(dt))
+        newW.append(bw)
+        newM.append(bm)
+    return newW, newM
+
+
+def chunk_update_explicit(W, M, grads, eta, beta, gamma):
+    """The per-token recursion itself ([E2-TTT] 原始公式), with every G_t
+    materialised:  M_t = beta_t M_{t-1} + eta_t G_t,  W_t = gamma_t W_{t-1} + M_t."""
+    newW, newM = [], []
+    C = len(eta)
+    for l in range(len(W)):
+        bw, bm = [], []
+        for j in range(len(W[l])):
+            Lf, Rf = grads[l][j]
+            Wt = W[l][j].copy()
+            Mt = M[l][j].copy()
+            for k in range(C):
+                G = -np.outer(Lf[k], Rf[k])
+                Mt = beta[k] * Mt + eta[k] * G
+                Wt = gamma[k] * Wt + Mt
+            bw.append(Wt)
+            bm.append(Mt)
+        newW.append(bw)
+        newM.append(bm)
+    return newW, newM
+
+
+# ---------------------------------------------------------------------------
+# The inner loop over a whole sequence
+# ---------------------------------------------------------------------------
+
+def prefill_sequence(model: Model, W0, M0, hidden, tokens, eta, beta, gamma, b,
+                     update: str = "closed", n_chunks: Optional[int] = None):
+    """Chunk-serial inner loop for one sequence.
+
+    W0, M0: nested lists [n_blocks][m] of matrices; hidden [T, d]; tokens [T];
+    eta/beta/gamma [T].  Returns (W_final, M_final, chunk_loss [n_chunks]).
+    ``n_chunks`` limits the run to the first chunks (for sampled parity).
+    """
+    T = hidden.shape[0]
+    if T % b != 0:
+        raise ValueError("T must be a multiple of b")
+    nc = T // b if n_chunks is None else n_chunks
+    W = [[m.copy() for m in blk] for blk in W0]
+    M = [[m.copy() for m in blk] for blk in M0]
+    losses = np.zeros(nc, dtype=np.float64)
+    step = chunk_update_closed if update == "closed" else chunk_update_explicit
+    for c in range(nc):
+        s = slice(c * b, (c + 1) * b)
+        X = hidden[s]
+        y = tokens[s]
+        loss, fwd = chunk_forward(model, W, X, y)     # line 1: at chunk-start weights
+        losses[c] = float(np.mean(loss))
+        grads = chunk_backward(model, W, y, fwd)      # line 3: single backward
+        W, M = step(W, M, grads, eta[s], beta[s], gamma[s])
+    return W, M, losses
+
+
+def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
+            dtype=np.float64, update: str = "closed", n_chunks: Optional[int] = None):
+    """Batched inner loop with the C-ABI's flat layouts.
+
+    hidden [B,T,d], tokens [B,T], eta/beta/gamma [B,T],
+    W0_flat / M0_flat [B * n_blocks * m * h * d].
+    Returns (W_flat, M_flat, chunk_loss [B, n_chunks]) in ``dtype``.
+    """
+    mdl = model.astype(dtype)
+    B = hidden.shape[0]
+    shapes = mdl.mat_shapes()
+    per_seq = mdl.n_blocks * sum(r * c for r, c in shapes)
+    W0_flat = np.asarray(W0_flat, dtype=dtype).reshape(B, per_seq)
+    M0_flat = np.asarray(M0_flat, dtype=dtype).reshape(B, per_seq)
+    Ws, Ms, Ls = [], [], []
+    for s in range(B):
+        W0 = unpack_blocks(W0_flat[s].copy(), mdl.n_blocks, shapes)
+        M0 = unpack_blocks(M0_flat[s].copy(), mdl.n_blocks, shapes)
+        W, M, L = prefill_sequence(mdl, W0, M0, np.asarray(hidden[s], dtype=dtype),
+                                   np.asarray(tokens[s]), eta[s], beta[s], gamma[s], b,
+                                   update=update, n_chunks=n_chunks)
+        Ws.append(pack_blocks(W))
+        Ms.append(pack_blocks(M))
+        Ls.append(L)
+    return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls)
+
+
+def token_losses(model: Model, W_flat, X, y, dtype=np.float64):
+    """Per-token losses of rows X at fast weights W_flat (one sequence)."""
+    mdl = model.astype(dtype)
+    W = unpack_blocks(np.asarray(W_flat, dtype=dtype), mdl.n_blocks, mdl.mat_shapes())
+    loss, _ = chunk_forward(mdl, W, np.asarray(X, dtype=dtype), np.asarray(y))
+    return loss
+
+
+def token_gradients(model: Model, W_flat, X, y, dtype=np.float64):
+    """Per-token gradients dl_t/dW as a dense array [n, n_params] (tiny shapes only)."""
+    mdl = model.astype(dtype)
+    W = unpack_blocks(np.asarray(W_flat, dtype=dtype), mdl.n_blocks, mdl.mat_shapes())
+    X = np.asarray(X, dtype=dtype)
+    y = np.asarray(y)
+    _, fwd = chunk_forward(mdl, W, X, y)
+    grads = chunk_backward(mdl, W, y, fwd)
+    n = X.shape[0]
+    rows = []
+    for t in range(n):
+        parts = []
+        for l in range(mdl.n_blocks):
+            for (Lf, Rf) in grads[l]:
+                parts.append(np.outer(Lf[t], Rf[t]).reshape(-1))
+        rows.append(np.concatenate(parts))
+    return np.stack(rows)

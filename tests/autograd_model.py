@@ -1,0 +1,61 @@
+"""An independent restatement of the per-token loss in torch (float64, CPU), used
+only to pin the numpy oracle: gradients come from torch autograd, not from the
+oracle's hand-written backward.
+
+Model ("TTT-E2E：端到端测试时训练的长上下文语言建模", 核心方法; dynamic MLP forms
+from "Rethinking Expressivity and Efficiency in Test-Time Training",
+快速权重网络实例化): per block, optional frozen static MLP then the dynamic MLP,
+each with a residual; frozen RMSNorm; frozen LM head; next-token cross-entropy
+per token.
+"""
+import torch
+import torch.nn.functional as F
+
+
+def _mlp(kind, mats, x):
+    if kind == "gelu":
+        w1, w2 = mats
+        return F.gelu(x @ w1.T, approximate="none") @ w2.T
+    w1, w2, w3 = mats
+    return (F.silu(x @ w1.T) * (x @ w2.T)) @ w3.T
+
+
+def split_blocks(flat, n_blocks, shapes):
+    out, off = [], 0
+    for _ in range(n_blocks):
+        blk = []
+        for r, c in shapes:
+            blk.append(flat[off:off + r * c].reshape(r, c))
+            off += r * c
+        out.append(blk)
+    return out
+
+
+def shapes_of(kind, d, h):
+    return [(h, d), (d, h)] if kind == "gelu" else [(h, d), (h, d), (d, h)]
+
+
+def losses(kind, d, h, n_blocks, eps, E, g, static_flat, W_flat, X, y):
+    """Per-token losses (torch tensors, float64)."""
+    shapes = shapes_of(kind, d, h)
+    Wb = split_blocks(W_flat, n_blocks, shapes)
+    Sb = split_blocks(static_flat, n_blocks, shapes) if static_flat is not None else None
+    hcur = X
+    for l in range(n_blocks):
+        if Sb is not None:
+            hcur = hcur + _mlp(kind, Sb[l], hcur)
+        hcur = hcur + _mlp(kind, Wb[l], hcur)
+    z = hcur * torch.rsqrt(hcur.pow(2).mean(dim=1, keepdim=True) + eps) * g
+    logits = z @ E.T
+    return F.cross_entropy(logits, y, reduction="none")
+
+
+def per_token_grads(kind, d, h, n_blocks, eps, E, g, static_flat, W_flat, X, y):
+    """[n, n_params] per-token gradients by autograd."""
+    W = W_flat.clone().requires_grad_(True)
+    L = losses(kind, d, h, n_blocks, eps, E, g, static_flat, W, X, y)
+    rows = []
+    for t in range(L.shape[0]):
+        (gt,) = torch.autograd.grad(L[t], W, retain_graph=True)
+        rows.append(gt.clone())
+    return torch.stack(rows), L.detach()

@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each pin cites the passage it checks.  Pages by title:
+  [E2-TTT]  "Rethinking Expressivity and Efficiency in Test-Time Training"
+  [TTT-E2E] "TTT-E2E：端到端测试时训练的长上下文语言建模"
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import ttt_oracle as O
+from tests import autograd_model as AM
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def tiny_setup(kind="gelu", d=4, h=6, V=7, L=2, static=True, T=12, seed=1,
+               m0=0.05, scalars="e2ttt"):
+    rng = np.random.default_rng(seed)
+    shapes = AM.shapes_of(kind, d, h)
+    per_block = sum(r * c for r, c in shapes)
+    E = rng.normal(0, 0.5, (V, d))
+    g = rng.uniform(0.5, 1.5, d)
+    static_w = rng.normal(0, 0.4, L * per_block) if static else None
+    W0 = rng.normal(0, 0.4, L * per_block)
+    M0 = rng.normal(0, m0, L * per_block) if m0 else np.zeros(L * per_block)
+    X = rng.normal(0, 1, (T, d))
+    y = rng.integers(0, V, T)
+    if scalars == "sgd":
+        eta = np.full(T, 0.1)
+        beta = np.zeros(T)
+        gamma = np.ones(T)
+    else:
+        eta = 0.05 / (1 + np.exp(-rng.normal(size=T)))
+        beta = rng.uniform(0.8, 0.99, T)
+        gamma = rng.uniform(0.99, 1.0, T)
+    model = O.make_model(d, h, V, L, kind, 1e-6, E, g, static_w)
+    return dict(model=model, kind=kind, d=d, h=h, V=V, L=L, E=E, g=g, static_w=static_w,
+                W0=W0, M0=M0, X=X, y=y, eta=eta, beta=beta, gamma=gamma)
+
+
+def run_prefill(s, b, update="closed", **over):
+    p = dict(s)
+    p.update(over)
+    W, M, Ls = O.prefill(p["model"], p["W0"], p["M0"], p["X"][None], p["y"][None],
+                         p["eta"][None], p["beta"][None], p["gamma"][None], b,
+                         update=update)
+    return W, M, Ls[0]
+
+
+def rel(a, b):
+    return float(np.linalg.norm(np.asarray(a) - np.asarray(b)) / max(np.linalg.norm(np.asarray(b)), 1e-300))
+
+
+# ---------------------------------------------------------------------------
+# 1. Scalar kernels against the exact recursion in rational arithmetic
+#    ([E2-TTT] 原始公式 vs 命题3.1)
+# ---------------------------------------------------------------------------
+
+def exact_coefficients(eta, beta, gamma):
+    """Run M_t = beta_t M_{t-1} + eta_t G_t, W_t = gamma_t W_{t-1} + M_t exactly,
+    with W_0, M_0, G_1..G_C as independent basis vectors.  Returns the
+    coefficient vectors of W_C and M_C over (W_0, M_0, G_1..G_C)."""
+    C = len(eta)
+    n = C + 2
+    W = [Fraction(0)] * n
+    M = [Fraction(0)] * n
+    W[0] = Fraction(1)
+    M[1] = Fraction(1)
+    for t in range(C):
+        M = [beta[t] * m for m in M]
+        M[2 + t] += eta[t]
+        W = [gamma[t] * w + m for w, m in zip(W, M)]
+    return W, M
+
+
+@pytest.mark.parametrize("case", ["random", "beta_zero", "ones", "mixed_zero"])
+def test_scalar_kernels_match_exact_recursion(case):
+    rng = np.random.default_rng(7)
+    C = 9
+    den = 97
+    eta = [Fraction(int(rng.integers(1, 50)), 1000) for _ in range(C)]
+    if case == "random":
+        beta = [Fraction(int(rng.integers(60, 97)), den) for _ in range(C)]
+        gamma = [Fraction(int(rng.integers(80, 97)), den) for _ in range(C)]
+    elif case == "beta_zero":          # plain SGD-like momentum-free chunk
+        beta = [Fraction(0)] * C
+        gamma = [Fraction(1)] * C
+    elif case == "ones":
+        beta = [Fraction(1)] * C
+        gamma = [Fraction(1)] * C
+    else:                              # a zero momentum factor in mid-chunk
+        beta = [Fraction(int(rng.integers(60, 97)), den) for _ in range(C)]
+        beta[4] = Fraction(0)
+        gamma = [Fraction(int(rng.integers(80, 97)), den) for _ in range(C)]
+    Wc, Mc = exact_coefficients(eta, beta, gamma)
+    KW, KM, g0, b0, cM = O.scalar_kernels([float(x) for x in eta], [float(x) for x in beta],
+                                          [float(x) for x in gamma])
+    tol = 1e-14
+    assert abs(g0 - float(Wc[0])) <= tol * max(1, abs(float(Wc[0])))
+    assert abs(cM - float(Wc[1])) <= tol * max(1, abs(float(Wc[1])))
+    assert abs(b0 - float(Mc[1])) <= tol
+    assert float(Mc[0]) == 0.0
+    np.testing.assert_allclose(KW, [float(x) for x in Wc[2:]], rtol=1e-13, atol=1e-18)
+    np.testing.assert_allclose(KM, [float(x) for x in Mc[2:]], rtol=1e-13, atol=1e-18)
+
+
+def test_scalar_kernels_match_ratio_form():
+    """Division-free evaluation == the printed R_t = sum gtilde_i / btilde_i form."""
+    rng = np.random.default_rng(3)
+    for C in (1, 2, 16, 64):
+        eta = 0.01 / (1 + np.exp(-rng.normal(size=C)))
+        beta = rng.uniform(0.8, 0.99, C)
+        gamma = rng.uniform(0.99, 1.0, C)
+        a = O.scalar_kernels(eta, beta, gamma)
+        r = O.scalar_kernels_ratio_form(eta, beta, gamma)
+        np.testing.assert_allclose(a[0], r[0], rtol=1e-12)
+        np.testing.assert_allclose(a[1], r[1], rtol=1e-12)
+        np.testing.assert_allclose(a[2:], r[2:], rtol=1e-12)
+
+
+def test_R_limits_and_bounds():
+    """[E2-TTT] 累积核 R_t 的稳定性分析: beta, gamma -> 1 gives R_t = C - t + 1,
+    so K_W <= eta * C; and 0 <= K_M <= eta, 0 <= K_W <= eta (C - t + 1)."""
+    C = 32
+    eta = np.linspace(0.001, 0.01, C)
+    KW, KM, g0, b0, cM = O.scalar_kernels(eta, np.ones(C), np.ones(C))
+    t = np.arange(1, C + 1)
+    np.testing.assert_allclose(KW, eta * (C - t + 1), rtol=1e-15)
+    np.testing.assert_allclose(KM, eta, rtol=1e-15)
+    assert g0 == 1.0 and b0 == 1.0 and cM == pytest.approx(C, rel=1e-15)
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        beta = rng.uniform(0, 1, C)
+        gamma = rng.uniform(0, 1, C)
+        KW, KM, g0, b0, cM = O.scalar_kernels(eta, beta, gamma)
+        assert np.all(KM >= 0) and np.all(KM <= eta * (1 + 1e-15))
+        assert np.all(KW >= 0) and np.all(KW <= eta * (C - t + 1) * (1 + 1e-15))
+        assert 0 <= cM <= C
+
+
+def test_scalar_kernels_underflow_finite():
+    """b = 1024 with beta ~ U(.8,.99): prod beta underflows float32 (about 1e-47),
+    the ratio form would divide by it; the coefficients must stay finite."""
+    rng = np.random.default_rng(0)
+    C = 1024
+    beta = rng.uniform(0.8, 0.99, C)
+    gamma = rng.uniform(0.99, 1.0, C)
+    eta = np.full(C, 0.01)
+    KW, KM, g0, b0, cM = O.scalar_kernels(eta, beta, gamma)
+    assert np.all(np.isfinite(KW)) and np.all(np.isfinite(KM))
+    assert np.float32(b0) == 0.0          # would underflow in float32
+    assert np.all(KW <= 0.01 * (C - np.arange(C)))
+
+
+# ---------------------------------------------------------------------------
+# 2. Closed form == explicit per-token recursion on the full model
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind,static", [("gelu", False), ("gelu", True), ("swiglu", True), ("swiglu", False)])
+def test_closed_form_equals_recursion(kind, static):
+    s = tiny_setup(kind=kind, static=static, h=6 if kind == "gelu" else 5, T=12)
+    W1, M1, L1 = run_prefill(s, 4, "closed")
+    W2, M2, L2 = run_prefill(s, 4, "explicit")
+    assert rel(W1, W2) < 1e-12
+    assert rel(M1, M2) < 1e-12
+    np.testing.assert_allclose(L1, L2, rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# 3. Per-token gradients: finite differences and autograd
+#    ([E2-TTT] 单次反向传播的链式法则分解)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["gelu", "swiglu"])
+def test_gradients_match_finite_differences(kind):
+    s = tiny_setup(kind=kind, d=3, h=4, V=5, L=2, static=True, T=3)
+    model, W, X, y = s["model"], s["W0"], s["X"], s["y"]
+    G = O.token_gradients(model, W, X, y)
+    eps = 1e-6
+    fd = np.zeros_like(G)
+    for i in range(W.size):
+        Wp = W.copy(); Wp[i] += eps
+        Wm = W.copy(); Wm[i] -= eps
+        fd[:, i] = (O.token_losses(model, Wp, X, y) - O.token_losses(model, Wm, X, y)) / (2 * eps)
+    np.testing.assert_allclose(G, fd, rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("kind,static,L", [("gelu", False, 1), ("gelu", True, 3), ("swiglu", True, 2)])
+def test_gradients_and_losses_match_autograd(kind, static, L):
+    s = tiny_setup(kind=kind, d=6, h=8, V=11, L=L, static=static, T=5)
+    T_ = lambda a: None if a is None else torch.tensor(a, dtype=torch.float64)
+    Ga, La = AM.per_token_grads(kind, 6, 8, L, 1e-6, T_(s["E"]), T_(s["g"]), T_(s["static_w"]),
+                                T_(s["W0"]), T_(s["X"]), torch.tensor(s["y"]))
+    G = O.token_gradients(s["model"], s["W0"], s["X"], s["y"])
+    Lo = O.token_losses(s["model"], s["W0"], s["X"], s["y"])
+    np.testing.assert_allclose(Lo, La.numpy(), rtol=1e-12)
+    np.testing.assert_allclose(G, Ga.numpy(), rtol=1e-10, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# 4. SGD reduction ([TTT-E2E] 持续学习框架: W_t = W_{t-1} - alpha grad l_t)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["gelu", "swiglu"])
+def test_b1_sgd_is_online_sgd(kind):
+    """b = 1, beta = 0, gamma = 1, eta = alpha: the chunk update is exactly one
+    online SGD step per token, with the loss taken before the step."""
+    s = tiny_setup(kind=kind, d=5, h=7, V=9, L=2, static=True, T=10, scalars="sgd", m0=0.3)
+    alpha = 0.1
+    W, M, Ls = run_prefill(s, 1)
+    T_ = lambda a: None if a is None else torch.tensor(a, dtype=torch.float64)
+    Wt = T_(s["W0"])
+    ref_losses = []
+    for t in range(10):
+        Wv = Wt.clone().requires_grad_(True)
+        l = AM.losses(kind, 5, 7, 2, 1e-6, T_(s["E"]), T_(s["g"]), T_(s["static_w"]), Wv,
+                      T_(s["X"][t:t + 1]), torch.tensor(s["y"][t:t + 1]))[0]
+        (gr,) = torch.autograd.grad(l, Wv)
+        ref_losses.append(float(l))
+        Wt = Wt - alpha * gr
+    assert rel(W, Wt.numpy()) < 1e-12
+    np.testing.assert_allclose(Ls, ref_losses, rtol=1e-12)
+
+
+def test_chunked_sgd_uses_chunk_start_gradients():
+    """b = 4 SGD: W_C = W_0 - alpha sum_t grad l_t(W_0) and M_C = eta_C G_C
+    (only the last token's gradient survives when beta = 0)."""
+    s = tiny_setup(kind="gelu", d=5, h=7, V=9, L=1, static=False, T=4, scalars="sgd", m0=0.3)
+    W, M, Ls = run_prefill(s, 4)
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    Wv = T_(s["W0"]).requires_grad_(True)
+    l = AM.losses("gelu", 5, 7, 1, 1e-6, T_(s["E"]), T_(s["g"]), None, Wv, T_(s["X"]), torch.tensor(s["y"]))
+    (gsum,) = torch.autograd.grad(l.sum(), Wv, retain_graph=True)
+    (glast,) = torch.autograd.grad(l[3], Wv)
+    assert rel(W, (T_(s["W0"]) - 0.1 * gsum).numpy()) < 1e-12
+    assert rel(M, (-0.1 * glast).numpy()) < 1e-12
+    assert Ls[0] == pytest.approx(float(l.mean()), rel=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 5. Cross-entropy closed forms
+# ---------------------------------------------------------------------------
+
+def test_zero_lm_head_gives_log_v_and_no_gradient():
+    s = tiny_setup(kind="swiglu", d=4, h=5, V=13, L=2, static=True, T=8)
+    s["model"].lm_head[:] = 0.0
+    W, M, Ls = run_prefill(s, 4)
+    np.testing.assert_allclose(Ls, np.log(13.0), rtol=1e-14)
+    # no gradient: only decay / momentum act
+    W_ref, M_ref = s["W0"].copy(), s["M0"].copy()
+    for c in range(2):
+        sl = slice(4 * c, 4 * c + 4)
+        KW, KM, g0, b0, cM = O.scalar_kernels(s["eta"][sl], s["beta"][sl], s["gamma"][sl])
+        W_ref, M_ref = g0 * W_ref + cM * M_ref, b0 * M_ref
+    assert rel(W, W_ref) < 1e-13 and rel(M, M_ref) < 1e-13
+
+
+def test_two_class_loss_is_softplus():
+    """V = 2: l = softplus(logit_other - logit_target).  With W1 = 0 every
+    dynamic MLP outputs 0 (GELU(0) = 0), so h = x and the logits are
+    RMSNorm(x) E^T, computed here directly."""
+    s = tiny_setup(kind="gelu", d=6, h=4, V=2, L=1, static=False, T=8)
+    W = s["W0"].copy()
+    W[:4 * 6] = 0.0
+    X, y, E, g = s["X"], s["y"], s["E"], s["g"]
+    z = X / np.sqrt(np.mean(X ** 2, axis=1, keepdims=True) + 1e-6) * g
+    lg = z @ E.T
+    other = lg[np.arange(8), 1 - y]
+    target = lg[np.arange(8), y]
+    expect = np.log1p(np.exp(other - target))
+    np.testing.assert_allclose(O.token_losses(s["model"], W, X, y), expect, rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# 6. Resume, linearity, chunk-start losses
+# ---------------------------------------------------------------------------
+
+def test_resume_equivalence():
+    """Only the chunk-end state crosses chunk boundaries ([E2-TTT] 原始公式,
+    last sentence): prefill(T) == prefill(T1) then prefill(T - T1)."""
+    s = tiny_setup(kind="swiglu", d=4, h=5, V=7, L=2, static=True, T=12)
+    W, M, Ls = run_prefill(s, 3)
+    T1 = 6
+    s1 = dict(s, X=s["X"][:T1], y=s["y"][:T1], eta=s["eta"][:T1], beta=s["beta"][:T1], gamma=s["gamma"][:T1])
+    Wa, Ma, La = run_prefill(s1, 3)
+    s2 = dict(s, X=s["X"][T1:], y=s["y"][T1:], eta=s["eta"][T1:], beta=s["beta"][T1:], gamma=s["gamma"][T1:],
+              W0=Wa, M0=Ma)
+    Wb, Mb, Lb = run_prefill(s2, 3)
+    assert rel(Wb, W) < 1e-14 and rel(Mb, M) < 1e-14
+    np.testing.assert_allclose(np.concatenate([La, Lb]), Ls, rtol=1e-14)
+
+
+def test_single_chunk_update_is_linear_in_eta():
+    s = tiny_setup(kind="gelu", d=4, h=6, V=7, L=2, static=True, T=6)
+    W1, M1, _ = run_prefill(s, 6)
+    W3, M3, _ = run_prefill(s, 6, eta=3.0 * s["eta"])
+    KW, KM, g0, b0, cM = O.scalar_kernels(s["eta"], s["beta"], s["gamma"])
+    base_W = g0 * s["W0"] + cM * s["M0"]
+    base_M = b0 * s["M0"]
+    assert rel(W3 - base_W, 3.0 * (W1 - base_W)) < 1e-12
+    assert rel(M3 - base_M, 3.0 * (M1 - base_M)) < 1e-12
+
+
+def test_chunk_loss_is_mean_at_chunk_start_weights():
+    """[E2-TTT] O^[r] = f_{W^[r-1]}(Q^[r]): chunk c's loss uses the state after c chunks."""
+    s = tiny_setup(kind="swiglu", d=4, h=5, V=7, L=2, static=True, T=12)
+    _, _, Ls = run_prefill(s, 4)
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    for c in range(3):
+        if c == 0:
+            Wc = s["W0"]
+        else:
+            sc = dict(s, X=s["X"][:4 * c], y=s["y"][:4 * c], eta=s["eta"][:4 * c],
+                      beta=s["beta"][:4 * c], gamma=s["gamma"][:4 * c])
+            Wc, _, _ = run_prefill(sc, 4)
+        l = AM.losses("swiglu", 4, 5, 2, 1e-6, T_(s["E"]), T_(s["g"]), T_(s["static_w"]), T_(Wc),
+                      T_(s["X"][4 * c:4 * c + 4]), torch.tensor(s["y"][4 * c:4 * c + 4]))
+        assert Ls[c] == pytest.approx(float(l.mean()), rel=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 7. Planted mistakes: a plausible bug anywhere must fail one of the pins
+# ---------------------------------------------------------------------------
+
+def _must_fail(fn, *a, **k):
+    with pytest.raises(AssertionError):
+        fn(*a, **k)
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    # (a) wrong sign of G in the aggregation
+    orig = O.chunk_update_closed
+
+    def flipped(W, M, grads, eta, beta, gamma):
+        g2 = [[(-Lf, Rf) for (Lf, Rf) in blk] for blk in grads]
+        return orig(W, M, g2, eta, beta, gamma)
+    monkeypatch.setattr(O, "chunk_update_closed", flipped)
+    _must_fail(test_chunked_sgd_uses_chunk_start_gradients)
+    monkeypatch.setattr(O, "chunk_update_closed", orig)
+
+    # (b) dropped momentum carry c_M in W_C
+    orig_sk = O.scalar_kernels
+
+    def no_cm(eta, beta, gamma):
+        KW, KM, g0, b0, cM = orig_sk(eta, beta, gamma)
+        return KW, KM, g0, b0, 0.0
+    monkeypatch.setattr(O, "scalar_kernels", no_cm)
+    _must_fail(test_closed_form_equals_recursion, "gelu", True)
+    monkeypatch.setattr(O, "scalar_kernels", orig_sk)
+
+    # (c) off-by-one suffix product (btilde_{t-1} instead of btilde_t)
+    def shifted(eta, beta, gamma):
+        KW, KM, g0, b0, cM = orig_sk(eta, beta, gamma)
+        bt = O.suffix_products(np.asarray(beta, dtype=np.float64))
+        return KW, np.asarray(eta) * bt[:-1], g0, b0, cM
+    monkeypatch.setattr(O, "scalar_kernels", shifted)
+    _must_fail(test_scalar_kernels_match_exact_recursion, "random")
+    monkeypatch.setattr(O, "scalar_kernels", orig_sk)
+
+    # (d) GELU derivative missing its x * pdf term
+    monkeypatch.setattr(O, "gelu_grad", lambda x: 0.5 * (1.0 + O.erf(x / np.sqrt(2.0))))
+    _must_fail(test_gradients_match_finite_differences, "gelu")
+    monkeypatch.undo()
+
+    # (e) RMSNorm backward without the projection term
+    def _bwd_no_proj(model, W, y, fwd):
+        caches, h, r, logits, lse = fwd
+        n = h.shape[0]
+        p = np.exp(logits - lse[:, None])
+        p[np.arange(n), y] -= 1.0
+        dh = (p @ model.lm_head) * model.rms_gain[None, :] * r[:, None]
+        grads = [None] * model.n_blocks
+        for kind, l, cache in reversed(caches):
+            mats = model.static[l] if kind == "static" else W[l]
+            dxb, pairs = O.mlp_backward(model.mlp, mats, cache, dh)
+            if kind == "dynamic":
+                grads[l] = pairs
+            dh = dh + dxb
+        return grads
+    monkeypatch.setattr(O, "chunk_backward", _bwd_no_proj)
+    _must_fail(test_gradients_match_finite_differences, "swiglu")
+    monkeypatch.undo()
+
+    # (f) the residual dropped from the backward of a block
+    orig_mb = O.mlp_backward
+
+    def no_resid(kind, mats, cache, d_out):
+        dx, pairs = orig_mb(kind, mats, cache, d_out)
+        return dx - d_out, pairs   # cancels the residual the caller adds
+    monkeypatch.setattr(O, "mlp_backward", no_resid)
+    _must_fail(test_gradients_and_losses_match_autograd, "gelu", True, 3)
+    monkeypatch.undo()
