@@ -1,0 +1,171 @@
+/*
+ * ttt.h -- C ABI of libttt: the inner loop of end-to-end test-time training
+ * (TTT-E2E) with the E2-TTT closed-form chunk update, on one B200 (sm_100a).
+ *
+ * Pages (cited by title and section):
+ *   [TTT-E2E] "TTT-E2E：端到端测试时训练的长上下文语言建模"
+ *   [E2-TTT]  "Rethinking Expressivity and Efficiency in Test-Time Training"
+ *   [Review]  "NVIDIA开源TTT-E2E：128K上下文快2.7倍"
+ *
+ * What one call computes ([TTT-E2E] 内层循环：测试时训练; [E2-TTT] 方法细节,
+ * Algorithm 1).  For each sequence, the T hidden rows are cut into chunks of b
+ * rows.  For each chunk, in order:
+ *   1. forward at the chunk-start fast weights through n_blocks residual
+ *      blocks, each  h <- h + S_l(h)  (frozen static MLP, optional) then
+ *      h <- h + D_l(h)  (dynamic MLP, fast weights W_l);
+ *      GELU:   D(x) = W2 GELU(W1 x);   SwiGLU: D(x) = W3 (SiLU(W1 x) * (W2 x))
+ *      ([E2-TTT] 快速权重网络实例化, without the inner LayerNorm; [Review]
+ *      dual-MLP paragraph);
+ *   2. frozen RMSNorm + LM head, next-token cross-entropy l_t against
+ *      tokens[t] ([TTT-E2E] 核心方法);
+ *   3. one backward giving the per-token negative gradients G_t of every
+ *      dynamic matrix at the chunk-start weights;
+ *   4. chunk-end state by Proposition 3.1 ([E2-TTT] 命题3.1):
+ *        M_C = btilde_0 M_0 + sum_t eta_t btilde_t G_t
+ *        W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + sum_t eta_t btilde_t R_t G_t
+ *      with btilde_t = prod_{i>t} beta_i, gtilde_t = prod_{i>t} gamma_i,
+ *      R_t = sum_{i>=t} gtilde_i / btilde_i (evaluated without division).
+ * This equals the per-token recursion M_t = beta_t M_{t-1} + eta_t G_t,
+ * W_t = gamma_t W_{t-1} + M_t ([E2-TTT] 原始公式) at every chunk end.
+ *
+ * Conventions shared by every entry point
+ *   - Every array argument is a DEVICE pointer on the handle's device,
+ *     row-major, float32 unless stated, owned by the caller.  Nothing is
+ *     freed or retained by the library after a call returns, except the
+ *     frozen-parameter copies a handle owns.
+ *   - Enqueued work is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Argument and shape errors are returned
+ *     synchronously and launch nothing.
+ *   - Errors found on the device (token out of range, non-finite loss, a
+ *     bounded wait that ran out) are recorded in the handle's device status
+ *     word and read back with ttt_get_device_status().
+ *   - Not thread-safe per handle; different handles are independent.
+ *   - Fast-weight packing, per sequence: [n_blocks][m] matrices, each
+ *     row-major and contiguous, m = 2 for GELU (W1 [h,d], W2 [d,h]) and 3 for
+ *     SwiGLU (W1 gate [h,d], W2 up [h,d], W3 down [d,h]).  The static MLPs use
+ *     the same packing without the sequence dimension.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ttt_status {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1, /* null pointer, bad enum, negative size           */
+  TTT_ERR_SHAPE = 2,       /* T % b != 0, b < 1, sizes out of range           */
+  TTT_ERR_UNSUPPORTED = 3, /* d, hidden or vocab not a multiple of 16; no GPU  */
+  TTT_ERR_WORKSPACE = 4,   /* workspace pointer null or smaller than needed    */
+  TTT_ERR_TOKEN_RANGE = 5, /* device: a token outside [0, vocab)               */
+  TTT_ERR_NONFINITE = 6,   /* device: a chunk loss is NaN or infinite          */
+  TTT_ERR_TIMEOUT = 7,     /* device: a bounded wait ran out of iterations     */
+  TTT_ERR_CUDA = 8         /* a CUDA runtime call failed (see ttt_last_error)  */
+} ttt_status;
+
+enum { TTT_MLP_GELU = 0, TTT_MLP_SWIGLU = 1 };
+enum { TTT_PREC_FP32 = 0, TTT_PREC_BF16 = 1 };
+enum { TTT_REDUCE_MEAN = 0, TTT_REDUCE_SUM = 1 };
+
+/* Model shape.  d, hidden, vocab: multiples of 16, at least 16, and
+ * d <= 16384, hidden <= 65536, vocab < 2^26.  n_blocks in [1, 64].
+ * precision: TTT_PREC_FP32 = every contraction in float32 on CUDA cores;
+ * TTT_PREC_BF16 = contractions on tcgen05 tensor cores with bfloat16
+ * operands (round to nearest even) and float32 accumulation, while the
+ * state W, M, the residual stream, the softmax and all elementwise work stay
+ * float32.  rms_eps: the RMSNorm epsilon (z = g * h / sqrt(mean(h^2)+eps)).
+ * loss_reduction: the chunk objective.  TTT_REDUCE_MEAN (default reading):
+ * the mean next-token loss over the chunk, as in the first inner-loop sketch
+ * of [TTT-E2E] (F.cross_entropy with its default mean); the per-token loss in
+ * the recursion is l_t / b, so beta = 0, gamma = 1, eta = alpha is one SGD
+ * step on the chunk's mean loss and b = 1 is online SGD.  TTT_REDUCE_SUM:
+ * l_t itself (the second sketch's reduction='sum').  The reported chunk loss
+ * is the mean either way. */
+typedef struct ttt_config {
+  int32_t d;
+  int32_t hidden;
+  int32_t vocab;
+  int32_t n_blocks;
+  int32_t mlp;        /* TTT_MLP_GELU or TTT_MLP_SWIGLU */
+  int32_t has_static; /* 1: each block has a frozen static MLP before the dynamic one */
+  int32_t precision;  /* TTT_PREC_FP32 or TTT_PREC_BF16 */
+  int32_t loss_reduction; /* TTT_REDUCE_MEAN or TTT_REDUCE_SUM */
+  float rms_eps;
+} ttt_config;
+
+typedef struct ttt_handle ttt_handle;
+
+/* Create a handle on the current CUDA device and bind the frozen parameters
+ * ([TTT-E2E] 架构设计: frozen final norm and LM head; [Review] dual MLP).
+ *   lm_head  [vocab, d]  device float32 (E; logits = z E^T)
+ *   rms_gain [d]         device float32 (g)
+ *   static_w [n_blocks * m * hidden * d] device float32, packed as above, or
+ *            NULL when cfg->has_static == 0 (must be non-NULL otherwise).
+ * The handle copies (and for bf16 converts) these; the caller may free them
+ * after this call returns.  Synchronous.  *out is set only on TTT_OK. */
+ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* rms_gain,
+                      const float* static_w, ttt_handle** out);
+
+/* Release the handle and everything it owns (waits for its device work). */
+void ttt_destroy(ttt_handle* h);
+
+/* Bytes of device workspace ttt_prefill needs for (batch, T, b).  Host-only. */
+ttt_status ttt_workspace_size(const ttt_handle* h, int32_t batch, int32_t T, int32_t b,
+                              size_t* bytes);
+
+/* The inner loop over `batch` independent sequences of T tokens, chunk size b
+ * ([E2-TTT] Algorithm 1, applied chunk after chunk; [TTT-E2E] 内层循环).
+ *   hidden     [batch, T, d]  hidden rows entering the updated blocks
+ *   tokens     [batch, T]     int32, tokens[s,t] is the label of hidden row t
+ *                             (the caller pre-shifts; every chunk has b terms)
+ *   W          [batch * n_blocks * m * hidden * d]  in: W_0, out: final W
+ *   M          same shape                            in: M_0, out: final M
+ *   eta, beta, gamma [batch, T]  per-token learning rate, momentum, decay
+ *                             ([E2-TTT] 原始公式); any finite values accepted
+ *   chunk_loss [batch, T/b]   out: mean of the b token losses of each chunk,
+ *                             taken at that chunk's start weights
+ *   workspace  device scratch of at least ttt_workspace_size() bytes, 256-byte
+ *              aligned; its contents are not preserved
+ * W and M are updated in place.  T must be a multiple of b (TTT_ERR_SHAPE
+ * otherwise); T == 0 or batch == 0 is a no-op.  hidden, tokens and the
+ * scalars must not alias W, M, chunk_loss or the workspace. */
+ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
+                       const float* hidden, const int32_t* tokens, float* W, float* M,
+                       const float* eta, const float* beta, const float* gamma,
+                       float* chunk_loss, void* workspace, size_t ws_bytes, void* stream);
+
+/* The scalar kernels of Proposition 3.1 for every chunk, on the device
+ * ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1; computed in the division-free form
+ * K_W_t = eta_t sum_{j>=t} (prod_{i=t+1}^{j} beta_i) gtilde_j, float64 inside).
+ *   eta, beta, gamma [batch, T]  in
+ *   KW, KM [batch, T]            out: eta_t btilde_t R_t and eta_t btilde_t
+ *   consts [batch, T/b, 4]       out: (gtilde_0, btilde_0, btilde_0 R_1, 0)
+ * T % b == 0 required.  No handle needed; asynchronous on `stream`. */
+ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* eta,
+                              const float* beta, const float* gamma, float* KW, float* KM,
+                              float* consts, void* stream);
+
+/* Synchronise `stream`, return the first device-side error recorded by this
+ * handle's kernels since the last call (TTT_OK if none) and clear it. */
+ttt_status ttt_get_device_status(ttt_handle* h, void* stream);
+
+/* Self-test of the bounded-wait mechanism every spin loop in the library
+ * uses: launches one kernel that waits on a device flag nothing sets, giving
+ * up after `spin_limit` polls and recording TTT_ERR_TIMEOUT in the handle's
+ * status word.  No fault, no trap; the context stays usable. */
+ttt_status ttt_selftest_bounded_wait(ttt_handle* h, uint32_t spin_limit, void* stream);
+
+/* Static description of a status code. */
+const char* ttt_status_string(ttt_status s);
+
+/* Text of the last host-side error on this thread ("" if none). */
+const char* ttt_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_H_ */

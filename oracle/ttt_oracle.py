@@ -35,8 +35,13 @@ Pages cited by title:
 
 Readings where the pages leave a step open (each listed in the design doc):
   * tokens[t] is the label of hidden row t (the caller pre-shifts);
-  * the reported chunk loss is the mean of the b token losses at chunk-start
-    weights, while the update uses the per-token gradients (a sum);
+  * the chunk objective is the MEAN next-token loss over the chunk (the default
+    reduction of the first inner-loop sketch on [TTT-E2E]); the per-token loss
+    entering the recursion is therefore l_t / b, so that with beta = 0,
+    gamma = 1, eta_t = alpha one chunk is one mini-batch gradient step on the
+    chunk's mean loss, and b = 1 is plain online SGD.  reduction="sum" (the
+    second sketch's reduction='sum') uses l_t itself.  The reported chunk loss
+    is the mean of the b token losses at chunk-start weights either way;
   * RMSNorm: z = g * h / sqrt(mean(h^2) + eps), computed per row;
   * GELU is the exact erf form; SiLU(x) = x sigmoid(x);
   * the coefficients eta_t btilde_t R_t and btilde_0 R_1 are evaluated in the
@@ -313,16 +318,17 @@ def scalar_kernels_ratio_form(eta, beta, gamma):
 # Chunk update: closed form (Prop. 3.1 / Algorithm 1) and explicit recursion
 # ---------------------------------------------------------------------------
 
-def chunk_update_closed(W, M, grads, eta, beta, gamma):
+def chunk_update_closed(W, M, grads, eta, beta, gamma, gscale=1.0):
     """Algorithm 1 lines 2 and 4-7: aggregate with K_W and K_M, then
     W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + dW and M_C = btilde_0 M_0 + dM.
 
-    G_t = -outer(L[t], R[t]), so sum_t K_t G_t = -(K * L)^T R.
+    G_t = -gscale * outer(L[t], R[t]) (gscale = 1/b for the mean reduction),
+    so sum_t K_t G_t = -gscale (K * L)^T R.
     """
     KW, KM, g0, b0, cM = scalar_kernels(eta, beta, gamma)
     dt = W[0][0].dtype
-    KW = KW.astype(dt)
-    KM = KM.astype(dt)
+    KW = (KW * gscale).astype(dt)
+    KM = (KM * gscale).astype(dt)
     newW, newM = [], []
     for l in range(len(W)):
         bw, bm = [], []
@@ -337,7 +343,7 @@ def chunk_update_closed(W, M, grads, eta, beta, gamma):
     return newW, newM
 
 
-def chunk_update_explicit(W, M, grads, eta, beta, gamma):
+def chunk_update_explicit(W, M, grads, eta, beta, gamma, gscale=1.0):
     """The per-token recursion itself ([E2-TTT] 原始公式), with every G_t
     materialised:  M_t = beta_t M_{t-1} + eta_t G_t,  W_t = gamma_t W_{t-1} + M_t."""
     newW, newM = [], []
@@ -349,7 +355,7 @@ def chunk_update_explicit(W, M, grads, eta, beta, gamma):
             Wt = W[l][j].copy()
             Mt = M[l][j].copy()
             for k in range(C):
-                G = -np.outer(Lf[k], Rf[k])
+                G = -gscale * np.outer(Lf[k], Rf[k])
                 Mt = beta[k] * Mt + eta[k] * G
                 Wt = gamma[k] * Wt + Mt
             bw.append(Wt)
@@ -364,13 +370,18 @@ def chunk_update_explicit(W, M, grads, eta, beta, gamma):
 # ---------------------------------------------------------------------------
 
 def prefill_sequence(model: Model, W0, M0, hidden, tokens, eta, beta, gamma, b,
-                     update: str = "closed", n_chunks: Optional[int] = None):
+                     update: str = "closed", n_chunks: Optional[int] = None,
+                     reduction: str = "mean"):
     """Chunk-serial inner loop for one sequence.
 
     W0, M0: nested lists [n_blocks][m] of matrices; hidden [T, d]; tokens [T];
     eta/beta/gamma [T].  Returns (W_final, M_final, chunk_loss [n_chunks]).
     ``n_chunks`` limits the run to the first chunks (for sampled parity).
+    ``reduction``: "mean" (per-token loss l_t / b) or "sum" (l_t).
     """
+    if reduction not in ("mean", "sum"):
+        raise ValueError("reduction must be 'mean' or 'sum'")
+    gscale = 1.0 / b if reduction == "mean" else 1.0
     T = hidden.shape[0]
     if T % b != 0:
         raise ValueError("T must be a multiple of b")
@@ -386,12 +397,13 @@ def prefill_sequence(model: Model, W0, M0, hidden, tokens, eta, beta, gamma, b,
         loss, fwd = chunk_forward(model, W, X, y)     # line 1: at chunk-start weights
         losses[c] = float(np.mean(loss))
         grads = chunk_backward(model, W, y, fwd)      # line 3: single backward
-        W, M = step(W, M, grads, eta[s], beta[s], gamma[s])
+        W, M = step(W, M, grads, eta[s], beta[s], gamma[s], gscale)
     return W, M, losses
 
 
 def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
-            dtype=np.float64, update: str = "closed", n_chunks: Optional[int] = None):
+            dtype=np.float64, update: str = "closed", n_chunks: Optional[int] = None,
+            reduction: str = "mean"):
     """Batched inner loop with the C-ABI's flat layouts.
 
     hidden [B,T,d], tokens [B,T], eta/beta/gamma [B,T],
@@ -410,7 +422,7 @@ def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
         M0 = unpack_blocks(M0_flat[s].copy(), mdl.n_blocks, shapes)
         W, M, L = prefill_sequence(mdl, W0, M0, np.asarray(hidden[s], dtype=dtype),
                                    np.asarray(tokens[s]), eta[s], beta[s], gamma[s], b,
-                                   update=update, n_chunks=n_chunks)
+                                   update=update, n_chunks=n_chunks, reduction=reduction)
         Ws.append(pack_blocks(W))
         Ms.append(pack_blocks(M))
         Ls.append(L)

@@ -1,0 +1,275 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same
+seeded inputs.  Tolerances: relative Frobenius error on final W and M <= 1e-4
+(fp32 mode) or 3e-2 (bf16 mode); per-chunk mean loss within 1e-2 absolute."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from tests import helpers as H
+from weight_long_context_b200 import inputs as I
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def W(name, **kw):
+    return I.WORKLOADS[name].with_(**kw)
+
+
+# ---------------------------------------------------------------------------
+# K1 scalar scan alone
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b,kind", [(1, "e2ttt"), (16, "sgd"), (64, "e2ttt"), (100, "mixed"),
+                                    (1024, "e2ttt"), (1024, "sgd"), (4096, "e2ttt")])
+def test_scalar_scan_matches_oracle(dev, b, kind):
+    import oracle
+    from weight_long_context_b200 import ttt
+    rng = np.random.default_rng(b)
+    B, nc = 3, 4
+    T = b * nc
+    eta = (0.01 / (1 + np.exp(-rng.normal(size=(B, T))))).astype(np.float32)
+    if kind == "sgd":
+        beta = np.zeros((B, T), np.float32)
+        gamma = np.ones((B, T), np.float32)
+    else:
+        beta = rng.uniform(0.8, 0.99, (B, T)).astype(np.float32)
+        gamma = rng.uniform(0.99, 1.0, (B, T)).astype(np.float32)
+        if kind == "mixed":
+            beta[:, ::7] = 0.0
+            gamma[:, ::11] = 1.0
+    t = lambda a: torch.from_numpy(a).to(dev)
+    KW, KM, consts = ttt.ttt_scalar_kernels(t(eta), t(beta), t(gamma), b)
+    KW, KM, consts = KW.cpu().numpy(), KM.cpu().numpy(), consts.cpu().numpy()
+    for s in range(B):
+        for c in range(nc):
+            sl = slice(c * b, (c + 1) * b)
+            kw, km, g0, b0, cM = oracle.scalar_kernels(eta[s, sl], beta[s, sl], gamma[s, sl])
+            np.testing.assert_allclose(KW[s, sl], kw, rtol=2e-6, atol=1e-30)
+            np.testing.assert_allclose(KM[s, sl], km, rtol=2e-6, atol=1e-30)
+            np.testing.assert_allclose(consts[s, c, :3], [g0, b0, cM], rtol=2e-6, atol=1e-30)
+
+
+# ---------------------------------------------------------------------------
+# Small ragged shapes: several tiles and a ragged tail in every dimension
+# ---------------------------------------------------------------------------
+
+RAGGED = [
+    # name, d, h, V, L, mlp, static, T, b, batch
+    ("gelu_1blk", 80, 208, 528, 1, "gelu", False, 72, 24, 2),
+    ("swiglu_2blk_static", 48, 80, 272, 2, "swiglu", True, 60, 20, 2),
+    ("gelu_3blk_static", 64, 96, 400, 3, "gelu", True, 48, 16, 1),
+    ("swiglu_tile_tail", 208, 336, 1040, 1, "swiglu", False, 272, 136, 2),
+]
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("case", RAGGED, ids=[c[0] for c in RAGGED])
+def test_ragged_parity(dev, case, precision):
+    name, d, h, V, L, mlp, st, T, b, B = case
+    w = I.Workload(name, d, h, V, L, mlp, st, precision, T, b, B, "e2ttt")
+    x = I.make_inputs(w, seed=5, m0_scale=0.01, w0_per_sequence=True)
+    gpu = H.run_gpu(w, x, dev)
+    ref = H.run_oracle(w, x)
+    e = H.compare(w, x, gpu, ref)
+    print(name, precision, e)
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+def test_online_sgd_b1(dev, precision):
+    """b = 1, beta = 0, gamma = 1: online SGD, one token per chunk."""
+    w = I.Workload("b1", 32, 48, 64, 2, "gelu", True, precision, 12, 1, 2, "sgd", 0.05, "uniform")
+    x = I.make_inputs(w, seed=3)
+    H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x))
+
+
+# ---------------------------------------------------------------------------
+# The five workloads
+# ---------------------------------------------------------------------------
+
+def test_tiny_sgd_full(dev):
+    w = W("tiny_sgd")
+    x = I.make_inputs(w, seed=0)
+    e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x))
+    print("tiny_sgd", e)
+
+
+def test_e2ttt_block_full(dev):
+    w = W("e2ttt_block")
+    x = I.make_inputs(w, seed=0)
+    e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x, dtype=np.float32))
+    print("e2ttt_block", e)
+
+
+@pytest.mark.parametrize("name", ["sgd_3b", "stack_128k", "batched_16"])
+def test_full_dims_first_chunks(dev, name):
+    """Full model sizes and chunk size (the launch configuration the benchmark
+    times), first two chunks, element by element against the oracle."""
+    w = W(name)
+    w = w.with_(T=2 * w.b, batch=min(w.batch, 4))
+    x = I.make_inputs(w, seed=0, m0_scale=1e-3 if w.scalars == "e2ttt" else 0.0)
+    e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x, dtype=np.float32))
+    print(name, e)
+
+
+@pytest.mark.parametrize("name", ["sgd_3b", "stack_128k", "batched_16"])
+def test_full_length_sampled(dev, name):
+    """Full-length run at the benchmark's sizes vs stored oracle samples
+    (tests/golden/<name>_seed0.json, written by tests/golden/make_golden.py)."""
+    path = os.path.join(GOLDEN, f"{name}_seed0.json")
+    if not os.path.exists(path):
+        pytest.skip("golden file not generated")
+    try:
+        g = json.load(open(path))
+    except ValueError:
+        pytest.skip("golden file incomplete")
+    w = W(name)
+    x = I.make_inputs(w, seed=0)
+    Wg, Mg, Lg, st = H.run_gpu(w, x, dev)
+    assert st == 0
+    idx = np.asarray(g["sample_index"])
+    tol = H.TOL_STATE[w.precision]
+    eW = H.rel_fro(Wg[idx], np.asarray(g["W"]))
+    assert eW <= tol, eW
+    Mr = np.asarray(g["M"])
+    if np.any(Mr):
+        assert H.rel_fro(Mg[idx], Mr) <= tol
+    eL = float(np.max(np.abs(Lg - np.asarray(g["chunk_loss"]))))
+    assert eL <= H.TOL_LOSS, eL
+    print(name, "W", eW, "loss", eL)
+
+
+# ---------------------------------------------------------------------------
+# Properties that hold at any size
+# ---------------------------------------------------------------------------
+
+def test_resume_and_determinism_bitwise(dev):
+    """Chunk-end state is the only carried state: prefill(T) equals
+    prefill(T1) then prefill(T - T1) bit for bit, and reruns are identical."""
+    w = W("e2ttt_block", T=1024)
+    x = I.make_inputs(w, seed=2, m0_scale=1e-3)
+    Wa, Ma, La, _ = H.run_gpu(w, x, dev)
+    Wb, Mb, Lb, _ = H.run_gpu(w, x, dev)
+    assert np.array_equal(Wa, Wb) and np.array_equal(Ma, Mb) and np.array_equal(La, Lb)
+    T1 = 512
+    x1 = dict(x, hidden=x["hidden"][:, :T1], tokens=x["tokens"][:, :T1], eta=x["eta"][:, :T1],
+              beta=x["beta"][:, :T1], gamma=x["gamma"][:, :T1])
+    W1, M1, L1, _ = H.run_gpu(w.with_(T=T1), x1, dev)
+    x2 = dict(x, hidden=x["hidden"][:, T1:], tokens=x["tokens"][:, T1:], eta=x["eta"][:, T1:],
+              beta=x["beta"][:, T1:], gamma=x["gamma"][:, T1:], W0=W1, M0=M1)
+    W2, M2, L2, _ = H.run_gpu(w.with_(T=T1), x2, dev)
+    assert np.array_equal(W2, Wa) and np.array_equal(M2, Ma)
+    assert np.array_equal(np.concatenate([L1, L2], axis=1), La)
+
+
+def test_zero_head_gives_log_v(dev):
+    w = I.Workload("zh", 64, 96, 160, 1, "swiglu", False, "bf16", 64, 32, 1, "e2ttt")
+    x = I.make_inputs(w, seed=1, m0_scale=0.01)
+    x["lm_head"] = np.zeros_like(x["lm_head"])
+    Wg, Mg, Lg, st = H.run_gpu(w, x, dev)
+    np.testing.assert_allclose(Lg, np.log(160.0), rtol=1e-6)
+    Wr, Mr, _ = H.run_oracle(w, x)
+    assert H.rel_fro(Wg, Wr) < 1e-6 and H.rel_fro(Mg, Mr) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# Edge cases and errors
+# ---------------------------------------------------------------------------
+
+def test_empty_calls_are_noops(dev):
+    from weight_long_context_b200 import ttt
+    w = I.Workload("e", 32, 32, 32, 1, "gelu", False, "fp32", 16, 8, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    h = H.make_handle(w, x, dev)
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    W0 = t(x["W0"])
+    Wc = W0.clone()
+    empty = torch.empty((1, 0, 32), device=dev)
+    e2 = torch.empty((1, 0), device=dev)
+    h.prefill(empty, e2.to(torch.int32), Wc, t(x["M0"]), e2, e2, e2, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(Wc, W0)
+    assert h.device_status() == 0
+    h.close()
+
+
+def test_shape_and_argument_errors(dev):
+    from weight_long_context_b200 import ttt
+    w = I.Workload("e", 32, 32, 32, 1, "gelu", False, "fp32", 16, 8, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    h = H.make_handle(w, x, dev)
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    args = [t(x["hidden"]), t(x["tokens"], torch.int32), t(x["W0"]), t(x["M0"]), t(x["eta"]),
+            t(x["beta"]), t(x["gamma"])]
+    with pytest.raises(ttt.TTTError) as ei:
+        h.prefill(*args, b=5)           # T % b != 0
+    assert ei.value.code == 2
+    with pytest.raises(ttt.TTTError) as ei:
+        h.prefill(*args, b=0)
+    assert ei.value.code == 2
+    assert ttt.ttt_workspace_size(h._h, 1, 16, 8) > 0
+    # unsupported model shape
+    cfg = ttt.ttt_config(30, 32, 32, 1, 0, 0, 0, 0, 1e-6)
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_create(cfg, args[0], args[0], None)
+    assert ei.value.code == 3
+    h.close()
+
+
+def test_workspace_too_small(dev):
+    import ctypes
+    from weight_long_context_b200 import ttt
+    w = I.Workload("e", 32, 32, 32, 1, "gelu", False, "fp32", 16, 8, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    h = H.make_handle(w, x, dev)
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    loss = torch.empty((1, 2), device=dev)
+    p = lambda a: ctypes.c_void_p(a.data_ptr())
+    args = [t(x["hidden"]), t(x["tokens"], torch.int32), t(x["W0"]), t(x["M0"]), t(x["eta"]),
+            t(x["beta"]), t(x["gamma"])]
+    code = ttt.load_library().ttt_prefill(h._h, 1, 16, 8, *[p(a) for a in args], p(loss), p(ws), 256,
+                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert code == 4
+    h.close()
+
+
+def test_bad_token_sets_device_status(dev):
+    w = I.Workload("tok", 32, 32, 64, 1, "gelu", False, "bf16", 32, 16, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    x["tokens"][0, 5] = 64            # == V: outside [0, V)
+    *_, st = H.run_gpu(w, x, dev)
+    assert st == 5
+
+
+def test_nonfinite_hidden_sets_device_status(dev):
+    w = I.Workload("nan", 32, 32, 64, 1, "gelu", False, "fp32", 32, 16, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    x["hidden"][0, 3, :] = np.nan
+    *_, st = H.run_gpu(w, x, dev)
+    assert st == 6
+
+
+def test_bounded_wait_times_out_cleanly(dev):
+    """A wait on a flag nothing sets gives up after its limit and reports
+    TTT_ERR_TIMEOUT; the context stays usable afterwards."""
+    w = I.Workload("e", 32, 32, 32, 1, "gelu", False, "fp32", 16, 8, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    h = H.make_handle(w, x, dev)
+    h.selftest_bounded_wait(1000)
+    assert h.device_status() == 7
+    assert h.device_status() == 0
+    # still usable
+    Wg, Mg, Lg, st = H.run_gpu(w, x, dev, handle=h)
+    assert st == 0 and np.all(np.isfinite(Wg))
+    h.close()

@@ -44,12 +44,12 @@ def tiny_setup(kind="gelu", d=4, h=6, V=7, L=2, static=True, T=12, seed=1,
                 W0=W0, M0=M0, X=X, y=y, eta=eta, beta=beta, gamma=gamma)
 
 
-def run_prefill(s, b, update="closed", **over):
+def run_prefill(s, b, update="closed", reduction="mean", **over):
     p = dict(s)
     p.update(over)
     W, M, Ls = O.prefill(p["model"], p["W0"], p["M0"], p["X"][None], p["y"][None],
                          p["eta"][None], p["beta"][None], p["gamma"][None], b,
-                         update=update)
+                         update=update, reduction=reduction)
     return W, M, Ls[0]
 
 
@@ -162,11 +162,12 @@ def test_scalar_kernels_underflow_finite():
 # 2. Closed form == explicit per-token recursion on the full model
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("kind,static", [("gelu", False), ("gelu", True), ("swiglu", True), ("swiglu", False)])
-def test_closed_form_equals_recursion(kind, static):
+@pytest.mark.parametrize("kind,static,red", [("gelu", False, "mean"), ("gelu", True, "sum"),
+                                             ("swiglu", True, "mean"), ("swiglu", False, "sum")])
+def test_closed_form_equals_recursion(kind, static, red):
     s = tiny_setup(kind=kind, static=static, h=6 if kind == "gelu" else 5, T=12)
-    W1, M1, L1 = run_prefill(s, 4, "closed")
-    W2, M2, L2 = run_prefill(s, 4, "explicit")
+    W1, M1, L1 = run_prefill(s, 4, "closed", reduction=red)
+    W2, M2, L2 = run_prefill(s, 4, "explicit", reduction=red)
     assert rel(W1, W2) < 1e-12
     assert rel(M1, M2) < 1e-12
     np.testing.assert_allclose(L1, L2, rtol=1e-13)
@@ -228,18 +229,22 @@ def test_b1_sgd_is_online_sgd(kind):
     np.testing.assert_allclose(Ls, ref_losses, rtol=1e-12)
 
 
-def test_chunked_sgd_uses_chunk_start_gradients():
-    """b = 4 SGD: W_C = W_0 - alpha sum_t grad l_t(W_0) and M_C = eta_C G_C
-    (only the last token's gradient survives when beta = 0)."""
+@pytest.mark.parametrize("red", ["mean", "sum"])
+def test_chunked_sgd_uses_chunk_start_gradients(red):
+    """b = 4 SGD: one mini-batch step at the chunk-start weights,
+    W_C = W_0 - alpha grad (mean_t l_t)(W_0) (reduction "mean"; the sum for
+    "sum"), and M_C = eta_C G_C (only the last token survives when beta = 0)."""
     s = tiny_setup(kind="gelu", d=5, h=7, V=9, L=1, static=False, T=4, scalars="sgd", m0=0.3)
-    W, M, Ls = run_prefill(s, 4)
+    W, M, Ls = run_prefill(s, 4, reduction=red)
     T_ = lambda a: torch.tensor(a, dtype=torch.float64)
     Wv = T_(s["W0"]).requires_grad_(True)
     l = AM.losses("gelu", 5, 7, 1, 1e-6, T_(s["E"]), T_(s["g"]), None, Wv, T_(s["X"]), torch.tensor(s["y"]))
-    (gsum,) = torch.autograd.grad(l.sum(), Wv, retain_graph=True)
+    obj = l.mean() if red == "mean" else l.sum()
+    (gobj,) = torch.autograd.grad(obj, Wv, retain_graph=True)
     (glast,) = torch.autograd.grad(l[3], Wv)
-    assert rel(W, (T_(s["W0"]) - 0.1 * gsum).numpy()) < 1e-12
-    assert rel(M, (-0.1 * glast).numpy()) < 1e-12
+    scale = 0.25 if red == "mean" else 1.0
+    assert rel(W, (T_(s["W0"]) - 0.1 * gobj).numpy()) < 1e-12
+    assert rel(M, (-0.1 * scale * glast).numpy()) < 1e-12
     assert Ls[0] == pytest.approx(float(l.mean()), rel=1e-12)
 
 
@@ -337,11 +342,11 @@ def test_planted_mistakes_are_caught(monkeypatch):
     # (a) wrong sign of G in the aggregation
     orig = O.chunk_update_closed
 
-    def flipped(W, M, grads, eta, beta, gamma):
+    def flipped(W, M, grads, eta, beta, gamma, gscale=1.0):
         g2 = [[(-Lf, Rf) for (Lf, Rf) in blk] for blk in grads]
-        return orig(W, M, g2, eta, beta, gamma)
+        return orig(W, M, g2, eta, beta, gamma, gscale)
     monkeypatch.setattr(O, "chunk_update_closed", flipped)
-    _must_fail(test_chunked_sgd_uses_chunk_start_gradients)
+    _must_fail(test_chunked_sgd_uses_chunk_start_gradients, "mean")
     monkeypatch.setattr(O, "chunk_update_closed", orig)
 
     # (b) dropped momentum carry c_M in W_C
@@ -351,7 +356,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
         KW, KM, g0, b0, cM = orig_sk(eta, beta, gamma)
         return KW, KM, g0, b0, 0.0
     monkeypatch.setattr(O, "scalar_kernels", no_cm)
-    _must_fail(test_closed_form_equals_recursion, "gelu", True)
+    _must_fail(test_closed_form_equals_recursion, "gelu", True, "mean")
     monkeypatch.setattr(O, "scalar_kernels", orig_sk)
 
     # (c) off-by-one suffix product (btilde_{t-1} instead of btilde_t)

@@ -1,0 +1,58 @@
+// Shared host/device helpers for libttt (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/ttt.h"
+
+namespace ttt {
+
+// ----------------------------------------------------------------------------
+// Element types of the GEMM operands: float (fp32 mode) or bfloat16 (bf16 mode)
+// ----------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// ----------------------------------------------------------------------------
+// Device status word: first error wins (TTT_OK = 0 means none yet).
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// SwiGLU layout of the fused [gate; up] dimension inside the library:
+// 32-wide groups, gate columns j in [16g, 16g+16) at positions [32g, 32g+16),
+// up columns at [32g+16, 32g+32).  h must be a multiple of 16.
+__host__ __device__ __forceinline__ int swiglu_pos_gate(int j) { return ((j >> 4) << 5) + (j & 15); }
+__host__ __device__ __forceinline__ int swiglu_pos_up(int j) { return ((j >> 4) << 5) + 16 + (j & 15); }
+// Inverse: position p in [0, 2h) -> row of the packed [W1; W2] (W1 rows 0..h-1, W2 rows h..2h-1).
+__host__ __device__ __forceinline__ int swiglu_row_of_pos(int p, int h) {
+  int g = p >> 5, k = p & 31;
+  return k < 16 ? (g << 4) + k : h + (g << 4) + (k - 16);
+}
+
+}  // namespace ttt
+
+#define TTT_CUDA_TRY(expr)                                             \
+  do {                                                                 \
+    cudaError_t _e = (expr);                                           \
+    if (_e != cudaSuccess) {                                           \
+      ::ttt::set_last_error(#expr, cudaGetErrorString(_e), __FILE__, __LINE__); \
+      return TTT_ERR_CUDA;                                             \
+    }                                                                  \
+  } while (0)
+
+namespace ttt {
+void set_last_error(const char* what, const char* why, const char* file, int line);
+void set_last_error_msg(const char* msg);
+}  // namespace ttt

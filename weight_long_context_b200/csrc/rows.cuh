@@ -1,0 +1,203 @@
+// Row-wise kernels of the chunk step: gather of the chunk's hidden rows,
+// RMSNorm forward/backward, the cross-entropy reduction, operand casts, and
+// the bounded-wait primitive.  All are bandwidth-bound, one warp per row with
+// 16-byte accesses where the layout allows.
+#pragma once
+
+#include "common.cuh"
+#include "epilogue.cuh"
+
+namespace ttt {
+
+// ---------------------------------------------------------------------------
+// Gather chunk c of every sequence: resid[s*b + i] = hidden[s, c*b + i] and
+// its operand copy.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void gather_chunk_kernel(const float* __restrict__ hidden, int T_, int b, int chunk, int d,
+                                    int64_t n, float* __restrict__ resid, T* __restrict__ act) {
+  const int64_t q = d >> 2;  // float4 per row (d % 16 == 0)
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * q;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    int64_t r = e / q, c4 = e - r * q;
+    int64_t s = r / b, i = r - s * b;
+    const float4 x = reinterpret_cast<const float4*>(hidden + ((s * T_ + (int64_t)chunk * b + i) * d))[c4];
+    reinterpret_cast<float4*>(resid + r * d)[c4] = x;
+    T* a = act + r * d + c4 * 4;
+    a[0] = from_f<T>(x.x); a[1] = from_f<T>(x.y); a[2] = from_f<T>(x.z); a[3] = from_f<T>(x.w);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm forward: z = g * h / sqrt(mean(h^2) + eps); keeps 1/rms for backward.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ h, const float* __restrict__ g, float eps,
+                                   int64_t n, int d, T* __restrict__ z, float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const float4* hr = reinterpret_cast<const float4*>(h + row * d);
+  float ss = 0.f;
+  for (int c = lane; c < (d >> 2); c += 32) {
+    float4 x = hr[c];
+    ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss / (float)d + eps);
+  if (lane == 0) rstd[row] = r;
+  T* zr = z + row * d;
+  const float4* gr = reinterpret_cast<const float4*>(g);
+  for (int c = lane; c < (d >> 2); c += 32) {
+    float4 x = hr[c], gg = gr[c];
+    zr[4 * c + 0] = from_f<T>(x.x * r * gg.x);
+    zr[4 * c + 1] = from_f<T>(x.y * r * gg.y);
+    zr[4 * c + 2] = from_f<T>(x.z * r * gg.z);
+    zr[4 * c + 3] = from_f<T>(x.w * r * gg.w);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm backward: dh = r * (g*dz) - h * r^3 * <g*dz, h> / d.
+// Writes the gradient of the residual stream (fp32), its operand copy, and,
+// when the top MLP is dynamic, the K-scaled negated copies.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dz, const float* __restrict__ h,
+                                   const float* __restrict__ rstd, const float* __restrict__ g,
+                                   int64_t n, int d, float* __restrict__ dout, T* __restrict__ dout_a,
+                                   T* __restrict__ doutW, T* __restrict__ doutM,
+                                   const float* __restrict__ KW, const float* __restrict__ KM, float kscale,
+                                   TokenMap tm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= n) return;
+  const float4* dzr = reinterpret_cast<const float4*>(dz + row * d);
+  const float4* hr = reinterpret_cast<const float4*>(h + row * d);
+  const float4* gr = reinterpret_cast<const float4*>(g);
+  float dot = 0.f;
+  for (int c = lane; c < (d >> 2); c += 32) {
+    float4 a = dzr[c], x = hr[c], gg = gr[c];
+    dot += a.x * gg.x * x.x + a.y * gg.y * x.y + a.z * gg.z * x.z + a.w * gg.w * x.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  const float r = rstd[row];
+  const float coef = r * r * r * dot / (float)d;
+  float kw = 0.f, km = 0.f;
+  if (doutW) {
+    int64_t ti = tm.index((int)row);
+    kw = -KW[ti] * kscale;
+    km = -KM[ti] * kscale;
+  }
+  for (int c = lane; c < (d >> 2); c += 32) {
+    float4 a = dzr[c], x = hr[c], gg = gr[c];
+    float o4[4] = {r * a.x * gg.x - x.x * coef, r * a.y * gg.y - x.y * coef,
+                   r * a.z * gg.z - x.z * coef, r * a.w * gg.w - x.w * coef};
+    reinterpret_cast<float4*>(dout + row * d)[c] = make_float4(o4[0], o4[1], o4[2], o4[3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int64_t idx = row * d + 4 * c + j;
+      dout_a[idx] = from_f<T>(o4[j]);
+      if (doutW) { doutW[idx] = from_f<T>(kw * o4[j]); doutM[idx] = from_f<T>(km * o4[j]); }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Cross-entropy reduction: one block per sequence.  Combines each row's
+// per-tile (max, sum exp) partials into lse, forms l_t = lse - logit[y_t],
+// and writes the chunk's mean loss.  Fixed thread-to-row mapping and a fixed
+// reduction tree: the result does not depend on scheduling.
+// ---------------------------------------------------------------------------
+__global__ void ce_reduce_kernel(const float* __restrict__ part, const float* __restrict__ tgt, int ntn,
+                                 const int* __restrict__ tokens, TokenMap tm, int V,
+                                 float* __restrict__ lse, float* __restrict__ chunk_loss, int nchunks,
+                                 int* status) {
+  __shared__ float red[32];
+  const int s = blockIdx.x;
+  const int b = tm.b;
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < b; i += blockDim.x) {
+    int r = s * b + i;
+    const float* p = part + (int64_t)r * ntn * 2;
+    float m = -INFINITY;
+    for (int t = 0; t < ntn; ++t) m = fmaxf(m, p[2 * t]);
+    float sum = 0.f;
+    for (int t = 0; t < ntn; ++t) sum += p[2 * t + 1] * expf(p[2 * t] - m);
+    float l = m + logf(sum);
+    lse[r] = l;
+    int y = tokens[tm.index(r)];
+    if (y < 0 || y >= V) {
+      record_error(status, TTT_ERR_TOKEN_RANGE);
+      continue;
+    }
+    acc += l - tgt[r];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int nw = blockDim.x >> 5;
+    float v = threadIdx.x < nw ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) {
+      float mean = v / (float)b;
+      chunk_loss[(int64_t)s * nchunks + tm.chunk] = mean;
+      if (!isfinite(mean)) record_error(status, TTT_ERR_NONFINITE);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Operand shadow of packed fast weights (or static weights): a cast to the
+// operand type, with the SwiGLU [W1; W2] rows placed in the interleaved
+// library order.  count = number of blocks (sequences x n_blocks).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void build_shadow_kernel(const float* __restrict__ W, T* __restrict__ sh, int64_t count,
+                                    int h, int d, int swiglu) {
+  const int64_t blk = (swiglu ? 3 : 2) * (int64_t)h * d;
+  const int64_t total = count * blk;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    int64_t o = e % blk, base = e - o;
+    int64_t src = e;
+    if (swiglu && o < 2 * (int64_t)h * d) {
+      int p = (int)(o / d);
+      int64_t c = o - (int64_t)p * d;
+      src = base + (int64_t)swiglu_row_of_pos(p, h) * d + c;
+    }
+    sh[e] = from_f<T>(W[src]);
+  }
+}
+
+template <typename T>
+__global__ void cast_kernel(const float* __restrict__ x, T* __restrict__ y, int64_t n) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x)
+    y[e] = from_f<T>(x[e]);
+}
+
+// ---------------------------------------------------------------------------
+// Bounded wait: poll a device flag at most `limit` times.  Returns true if
+// the flag became nonzero; otherwise records TTT_ERR_TIMEOUT and returns
+// false.  Every spin loop in the library has such a limit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool bounded_wait_flag(const volatile int* flag, uint32_t limit, int* status) {
+  for (uint32_t i = 0; i < limit; ++i) {
+    if (*flag != 0) return true;
+    __nanosleep(64);
+  }
+  record_error(status, TTT_ERR_TIMEOUT);
+  return false;
+}
+
+__global__ void selftest_wait_kernel(const int* flag, uint32_t limit, int* status) {
+  if (threadIdx.x == 0) bounded_wait_flag(flag, limit, status);
+}
+
+}  // namespace ttt

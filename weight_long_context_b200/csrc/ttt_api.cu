@@ -1,0 +1,552 @@
+// libttt: C ABI, argument validation, workspace plan and the chunk-serial
+// driver of the TTT inner loop ("Rethinking Expressivity and Efficiency in
+// Test-Time Training", Algorithm 1, applied chunk after chunk as the
+// "TTT-E2E：端到端测试时训练的长上下文语言建模" inner loop describes).
+//
+// One prefill call = K1 scan over all chunks, the operand shadow of W, then
+// per chunk (strictly serial: chunk r's gradients need chunk r-1's state):
+//   gather -> [static F1, F2] / dynamic F1, F2 per block -> RMSNorm ->
+//   CE pass A (logit tiles -> online-softmax partials) -> CE reduce ->
+//   per vocabulary slab: CE pass B (softmax - onehot) and dz += P E_slab ->
+//   RMSNorm backward -> per MLP, top down: B1 (dA, dU), B2 (dX) when a
+//   dynamic MLP lies below, and for dynamic MLPs the dual-accumulator
+//   aggregation whose epilogue writes W, M and the operand shadow in place.
+// The whole sequence of launches is captured once into a CUDA graph on a
+// private stream and replayed on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <type_traits>
+#include <vector>
+
+#include "common.cuh"
+#include "epilogue.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "rows.cuh"
+#include "scan.cuh"
+
+namespace ttt {
+
+static thread_local std::string g_last_error;
+
+void set_last_error(const char* what, const char* why, const char* file, int line) {
+  char buf[512];
+  snprintf(buf, sizeof(buf), "%s failed: %s (%s:%d)", what, why, file, line);
+  g_last_error = buf;
+}
+void set_last_error_msg(const char* msg) { g_last_error = msg; }
+
+static ttt_status fail(ttt_status s, const char* msg) {
+  g_last_error = msg;
+  return s;
+}
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------------------
+// Handle
+// ---------------------------------------------------------------------------
+struct GraphKey {
+  int batch, T, b;
+  const void *hidden, *tokens, *W, *M, *eta, *beta, *gamma, *loss, *ws;
+  size_t ws_bytes;
+  bool operator==(const GraphKey& o) const {
+    return batch == o.batch && T == o.T && b == o.b && hidden == o.hidden && tokens == o.tokens &&
+           W == o.W && M == o.M && eta == o.eta && beta == o.beta && gamma == o.gamma &&
+           loss == o.loss && ws == o.ws && ws_bytes == o.ws_bytes;
+  }
+};
+
+}  // namespace ttt
+
+struct ttt_handle {
+  ttt_config cfg;
+  int device = 0;
+  void* E = nullptr;        // [V, d] operand copy
+  float* gain = nullptr;    // [d]
+  void* S = nullptr;        // static shadow [n_blocks][m*h*d] or nullptr
+  int* status = nullptr;    // device status word
+  int* zero_flag = nullptr; // a device int that stays 0 (bounded-wait self-test)
+  cudaStream_t cap = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  ttt::GraphKey key;
+  bool have_key = false;
+  bool use_graph = true;
+};
+
+namespace ttt {
+
+// ---------------------------------------------------------------------------
+// Workspace plan
+// ---------------------------------------------------------------------------
+struct Plan {
+  int B, T, b, nchunks, n, d, h, H2, V, L, m, nM, Vs, nslabs, ntn;
+  float kscale;  // 1/b for the mean reduction, 1 for the sum
+  bool swiglu, has_static;
+  size_t esz;  // operand element size
+  size_t KW, KM, consts, Wsh, resid, actin, act, fac, z, rstd, part, tgt, lse, P, dz, dout, dout_a,
+      doutW[2], doutM[2], dU, dUW, dUM, total;
+};
+
+static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static int head_tile_n(int precision) { return precision == TTT_PREC_FP32 ? simt::BN : tc::HEAD_BN; }
+
+static Plan make_plan(const ttt_config& c, int B, int T, int b) {
+  Plan p{};
+  p.B = B; p.T = T; p.b = b; p.nchunks = b > 0 ? T / b : 0; p.n = B * b;
+  p.d = c.d; p.h = c.hidden; p.V = c.vocab; p.L = c.n_blocks;
+  p.swiglu = c.mlp == TTT_MLP_SWIGLU; p.has_static = c.has_static != 0;
+  p.m = p.swiglu ? 3 : 2; p.H2 = p.swiglu ? 2 * p.h : p.h;
+  p.nM = p.L * (p.has_static ? 2 : 1);
+  p.esz = c.precision == TTT_PREC_FP32 ? 4 : 2;
+  p.kscale = (c.loss_reduction == TTT_REDUCE_MEAN && b > 0) ? 1.0f / (float)b : 1.0f;
+  p.ntn = (p.V + head_tile_n(c.precision) - 1) / head_tile_n(c.precision);
+  // vocabulary slab: the [n, Vs] slab of dl/dlogits is the only per-vocabulary
+  // buffer; capped at 32 MiB so it stays resident in L2.
+  const size_t cap = 32ull << 20;
+  int64_t vs = (int64_t)(cap / ((size_t)p.n * p.esz));
+  vs = vs / 256 * 256;
+  if (vs < 256) vs = 256;
+  if (vs >= p.V) vs = p.V;
+  p.Vs = (int)vs;
+  p.nslabs = (p.V + p.Vs - 1) / p.Vs;
+
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  const size_t n = p.n, d = p.d, h = p.h, H2 = p.H2, e = p.esz;
+  p.KW = take(4ull * B * T);
+  p.KM = take(4ull * B * T);
+  p.consts = take(16ull * B * p.nchunks);
+  p.Wsh = take(e * B * p.L * p.m * h * d);
+  p.resid = take(4 * n * d);
+  p.actin = take(e * p.nM * n * d);
+  p.act = take(e * p.nM * n * h);
+  p.fac = take(e * p.nM * n * H2);
+  p.z = take(e * n * d);
+  p.rstd = take(4 * n);
+  p.part = take(8 * n * p.ntn);
+  p.tgt = take(4 * n);
+  p.lse = take(4 * n);
+  p.P = take(e * n * p.Vs);
+  p.dz = take(4 * n * d);
+  p.dout = take(4 * n * d);
+  p.dout_a = take(e * n * d);
+  for (int i = 0; i < 2; ++i) { p.doutW[i] = take(e * n * d); p.doutM[i] = take(e * n * d); }
+  p.dU = take(e * n * H2);
+  p.dUW = take(e * n * H2);
+  p.dUM = take(e * n * H2);
+  p.total = off;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM dispatch by operand type: fp32 -> CUDA-core engine, bf16 -> tcgen05.
+// ---------------------------------------------------------------------------
+template <typename T, int NACC, class Epi>
+static cudaError_t gemm(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B,
+                        const Epi& epi, cudaStream_t st, int* status) {
+  if constexpr (std::is_same<T, float>::value) {
+    (void)status;
+    return launch_gemm_simt<T, NACC, Epi>(s, A, A2, B, epi, st);
+  } else {
+    return tc::launch_gemm_tc<NACC, Epi>(s, A, A2, B, epi, st, status);
+  }
+}
+
+static Operand opnd(const void* p, int64_t ld, int64_t bs, int kmajor, int64_t rows_per_batch) {
+  Operand o;
+  o.ptr = p; o.ld = ld; o.batch_stride = bs; o.kmajor = kmajor; o.rows_per_batch = rows_per_batch;
+  return o;
+}
+
+// ---------------------------------------------------------------------------
+// Enqueue one prefill (all chunks) on `st`.
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
+                                   float* W, float* M, const float* eta, const float* beta,
+                                   const float* gamma, float* chunk_loss, char* ws, cudaStream_t st) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, V = p.V, L = p.L;
+  float* KW = reinterpret_cast<float*>(ws + p.KW);
+  float* KM = reinterpret_cast<float*>(ws + p.KM);
+  float* consts = reinterpret_cast<float*>(ws + p.consts);
+  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+  float* resid = reinterpret_cast<float*>(ws + p.resid);
+  T* actin = reinterpret_cast<T*>(ws + p.actin);
+  T* act = reinterpret_cast<T*>(ws + p.act);
+  T* fac = reinterpret_cast<T*>(ws + p.fac);
+  T* z = reinterpret_cast<T*>(ws + p.z);
+  float* rstd = reinterpret_cast<float*>(ws + p.rstd);
+  float* part = reinterpret_cast<float*>(ws + p.part);
+  float* tgt = reinterpret_cast<float*>(ws + p.tgt);
+  float* lse = reinterpret_cast<float*>(ws + p.lse);
+  T* P = reinterpret_cast<T*>(ws + p.P);
+  float* dz = reinterpret_cast<float*>(ws + p.dz);
+  float* dout = reinterpret_cast<float*>(ws + p.dout);
+  T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
+  T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
+  T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
+  T* dU = reinterpret_cast<T*>(ws + p.dU);
+  T* dUW = reinterpret_cast<T*>(ws + p.dUW);
+  T* dUM = reinterpret_cast<T*>(ws + p.dUM);
+  const T* E = static_cast<const T*>(hd->E);
+  const T* S = static_cast<const T*>(hd->S);
+  int* status = hd->status;
+  cudaError_t err;
+#define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
+
+  // K1 for all chunks (depends only on the scalars).
+  TRY(launch_scalar_scan(eta, beta, gamma, B, p.T, b, KW, KM, consts, st));
+  // Operand shadow of W_0.
+  build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0);
+  TRY(cudaGetLastError());
+
+  const int64_t blk = (int64_t)p.m * h * d;          // params per block
+  const int64_t seqW = (int64_t)L * blk;             // params per sequence
+  const bool sw = p.swiglu;
+  // Lowest dynamic MLP index (forward order: per block [static], dynamic).
+  const int per_blk = p.has_static ? 2 : 1;
+  const int i_min = per_blk - 1;
+  auto is_dyn = [&](int i) { return (i % per_blk) == per_blk - 1; };
+  auto blk_of = [&](int i) { return i / per_blk; };
+
+  for (int c = 0; c < p.nchunks; ++c) {
+    TokenMap tm{b, p.T, c};
+    gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin);
+    TRY(cudaGetLastError());
+
+    // ---- forward through the blocks ----
+    for (int i = 0; i < p.nM; ++i) {
+      const bool dyn = is_dyn(i);
+      const int l = blk_of(i);
+      const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+      const T* w2 = w1 + (int64_t)H2 * d;
+      const int64_t wstride = dyn ? seqW : 0;
+      const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+      T* ain = actin + (int64_t)i * n * d;
+      T* aout = act + (int64_t)i * n * h;
+      T* fi = fac + (int64_t)i * n * H2;
+      {
+        GemmShape s{Mz, H2, d, Bz};
+        Operand A = opnd(ain, d, (int64_t)Mz * d, 1, Mz);
+        Operand Bw = opnd(w1, d, wstride, 1, H2);
+        T* fptr = (i >= i_min) ? fi : nullptr;
+        if (sw) TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status)));
+        else TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status)));
+      }
+      {
+        GemmShape s{Mz, d, h, Bz};
+        Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
+        Operand Bw = opnd(w2, h, wstride, 1, d);
+        T* next = (i + 1 < p.nM) ? actin + (int64_t)(i + 1) * n * d : nullptr;
+        TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, d, Mz}, st, status)));
+      }
+    }
+
+    // ---- head: RMSNorm, CE pass A, reduce ----
+    rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd);
+    TRY(cudaGetLastError());
+    {
+      GemmShape s{n, V, d, 1};
+      Operand A = opnd(z, d, 0, 1, n);
+      Operand Be = opnd(E, d, 0, 1, V);
+      TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status)));
+    }
+    ce_reduce_kernel<<<B, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, lse, chunk_loss, p.nchunks, status);
+    TRY(cudaGetLastError());
+    // ---- CE pass B and dz, one vocabulary slab at a time ----
+    for (int sl = 0; sl < p.nslabs; ++sl) {
+      const int v0 = sl * p.Vs;
+      const int vs = V - v0 < p.Vs ? V - v0 : p.Vs;
+      {
+        GemmShape s{n, vs, d, 1};
+        Operand A = opnd(z, d, 0, 1, n);
+        Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
+        TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status)));
+      }
+      {
+        GemmShape s{n, d, vs, 1};
+        Operand A = opnd(P, p.Vs, 0, 1, n);
+        Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 0, vs);
+        TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status)));
+      }
+    }
+    {
+      const int top = p.nM - 1;  // always dynamic
+      rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
+                                                         doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm);
+      TRY(cudaGetLastError());
+    }
+
+    // ---- backward, top down ----
+    for (int i = p.nM - 1; i >= i_min; --i) {
+      const bool dyn = is_dyn(i);
+      const int l = blk_of(i);
+      const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+      const T* w2 = w1 + (int64_t)H2 * d;
+      const int64_t wstride = dyn ? seqW : 0;
+      const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+      const bool need_dx = i > i_min;
+      T* fi = fac + (int64_t)i * n * H2;
+      {  // B1: dA = dOut W2 -> dU (+ scaled copies)
+        GemmShape s{Mz, h, d, Bz};
+        Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
+        Operand Bw = opnd(w2, h, wstride, 0, d);
+        T* du = need_dx ? dU : nullptr;
+        T* dw = dyn ? dUW : nullptr;
+        T* dm = dyn ? dUM : nullptr;
+        if (sw) TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status)));
+        else TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status)));
+      }
+      if (need_dx) {  // B2: dout += dU W1
+        GemmShape s{Mz, d, H2, Bz};
+        Operand A = opnd(dU, H2, (int64_t)Mz * H2, 1, Mz);
+        Operand Bw = opnd(w1, d, wstride, 0, H2);
+        const bool below_dyn = is_dyn(i - 1);
+        T* ow = below_dyn ? doutW[(i - 1) & 1] : nullptr;
+        T* om = below_dyn ? doutM[(i - 1) & 1] : nullptr;
+        TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status)));
+      }
+      if (dyn) {
+        T* ain = actin + (int64_t)i * n * d;
+        T* aout = act + (int64_t)i * n * h;
+        float* Wl = W + l * blk;
+        float* Ml = M + l * blk;
+        T* Sl = Wsh + l * blk;
+        {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens
+          GemmShape s{H2, d, b, B};
+          Operand A = opnd(dUW, H2, (int64_t)b * H2, 0, b);
+          Operand A2 = opnd(dUM, H2, (int64_t)b * H2, 0, b);
+          Operand Bx = opnd(ain, d, (int64_t)b * d, 0, b);
+          EpiUpdate<T> e{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+          TRY((gemm<T, 2>(s, A, A2, Bx, e, st, status)));
+        }
+        {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
+          GemmShape s{d, h, b, B};
+          Operand A = opnd(doutW[i & 1], d, (int64_t)b * d, 0, b);
+          Operand A2 = opnd(doutM[i & 1], d, (int64_t)b * d, 0, b);
+          Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
+          EpiUpdate<T> e{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
+                         consts, c, p.nchunks, h, 0};
+          TRY((gemm<T, 2>(s, A, A2, Bx, e, st, status)));
+        }
+      }
+    }
+  }
+#undef TRY
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Validation
+// ---------------------------------------------------------------------------
+static ttt_status check_config(const ttt_config* c) {
+  if (!c) return fail(TTT_ERR_INVALID_ARG, "config is NULL");
+  if (c->mlp != TTT_MLP_GELU && c->mlp != TTT_MLP_SWIGLU) return fail(TTT_ERR_INVALID_ARG, "mlp must be GELU or SwiGLU");
+  if (c->precision != TTT_PREC_FP32 && c->precision != TTT_PREC_BF16)
+    return fail(TTT_ERR_INVALID_ARG, "precision must be FP32 or BF16");
+  if (c->has_static != 0 && c->has_static != 1) return fail(TTT_ERR_INVALID_ARG, "has_static must be 0 or 1");
+  if (c->loss_reduction != TTT_REDUCE_MEAN && c->loss_reduction != TTT_REDUCE_SUM)
+    return fail(TTT_ERR_INVALID_ARG, "loss_reduction must be MEAN or SUM");
+  if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return fail(TTT_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
+  if (c->d < 16 || c->hidden < 16 || c->vocab < 16 || c->n_blocks < 1)
+    return fail(TTT_ERR_SHAPE, "d, hidden, vocab must be >= 16 and n_blocks >= 1");
+  if (c->d > 16384 || c->hidden > 65536 || c->vocab >= (1 << 26) || c->n_blocks > 64)
+    return fail(TTT_ERR_SHAPE, "size above the supported maximum");
+  if (c->d % 16 || c->hidden % 16 || c->vocab % 16)
+    return fail(TTT_ERR_UNSUPPORTED, "d, hidden and vocab must be multiples of 16");
+  return TTT_OK;
+}
+
+static ttt_status check_shape(const ttt_handle* h, int batch, int T, int b) {
+  if (!h) return fail(TTT_ERR_INVALID_ARG, "handle is NULL");
+  if (batch < 0 || T < 0) return fail(TTT_ERR_SHAPE, "batch and T must be >= 0");
+  if (b < 1) return fail(TTT_ERR_SHAPE, "chunk size b must be >= 1");
+  if (T % b != 0) return fail(TTT_ERR_SHAPE, "T must be a multiple of b");
+  if ((int64_t)batch * b > (1 << 24)) return fail(TTT_ERR_SHAPE, "batch * b above 2^24 tokens per step");
+  if ((int64_t)batch * T > ((int64_t)1 << 31) - 1) return fail(TTT_ERR_SHAPE, "batch * T above 2^31 - 1");
+  return TTT_OK;
+}
+
+}  // namespace ttt
+
+using namespace ttt;
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+const char* ttt_status_string(ttt_status s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_ERR_SHAPE: return "invalid shape";
+    case TTT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TTT_ERR_WORKSPACE: return "workspace too small";
+    case TTT_ERR_TOKEN_RANGE: return "token outside [0, vocab)";
+    case TTT_ERR_NONFINITE: return "non-finite loss";
+    case TTT_ERR_TIMEOUT: return "bounded wait timed out";
+    case TTT_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* ttt_last_error(void) { return g_last_error.c_str(); }
+
+ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* rms_gain,
+                      const float* static_w, ttt_handle** out) {
+  ttt_status s = check_config(cfg);
+  if (s != TTT_OK) return s;
+  if (!lm_head || !rms_gain || !out) return fail(TTT_ERR_INVALID_ARG, "lm_head, rms_gain and out must be non-NULL");
+  if (cfg->has_static && !static_w) return fail(TTT_ERR_INVALID_ARG, "static_w is NULL but has_static = 1");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return fail(TTT_ERR_UNSUPPORTED, "no CUDA device");
+  }
+  ttt_handle* h = new ttt_handle();
+  h->cfg = *cfg;
+  const char* env = getenv("TTT_GRAPH");
+  h->use_graph = !(env && env[0] == '0');
+  auto bail = [&](ttt_status st) { ttt_destroy(h); return st; };
+#define CTRY(x) do { cudaError_t _e = (x); if (_e != cudaSuccess) { set_last_error(#x, cudaGetErrorString(_e), __FILE__, __LINE__); return bail(TTT_ERR_CUDA); } } while (0)
+  CTRY(cudaGetDevice(&h->device));
+  const int64_t V = cfg->vocab, d = cfg->d, hh = cfg->hidden;
+  const int m = cfg->mlp == TTT_MLP_SWIGLU ? 3 : 2;
+  const size_t esz = cfg->precision == TTT_PREC_FP32 ? 4 : 2;
+  CTRY(cudaMalloc(&h->E, esz * V * d));
+  CTRY(cudaMalloc(&h->gain, 4 * d));
+  CTRY(cudaMalloc(&h->status, 8));
+  h->zero_flag = h->status + 1;
+  CTRY(cudaMemset(h->status, 0, 8));
+  CTRY(cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking));
+  CTRY(cudaMemcpyAsync(h->gain, rms_gain, 4 * d, cudaMemcpyDeviceToDevice, h->cap));
+  if (cfg->precision == TTT_PREC_FP32) {
+    CTRY(cudaMemcpyAsync(h->E, lm_head, 4 * V * d, cudaMemcpyDeviceToDevice, h->cap));
+  } else {
+    cast_kernel<bf16><<<1184, 256, 0, h->cap>>>(lm_head, static_cast<bf16*>(h->E), V * d);
+    CTRY(cudaGetLastError());
+  }
+  if (cfg->has_static) {
+    const int64_t count = cfg->n_blocks;
+    CTRY(cudaMalloc(&h->S, esz * count * m * hh * d));
+    if (cfg->precision == TTT_PREC_FP32)
+      build_shadow_kernel<float><<<1184, 256, 0, h->cap>>>(static_w, static_cast<float*>(h->S), count, (int)hh, (int)d, m == 3);
+    else
+      build_shadow_kernel<bf16><<<1184, 256, 0, h->cap>>>(static_w, static_cast<bf16*>(h->S), count, (int)hh, (int)d, m == 3);
+    CTRY(cudaGetLastError());
+  }
+  CTRY(cudaStreamSynchronize(h->cap));
+#undef CTRY
+  *out = h;
+  return TTT_OK;
+}
+
+void ttt_destroy(ttt_handle* h) {
+  if (!h) return;
+  if (h->cap) cudaStreamSynchronize(h->cap);
+  if (h->exec) cudaGraphExecDestroy(h->exec);
+  if (h->E) cudaFree(h->E);
+  if (h->gain) cudaFree(h->gain);
+  if (h->S) cudaFree(h->S);
+  if (h->status) cudaFree(h->status);
+  if (h->cap) cudaStreamDestroy(h->cap);
+  delete h;
+}
+
+ttt_status ttt_workspace_size(const ttt_handle* h, int32_t batch, int32_t T, int32_t b, size_t* bytes) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (!bytes) return fail(TTT_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = make_plan(h->cfg, batch, T, b).total;
+  return TTT_OK;
+}
+
+ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                       const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
+                       const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
+                       void* stream) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
+    return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  Plan p = make_plan(h->cfg, batch, T, b);
+  if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (reinterpret_cast<uintptr_t>(hidden) % 16) return fail(TTT_ERR_INVALID_ARG, "hidden must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+
+  auto enqueue = [&](cudaStream_t q) -> cudaError_t {
+    if (h->cfg.precision == TTT_PREC_FP32)
+      return enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q);
+    return enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q);
+  };
+
+  if (!h->use_graph) {
+    cudaError_t e = enqueue(st);
+    if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    return TTT_OK;
+  }
+  GraphKey key{batch, T, b, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, workspace, ws_bytes};
+  if (!(h->have_key && h->key == key && h->exec)) {
+    if (h->exec) { cudaGraphExecDestroy(h->exec); h->exec = nullptr; }
+    h->have_key = false;
+    TTT_CUDA_TRY(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+    cudaError_t e = enqueue(h->cap);
+    cudaGraph_t g = nullptr;
+    cudaError_t e2 = cudaStreamEndCapture(h->cap, &g);
+    if (e != cudaSuccess || e2 != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      set_last_error("capture", cudaGetErrorString(e != cudaSuccess ? e : e2), __FILE__, __LINE__);
+      return TTT_ERR_CUDA;
+    }
+    e = cudaGraphInstantiate(&h->exec, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) { h->exec = nullptr; set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    h->key = key;
+    h->have_key = true;
+  }
+  TTT_CUDA_TRY(cudaGraphLaunch(h->exec, st));
+  return TTT_OK;
+}
+
+ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* eta, const float* beta,
+                              const float* gamma, float* KW, float* KM, float* consts, void* stream) {
+  if (batch < 0 || T < 0) return fail(TTT_ERR_SHAPE, "batch and T must be >= 0");
+  if (b < 1 || T % b) return fail(TTT_ERR_SHAPE, "b >= 1 and T % b == 0 required");
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!eta || !beta || !gamma || !KW || !KM || !consts) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  TTT_CUDA_TRY(launch_scalar_scan(eta, beta, gamma, batch, T, b, KW, KM, consts, static_cast<cudaStream_t>(stream)));
+  return TTT_OK;
+}
+
+ttt_status ttt_get_device_status(ttt_handle* h, void* stream) {
+  if (!h) return fail(TTT_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  TTT_CUDA_TRY(cudaStreamSynchronize(st));
+  int v = 0;
+  TTT_CUDA_TRY(cudaMemcpy(&v, h->status, 4, cudaMemcpyDeviceToHost));
+  TTT_CUDA_TRY(cudaMemset(h->status, 0, 4));
+  return static_cast<ttt_status>(v);
+}
+
+ttt_status ttt_selftest_bounded_wait(ttt_handle* h, uint32_t spin_limit, void* stream) {
+  if (!h) return fail(TTT_ERR_INVALID_ARG, "handle is NULL");
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->zero_flag, spin_limit, h->status);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // extern "C"

@@ -52,6 +52,7 @@ class Workload:
     sgd_lr: float = 0.0
     token_dist: str = "zipf"
     rms_eps: float = 1e-6
+    reduction: str = "mean"  # chunk objective: mean (default) or sum of token losses
 
     @property
     def n_mats(self) -> int:

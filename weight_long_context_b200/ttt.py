@@ -1,0 +1,244 @@
+"""Thin Python binding of libttt (ctypes).  Argument marshalling only: every
+step of the inner loop runs in the library's CUDA kernels.
+
+The C names are re-exported one to one (ttt_create, ttt_prefill, ...); the
+Handle class wraps them for torch tensors.  PyTorch provides device memory
+and streams; nothing here computes any part of the method.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttt.so")
+
+TTT_OK = 0
+STATUS_NAMES = ["TTT_OK", "TTT_ERR_INVALID_ARG", "TTT_ERR_SHAPE", "TTT_ERR_UNSUPPORTED",
+                "TTT_ERR_WORKSPACE", "TTT_ERR_TOKEN_RANGE", "TTT_ERR_NONFINITE",
+                "TTT_ERR_TIMEOUT", "TTT_ERR_CUDA"]
+MLP = {"gelu": 0, "swiglu": 1}
+PRECISION = {"fp32": 0, "bf16": 1}
+REDUCTION = {"mean": 0, "sum": 1}
+
+EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_scalar_kernels",
+            "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
+            "ttt_last_error"]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str = ""):
+        name = STATUS_NAMES[code] if 0 <= code < len(STATUS_NAMES) else str(code)
+        super().__init__(f"{where}: {name}" + (f" ({detail})" if detail else ""))
+        self.code = code
+
+
+class ttt_config(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("n_blocks", ctypes.c_int32), ("mlp", ctypes.c_int32), ("has_static", ctypes.c_int32),
+                ("precision", ctypes.c_int32), ("loss_reduction", ctypes.c_int32),
+                ("rms_eps", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libttt.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libttt.so not found at {path}; run python -m weight_long_context_b200.build")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.ttt_create.argtypes = [ctypes.POINTER(ttt_config), P, P, P, ctypes.POINTER(P)]
+    lib.ttt_create.restype = I32
+    lib.ttt_destroy.argtypes = [P]
+    lib.ttt_destroy.restype = None
+    lib.ttt_workspace_size.argtypes = [P, I32, I32, I32, ctypes.POINTER(SZ)]
+    lib.ttt_workspace_size.restype = I32
+    lib.ttt_prefill.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.ttt_prefill.restype = I32
+    lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
+    lib.ttt_scalar_kernels.restype = I32
+    lib.ttt_get_device_status.argtypes = [P, P]
+    lib.ttt_get_device_status.restype = I32
+    lib.ttt_selftest_bounded_wait.argtypes = [P, ctypes.c_uint32, P]
+    lib.ttt_selftest_bounded_wait.restype = I32
+    lib.ttt_status_string.argtypes = [I32]
+    lib.ttt_status_string.restype = ctypes.c_char_p
+    lib.ttt_last_error.argtypes = []
+    lib.ttt_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(code: int, where: str):
+    if code != TTT_OK:
+        detail = load_library().ttt_last_error().decode(errors="replace")
+        raise TTTError(code, where, detail)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> Optional[ctypes.c_void_p]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str, device) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on the CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# --- the C names, re-exported --------------------------------------------------
+
+def ttt_create(cfg: ttt_config, lm_head, rms_gain, static_w):
+    lib = load_library()
+    h = ctypes.c_void_p()
+    _check(lib.ttt_create(ctypes.byref(cfg), _ptr(lm_head), _ptr(rms_gain), _ptr(static_w),
+                          ctypes.byref(h)), "ttt_create")
+    return h
+
+
+def ttt_destroy(h):
+    load_library().ttt_destroy(h)
+
+
+def ttt_workspace_size(h, batch: int, T: int, b: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().ttt_workspace_size(h, batch, T, b, ctypes.byref(n)), "ttt_workspace_size")
+    return n.value
+
+
+def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tensor, b: int, stream=None):
+    """K1 alone: returns (KW [B,T], KM [B,T], consts [B,T/b,4]) as new CUDA tensors."""
+    B, T = eta.shape
+    for t, nm in ((eta, "eta"), (beta, "beta"), (gamma, "gamma")):
+        _dev(t, torch.float32, nm, eta.device)
+    KW = torch.empty_like(eta)
+    KM = torch.empty_like(eta)
+    consts = torch.empty((B, T // b if b > 0 else 0, 4), dtype=torch.float32, device=eta.device)
+    _check(load_library().ttt_scalar_kernels(B, T, b, _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(KW),
+                                             _ptr(KM), _ptr(consts), _stream_ptr(stream)),
+           "ttt_scalar_kernels")
+    return KW, KM, consts
+
+
+def ttt_status_string(code: int) -> str:
+    return load_library().ttt_status_string(code).decode()
+
+
+def ttt_last_error() -> str:
+    return load_library().ttt_last_error().decode(errors="replace")
+
+
+# --- object wrapper ------------------------------------------------------------
+
+class Handle:
+    """A libttt handle with the frozen head / static weights bound.
+
+    lm_head [V, d], rms_gain [d], static_w [n_blocks*m*h*d] or None: float32
+    tensors on the CUDA device (copied by the library).
+    """
+
+    def __init__(self, d: int, hidden: int, vocab: int, n_blocks: int, mlp: str, has_static: bool,
+                 precision: str, lm_head: torch.Tensor, rms_gain: torch.Tensor,
+                 static_w: Optional[torch.Tensor] = None, rms_eps: float = 1e-6,
+                 reduction: str = "mean"):
+        dev = lm_head.device
+        _dev(lm_head, torch.float32, "lm_head", dev)
+        _dev(rms_gain, torch.float32, "rms_gain", dev)
+        if static_w is not None:
+            _dev(static_w, torch.float32, "static_w", dev)
+        self.cfg = ttt_config(d, hidden, vocab, n_blocks, MLP[mlp], int(bool(has_static)),
+                              PRECISION[precision], REDUCTION[reduction], rms_eps)
+        self.device = dev
+        self.n_mats = 2 if mlp == "gelu" else 3
+        with torch.cuda.device(dev):
+            self._h = ttt_create(self.cfg, lm_head, rms_gain, static_w)
+        self._ws = None
+
+    # workspace cached per handle, grown on demand
+    def workspace(self, batch: int, T: int, b: int) -> torch.Tensor:
+        need = ttt_workspace_size(self._h, batch, T, b)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def prefill(self, hidden, tokens, W, M, eta, beta, gamma, b: int,
+                chunk_loss: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Run the inner loop on device tensors.  W and M are updated in place.
+
+        hidden [B,T,d] f32, tokens [B,T] i32, W/M [B*n_blocks*m*h*d] f32,
+        eta/beta/gamma [B,T] f32.  Returns chunk_loss [B, T/b] (f32, device).
+        """
+        dev = self.device
+        B, T, d = hidden.shape
+        for t, nm in ((hidden, "hidden"), (W, "W"), (M, "M"), (eta, "eta"), (beta, "beta"),
+                      (gamma, "gamma")):
+            _dev(t, torch.float32, nm, dev)
+        _dev(tokens, torch.int32, "tokens", dev)
+        nparams = B * self.cfg.n_blocks * self.n_mats * self.cfg.hidden * self.cfg.d
+        if W.numel() != nparams or M.numel() != nparams:
+            raise ValueError(f"W and M must hold {nparams} floats")
+        if tuple(tokens.shape) != (B, T) or tuple(eta.shape) != (B, T):
+            raise ValueError("tokens / eta / beta / gamma must be [B, T]")
+        nc = T // b if b > 0 else 0
+        if chunk_loss is None:
+            chunk_loss = torch.empty((B, nc), dtype=torch.float32, device=dev)
+        ws = self.workspace(B, T, b)
+        _check(load_library().ttt_prefill(self._h, B, T, b, _ptr(hidden), _ptr(tokens), _ptr(W), _ptr(M),
+                                          _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(chunk_loss),
+                                          _ptr(ws), ws.numel(), _stream_ptr(stream)), "ttt_prefill")
+        return chunk_loss
+
+    def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None):
+        """End-to-end call on HOST tensors: copies the inputs to the device,
+        runs the inner loop, copies W, M and the chunk losses back.  Returns
+        (W, M, chunk_loss) as host tensors."""
+        dev = self.device
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(st):
+            d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0, eta, beta, gamma)]
+            loss = self.prefill(*d_in, b=b, stream=st)
+            outs = []
+            for t in (d_in[2], d_in[3], loss):
+                o = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                o.copy_(t, non_blocking=True)
+                outs.append(o)
+        st.synchronize()
+        return tuple(outs)
+
+    def device_status(self, stream=None) -> int:
+        return load_library().ttt_get_device_status(self._h, _stream_ptr(stream))
+
+    def selftest_bounded_wait(self, spin_limit: int, stream=None):
+        _check(load_library().ttt_selftest_bounded_wait(self._h, spin_limit, _stream_ptr(stream)),
+               "ttt_selftest_bounded_wait")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            ttt_destroy(self._h)
+            self._h = None
+        self._ws = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
