@@ -149,6 +149,18 @@ ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* 
                               const float* beta, const float* gamma, float* KW, float* KM,
                               float* consts, void* stream);
 
+/* The tensor-core GEMM the inner loop is built on, exposed for testing and
+ * reuse: D[z] = A[z] B[z]^T for z < batch, i.e.
+ *   D[z](m, n) = sum_{k < K} A[z](m, k) * B[z](n, k)
+ * with bfloat16 operands (device, 16-byte aligned) and float32 output D
+ * (row-major, leading dimension ldd, batch stride strideD, in elements).
+ * A(m, k) is at A + z*strideA + (a_kmajor ? m*lda + k : k*lda + m); same for
+ * B(n, k).  lda, ldb, strideA, strideB: multiples of 8 elements; strides are
+ * nonzero when batch > 1.  Asynchronous on `stream`. */
+ttt_status ttt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
+                         int64_t strideA, int32_t a_kmajor, const void* B, int64_t ldb, int64_t strideB,
+                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* stream);
+
 /* Synchronise `stream`, return the first device-side error recorded by this
  * handle's kernels since the last call (TTT_OK if none) and clear it. */
 ttt_status ttt_get_device_status(ttt_handle* h, void* stream);

@@ -1,0 +1,45 @@
+"""The tcgen05 GEMM engine alone (through ttt_gemm_bf16) against a plain
+PyTorch fp32 matmul of the same bf16 operands: every operand layout, batching,
+ragged tails in M, N and K, and sizes spanning many tiles."""
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+SHAPES = [(128, 256, 64, 1), (24, 200, 80, 3), (296, 520, 136, 2), (1024, 2304, 1024, 1), (136, 96, 24, 4),
+          (64, 48, 16, 1)]
+
+
+@pytest.mark.parametrize("a_k", [True, False])
+@pytest.mark.parametrize("b_k", [True, False])
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"{m}x{n}x{k}b{z}" for m, n, k, z in SHAPES])
+def test_gemm_layouts(dev, shape, a_k, b_k):
+    from weight_long_context_b200 import ttt
+    M, N, K, Z = shape
+    g = torch.Generator(device="cpu").manual_seed(M * 7 + N * 3 + K)
+    A = torch.randn(Z, M, K, generator=g).to(dev, torch.bfloat16)
+    B = torch.randn(Z, N, K, generator=g).to(dev, torch.bfloat16)
+    ref = torch.matmul(A.float(), B.float().transpose(1, 2))
+    Ain = A if a_k else A.transpose(1, 2).contiguous()
+    Bin = B if b_k else B.transpose(1, 2).contiguous()
+    D = ttt.ttt_gemm_bf16(Ain, Bin, a_k, b_k)
+    torch.cuda.synchronize()
+    err = (D - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 1e-5, err
+
+
+def test_gemm_rejects_unaligned_strides(dev):
+    from weight_long_context_b200 import ttt
+    A = torch.zeros(1, 136, 300, device=dev, dtype=torch.bfloat16)   # MN-major, pitch 600 bytes
+    B = torch.zeros(1, 64, 136, device=dev, dtype=torch.bfloat16)
+    with pytest.raises(ttt.TTTError) as ei:
+        ttt.ttt_gemm_bf16(A, B, False, True)
+    assert ei.value.code == 3

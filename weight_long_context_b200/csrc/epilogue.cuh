@@ -3,7 +3,9 @@
 // spans of 32 consecutive columns (c0 % 32 == 0), after row_begin() and
 // before row_end().  A span carries the fp32 accumulator values v[0..31]
 // (and v2[] for the dual-accumulator update GEMM); only the first `nv`
-// columns are inside the matrix.
+// columns are inside the matrix.  One thread owns a row, so every span is a
+// contiguous run in memory: full spans use 16-byte vector accesses (all row
+// pitches are multiples of 16 elements), the ragged tail goes element-wise.
 //
 // The arithmetic here is the elementwise part of the chunk step:
 //   forward MLP activations ("Rethinking Expressivity and Efficiency in
@@ -30,6 +32,10 @@ struct TokenMap {
 
 struct NoRowState {};
 
+// Every epilogue declares kFixedHeadTile: true when its output layout depends
+// on the N tile of the tcgen05 engine (the engine then always uses its head
+// tile width), false when any N tile will do.
+
 __device__ __forceinline__ float gelu_f(float u) { return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f)); }
 __device__ __forceinline__ float gelu_grad_f(float u) {
   float cdf = 0.5f * (1.0f + erff(u * 0.70710678118654752f));
@@ -39,6 +45,57 @@ __device__ __forceinline__ float gelu_grad_f(float u) {
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
 
 // ---------------------------------------------------------------------------
+// Vector access helpers: N contiguous elements, 16-byte aligned.
+// ---------------------------------------------------------------------------
+template <int N>
+__device__ __forceinline__ void vld(const float* p, float* v) {
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    float4 x = reinterpret_cast<const float4*>(p)[i];
+    v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+  }
+}
+template <int N>
+__device__ __forceinline__ void vst(float* p, const float* v) {
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i)
+    reinterpret_cast<float4*>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+template <int N>
+__device__ __forceinline__ void vld(const __nv_bfloat16* p, float* v) {
+#pragma unroll
+  for (int i = 0; i < N / 8; ++i) {
+    uint4 x = reinterpret_cast<const uint4*>(p)[i];
+    float2 a = unpack_bf16x2(x.x), b = unpack_bf16x2(x.y), c = unpack_bf16x2(x.z), d = unpack_bf16x2(x.w);
+    v[8 * i] = a.x; v[8 * i + 1] = a.y; v[8 * i + 2] = b.x; v[8 * i + 3] = b.y;
+    v[8 * i + 4] = c.x; v[8 * i + 5] = c.y; v[8 * i + 6] = d.x; v[8 * i + 7] = d.y;
+  }
+}
+template <int N>
+__device__ __forceinline__ void vst(__nv_bfloat16* p, const float* v) {
+#pragma unroll
+  for (int i = 0; i < N / 8; ++i)
+    reinterpret_cast<uint4*>(p)[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                                pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+// Scaled store: p[j] = T(s * v[j]).
+template <int N, typename T>
+__device__ __forceinline__ void vst_scaled(T* p, const float* v, float s) {
+  float t[N];
+#pragma unroll
+  for (int j = 0; j < N; ++j) t[j] = s * v[j];
+  vst<N>(p, t);
+}
+
+// ---------------------------------------------------------------------------
 // F1: U = a W1^T (GELU: [n,h]; SwiGLU: [n,2h] in the interleaved layout).
 // Writes the activation A (input of the second matrix) and the factors the
 // backward needs: GELU'(U), or for SwiGLU dA/dgate = up * SiLU'(gate) and
@@ -46,6 +103,7 @@ __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf
 // ---------------------------------------------------------------------------
 template <typename T, bool SWIGLU>
 struct EpiF1 {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   T* act;        // [rows, h]
   T* fac;        // [rows, H2] or nullptr when no backward passes through
@@ -58,29 +116,37 @@ struct EpiF1 {
     if (!SWIGLU) {
       T* a = act + grow * h + c0;
       T* f = fac ? fac + grow * h + c0 : nullptr;
+      float av[32], fv[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        if (j < nv) {
-          float u = v[j];
-          a[j] = from_f<T>(gelu_f(u));
-          if (f) f[j] = from_f<T>(gelu_grad_f(u));
+        av[j] = gelu_f(v[j]);
+        fv[j] = f ? gelu_grad_f(v[j]) : 0.f;
+      }
+      if (nv == 32) {
+        vst<32>(a, av);
+        if (f) vst<32>(f, fv);
+      } else {
+  #pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) {
+          a[j] = from_f<T>(av[j]);
+          if (f) f[j] = from_f<T>(fv[j]);
         }
       }
     } else {
-      int g = c0 >> 5;            // full 32-wide group (2h % 32 == 0)
-      T* a = act + grow * h + (g << 4);
-      T* f = fac ? fac + grow * (2 * (int64_t)h) + c0 : nullptr;
+      // a full 32-wide group (2h % 32 == 0): gate in v[0..15], up in v[16..31]
+      const int g = c0 >> 5;
+      float av[16], fv[32];
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         float gv = v[k], uv = v[16 + k];
         float sg = sigmoid_f(gv);
         float silu = gv * sg;
-        a[k] = from_f<T>(silu * uv);
-        if (f) {
-          f[k] = from_f<T>(uv * sg * (1.0f + gv * (1.0f - sg)));
-          f[16 + k] = from_f<T>(silu);
-        }
+        av[k] = silu * uv;
+        fv[k] = uv * sg * (1.0f + gv * (1.0f - sg));
+        fv[16 + k] = silu;
       }
+      vst<16>(act + grow * h + (g << 4), av);
+      if (fac) vst<32>(fac + grow * (2 * (int64_t)h) + c0, fv);
     }
   }
 };
@@ -90,6 +156,7 @@ struct EpiF1 {
 // ---------------------------------------------------------------------------
 template <typename T>
 struct EpiResid {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   float* resid;   // [rows, d]
   T* act_next;    // [rows, d] or nullptr
@@ -101,9 +168,16 @@ struct EpiResid {
     int64_t grow = (int64_t)z * rows_per_z + r;
     float* p = resid + grow * d + c0;
     T* q = act_next ? act_next + grow * d + c0 : nullptr;
+    if (nv == 32) {
+      float x[32];
+      vld<32>(p, x);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nv) {
+      for (int j = 0; j < 32; ++j) x[j] += v[j];
+      vst<32>(p, x);
+      if (q) vst<32>(q, x);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) {
         float x = p[j] + v[j];
         p[j] = x;
         if (q) q[j] = from_f<T>(x);
@@ -117,9 +191,12 @@ struct EpiResid {
 // dynamic MLP also the K-scaled negated copies -K_W dU and -K_M dU that are
 // the A operands of the aggregation (so the aggregation GEMM yields
 // sum_t K_t G_t directly, G_t being the negative gradient).
+// SwiGLU: the 32 dA columns [c0, c0+32) own the 64 contiguous interleaved
+// positions [2 c0, 2 c0 + 64) (gate/up groups of 16).
 // ---------------------------------------------------------------------------
 template <typename T, bool SWIGLU>
 struct EpiB1 {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   const T* fac;   // [rows, H2]
   T* dU;          // [rows, H2] or nullptr
@@ -142,27 +219,42 @@ struct EpiB1 {
       kw = -KW[ti] * kscale;
       km = -KM[ti] * kscale;
     }
-    const T* f = fac + grow * H2;
-    int64_t ob = grow * H2;
+    const int64_t ob = grow * H2;
+    if (!SWIGLU) {
+      if (nv == 32) {
+        float f[32], du[32];
+        vld<32>(fac + ob + c0, f);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nv) {
-        int c = c0 + j;
-        float da = v[j];
-        if (!SWIGLU) {
-          float du = da * to_f<T>(f[c]);
+        for (int j = 0; j < 32; ++j) du[j] = v[j] * f[j];
+        if (dU) vst<32>(dU + ob + c0, du);
+        if (dUW) { vst_scaled<32>(dUW + ob + c0, du, kw); vst_scaled<32>(dUM + ob + c0, du, km); }
+      } else {
+  #pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) {
+          int c = c0 + j;
+          float du = v[j] * to_f<T>(fac[ob + c]);
           if (dU) dU[ob + c] = from_f<T>(du);
           if (dUW) { dUW[ob + c] = from_f<T>(kw * du); dUM[ob + c] = from_f<T>(km * du); }
-        } else {
-          int pg = swiglu_pos_gate(c), pu = pg + 16;
-          float dg = da * to_f<T>(f[pg]);
-          float du = da * to_f<T>(f[pu]);
-          if (dU) { dU[ob + pg] = from_f<T>(dg); dU[ob + pu] = from_f<T>(du); }
-          if (dUW) {
-            dUW[ob + pg] = from_f<T>(kw * dg); dUW[ob + pu] = from_f<T>(kw * du);
-            dUM[ob + pg] = from_f<T>(km * dg); dUM[ob + pu] = from_f<T>(km * du);
-          }
         }
+      }
+    } else {
+      // h % 16 == 0 and c0 % 32 == 0: nv is 16 or 32, whole groups of 16.
+      const int64_t p0 = ob + 2 * (int64_t)c0;
+      float f[64], du[64];
+      if (nv == 32) vld<64>(fac + p0, f);
+      else vld<32>(fac + p0, f);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int gi = (j >> 4) * 32 + (j & 15);   // gate position within the 64
+        du[gi] = v[j] * f[gi];
+        du[gi + 16] = v[j] * f[gi + 16];
+      }
+      if (nv == 32) {
+        if (dU) vst<64>(dU + p0, du);
+        if (dUW) { vst_scaled<64>(dUW + p0, du, kw); vst_scaled<64>(dUM + p0, du, km); }
+      } else {
+        if (dU) vst<32>(dU + p0, du);
+        if (dUW) { vst_scaled<32>(dUW + p0, du, kw); vst_scaled<32>(dUM + p0, du, km); }
       }
     }
   }
@@ -174,6 +266,7 @@ struct EpiB1 {
 // ---------------------------------------------------------------------------
 template <typename T>
 struct EpiB2 {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   float* dout;    // [rows, d]
   T* dout_a;      // [rows, d]
@@ -196,9 +289,17 @@ struct EpiB2 {
       km = -KM[ti] * kscale;
     }
     int64_t o = grow * d + c0;
+    if (nv == 32) {
+      float x[32];
+      vld<32>(dout + o, x);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nv) {
+      for (int j = 0; j < 32; ++j) x[j] += v[j];
+      vst<32>(dout + o, x);
+      vst<32>(dout_a + o, x);
+      if (doutW) { vst_scaled<32>(doutW + o, x, kw); vst_scaled<32>(doutM + o, x, km); }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) {
         float x = dout[o + j] + v[j];
         dout[o + j] = x;
         dout_a[o + j] = from_f<T>(x);
@@ -209,10 +310,12 @@ struct EpiB2 {
 };
 
 // ---------------------------------------------------------------------------
-// Cross-entropy, pass A: per (row, N-tile) running max and sum of exp of the
-// logits (online softmax), and the target logit.  The logits stay on chip.
+// Cross-entropy, pass A: per (row, column part) running max and sum of exp of
+// the logits (online softmax), and the target logit.  The logits stay on chip.
+// `part_index` (from the engine) numbers the column parts of a row.
 // ---------------------------------------------------------------------------
 struct EpiCEPartial {
+  static constexpr bool kFixedHeadTile = true;
   struct RowState { float m, s; int y; };
   float* part;        // [rows, ntn, 2]
   float* tgt;         // [rows]
@@ -239,10 +342,9 @@ struct EpiCEPartial {
       for (int j = 0; j < 32; ++j) if (j == k) tgt[r] = v[j];
     }
   }
-  __device__ void row_end(RowState& st, int, int r, int tile_n) const {
-    float* p = part + ((int64_t)r * ntn + tile_n) * 2;
-    p[0] = st.m;
-    p[1] = st.s;
+  __device__ void row_end(RowState& st, int, int r, int part_index) const {
+    float* p = part + ((int64_t)r * ntn + part_index) * 2;
+    *reinterpret_cast<float2*>(p) = make_float2(st.m, st.s);
   }
 };
 
@@ -252,6 +354,7 @@ struct EpiCEPartial {
 // ---------------------------------------------------------------------------
 template <typename T>
 struct EpiCEGrad {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = int;  // the row's label
   T* P;               // [rows, Vs]
   const float* lse;   // [rows]
@@ -262,16 +365,16 @@ struct EpiCEGrad {
   __device__ void row_begin(RowState& y, int, int r) const { y = tokens[tm.index(r)]; }
   __device__ void row_end(RowState&, int, int, int) const {}
   __device__ void span(RowState& y, int, int r, int c0, const float* v, const float*, int nv) const {
-    float l = lse[r];
+    const float l = lse[r];
     T* o = P + (int64_t)r * Vs + c0;
-    int k = y - slab0 - c0;
+    const int k = y - slab0 - c0;
+    float p[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nv) {
-        float p = expf(v[j] - l);
-        if (j == k) p -= 1.0f;
-        o[j] = from_f<T>(p);
-      }
+    for (int j = 0; j < 32; ++j) p[j] = expf(v[j] - l) - (j == k ? 1.0f : 0.0f);
+    if (nv == 32) vst<32>(o, p);
+    else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) o[j] = from_f<T>(p[j]);
     }
   }
 };
@@ -281,6 +384,7 @@ struct EpiCEGrad {
 // ones accumulate).
 // ---------------------------------------------------------------------------
 struct EpiStoreF32 {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   float* out;
   int ld;
@@ -289,8 +393,36 @@ struct EpiStoreF32 {
   __device__ void row_end(RowState&, int, int, int) const {}
   __device__ void span(RowState&, int, int r, int c0, const float* v, const float*, int nv) const {
     float* o = out + (int64_t)r * ld + c0;
+    if (nv == 32) {
+      float x[32];
+      if (accumulate) {
+        vld<32>(o, x);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) if (j < nv) o[j] = accumulate ? o[j] + v[j] : v[j];
+        for (int j = 0; j < 32; ++j) x[j] += v[j];
+        vst<32>(o, x);
+      } else {
+        vst<32>(o, v);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) o[j] = accumulate ? o[j] + v[j] : v[j];
+    }
+  }
+};
+
+// Batched fp32 store: out[z](r, c) at out + z * zstride + r * ld + c.
+struct EpiStoreBatched {
+  static constexpr bool kFixedHeadTile = false;
+  using RowState = NoRowState;
+  float* out;
+  int64_t ld;
+  int64_t zstride;
+  __device__ void row_begin(RowState&, int, int) const {}
+  __device__ void row_end(RowState&, int, int, int) const {}
+  __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
+    float* o = out + (int64_t)z * zstride + (int64_t)r * ld + c0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) if (j < nv) o[j] = v[j];
   }
 };
 
@@ -302,6 +434,7 @@ struct EpiStoreF32 {
 // ---------------------------------------------------------------------------
 template <typename T>
 struct EpiUpdate {
+  static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   float* W;            // this matrix, sequence 0 (rows of the packed layout)
   float* M;
@@ -316,15 +449,31 @@ struct EpiUpdate {
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float* v2, int nv) const {
-    const float* cs = consts + ((int64_t)z * nchunks + chunk) * 4;
-    float g0 = cs[0], b0 = cs[1], cM = cs[2];
+    const float4 cs = *reinterpret_cast<const float4*>(consts + ((int64_t)z * nchunks + chunk) * 4);
+    const float g0 = cs.x, b0 = cs.y, cM = cs.z;
     int fr = h > 0 ? swiglu_row_of_pos(r, h) : r;
     float* wp = W + z * seq_stride + (int64_t)fr * cols + c0;
     float* mp = M + z * seq_stride + (int64_t)fr * cols + c0;
     T* sp = Wsh + z * sh_stride + (int64_t)r * cols + c0;
+    if (nv == 32) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nv) {
+      for (int q = 0; q < 2; ++q) {   // two halves of 16 keep register use bounded
+        float w[16], m[16];
+        vld<16>(wp + 16 * q, w);
+        vld<16>(mp + 16 * q, m);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float wn = fmaf(g0, w[j], fmaf(cM, m[j], v[16 * q + j]));
+          m[j] = fmaf(b0, m[j], v2[16 * q + j]);
+          w[j] = wn;
+        }
+        vst<16>(wp + 16 * q, w);
+        vst<16>(mp + 16 * q, m);
+        vst<16>(sp + 16 * q, w);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) {
         float w = wp[j], m = mp[j];
         float wn = fmaf(g0, w, fmaf(cM, m, v[j]));
         float mn = fmaf(b0, m, v2[j]);

@@ -1,11 +1,471 @@
-// tcgen05 GEMM engine (placeholder: routes to the CUDA-core engine).
+// tcgen05 GEMM engine for sm_100a: D[z](m, n) = sum_k A[z](m, k) B[z](n, k),
+// bf16 operands, fp32 accumulation in tensor memory (TMEM).
+//
+// Structure (one persistent CTA per SM, 320 threads):
+//   warp 0      TMA producer: one lane streams 128x64 A tiles (and a second A
+//               for the dual-accumulator aggregation) and BNx64 B tiles into a
+//               ring of shared-memory stages, 128-byte swizzled, arriving on
+//               the stage's "full" mbarrier with the transaction byte count;
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//               K=16 per instruction) and frees each stage with tcgen05.commit;
+//   warps 2..9  epilogue: wait for a finished accumulator, tcgen05.ld 32
+//               columns at a time and hand the row spans to the epilogue
+//               functor.  A warp may only read the TMEM lane quarter
+//               (warp % 4); two warps share each quarter and split the tile's
+//               columns in halves, one row per thread.
+// Accumulators are double-buffered in TMEM so the epilogue of tile i overlaps
+// the MMAs of tile i+1.  Operands may be K-major or MN-major (the matrix
+// descriptors and the instruction descriptor carry the layout), so the
+// backward and aggregation GEMMs read the forward buffers without transposes.
+// No TMA multicast is used anywhere.
+//
+// Every mbarrier wait is bounded by the global timer; on expiry the kernel
+// records TTT_ERR_TIMEOUT, raises a CTA-wide abort flag, waits (bounded) for
+// its own TMA copies and MMAs in flight, frees its TMEM and returns.
 #pragma once
-#include "gemm_simt.cuh"
-namespace ttt { namespace tc {
-constexpr int HEAD_BN = simt::BN;
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "gemm_types.cuh"
+
+namespace ttt {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;             // 64 bf16 = 128 bytes: one swizzle row
+constexpr int HEAD_BN = 256;       // N tile of the single-accumulator GEMMs
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_PARTS = EPI_WARPS / 4;   // column parts per tile row
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint64_t WAIT_NS = 4000000000ull;   // 4 s per wait before giving up
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait.  Returns false on abort (flag raised elsewhere) or timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (global_ns() - t0 > WAIT_NS) {
+        record_error(status, TTT_ERR_TIMEOUT);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// 32 lanes x 32 columns of 32-bit: thread i of the warp gets row (lane base + i),
+// columns [col, col+32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1
+// at bit 46, layout type 2 at bits 61-63).  Addresses and offsets in bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M=128, N=n.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel configuration per (accumulators, N tile)
+// ---------------------------------------------------------------------------
+template <int NACC, int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;            // 16 KiB
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = NACC * A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * NACC * BN;         // two accumulator buffers
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(STAGES >= 2, "need at least two stages");
+};
+
+struct TcParams {
+  GemmShape s;
+  int a_mn, b_mn;       // 1 = MN-major operand
+  int tiles_m, tiles_n, num_tiles, num_kb;
+  int* status;
+};
+
+template <int NACC, int BN, class Epi>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
+               const __grid_constant__ CUtensorMap mapB, const TcParams p, const Epi epi) {
+  using C = Cfg<NACC, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 32 * EPI_WARPS); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const GemmShape& s = p.s;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int tm = t % p.tiles_m;
+        const int rest = t / p.tiles_m;
+        const int tn = rest % p.tiles_n;
+        const int z = rest / p.tiles_n;
+        const int m0 = tm * BM, n0 = tn * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* sa = smem + st * C::STAGE_BYTES;
+          uint8_t* sb = sa + NACC * C::A_BYTES;
+          mbar_expect_tx(&full[st], C::STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_3d(sa, &mapA, &full[st], k0, m0, z);
+            if (NACC == 2) tma_load_3d(sa + C::A_BYTES, &mapA2, &full[st], k0, m0, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j) {
+              tma_load_3d(sa + j * 8192, &mapA, &full[st], m0 + 64 * j, k0, z);
+              if (NACC == 2) tma_load_3d(sa + C::A_BYTES + j * 8192, &mapA2, &full[st], m0 + 64 * j, k0, z);
+            }
+          }
+          if (!p.b_mn) {
+            tma_load_3d(sb, &mapB, &full[st], k0, n0, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, &mapB, &full[st], n0 + 64 * j, k0, z);
+          }
+        }
+      }
+      // Drain: every copy issued above completes on its stage's full barrier.
+      const uint32_t issued = it;
+      const uint32_t first = issued > (uint32_t)C::STAGES ? issued - C::STAGES : 0;
+      for (uint32_t j = first; j < issued; ++j)
+        mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ----------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(BN, p.a_mn, p.b_mn);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++tcount) {
+        const uint32_t buf = tcount & 1u;
+        const uint32_t aph = (tcount >> 1) & 1u;
+        if (!mbar_wait(&tempty[buf], aph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * (NACC * BN);
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
+          const uint32_t sb = sa + NACC * C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // K-major: advance 16 elements = 32 bytes inside the swizzled row.
+            // MN-major: advance 16 K-rows = two 8-row groups of 1024 bytes.
+            const uint64_t bdesc = p.b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
+#pragma unroll
+            for (int a = 0; a < NACC; ++a) {
+              const uint32_t abase = sa + a * C::A_BYTES;
+              const uint64_t adesc = p.a_mn ? smem_desc_sw128(abase + kk * 2048, 8192, 1024)
+                                            : smem_desc_sw128(abase + kk * 32, 16, 1024);
+              mma_bf16(d0 + a * BN, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(&empty[st]);   // frees the stage once these MMAs have read it
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);    // accumulator ready for the epilogue
+      }
+      // Drain: wait for every MMA this thread issued.
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, p.status);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int part = (warp - 2) >> 2;       // which column part of the tile
+    constexpr int PART_COLS = BN / EPI_PARTS;
+    const int row_in_tile = q * 32 + lane;
+    uint32_t tcount = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
+      const int tm = t % p.tiles_m;
+      const int rest = t / p.tiles_m;
+      const int tn = rest % p.tiles_n;
+      const int z = rest / p.tiles_n;
+      const uint32_t buf = tcount & 1u;
+      const uint32_t aph = (tcount >> 1) & 1u;
+      // Warp-uniform decision: tcgen05.ld below is .sync.aligned.
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
+      if (!ready) break;
+      tc_fence_after();
+      const int r = tm * BM + row_in_tile;
+      const bool row_ok = r < s.M;
+      typename Epi::RowState rs;
+      if (row_ok) epi.row_begin(rs, z, r);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
+#pragma unroll 1
+      for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
+        float v[32], v2[32];
+        tmem_ld32(tbase + c, v);
+        if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
+        const int c0 = tn * BN + c;
+        if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+      }
+      if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps (via the driver entry point, no libcuda link) and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// 3-D map of a bf16 operand: dims (inner, outer, batch).  K-major: inner = K,
+// outer = MN rows; MN-major: inner = MN, outer = K rows.  Box: 64 inner
+// elements (128 bytes, 128-byte swizzle) by box_outer rows.
+inline cudaError_t make_map(CUtensorMap* m, const Operand& op, int64_t inner, int64_t outer, int batch,
+                            int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)(batch > 0 ? batch : 1)};
+  cuuint64_t bs = op.batch_stride > 0 ? (cuuint64_t)op.batch_stride * 2 : (cuuint64_t)op.ld * 2 * outer;
+  if (bs % 16) bs = (bs + 15) / 16 * 16;
+  cuuint64_t strides[2] = {(cuuint64_t)op.ld * 2, bs};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_outer, 1u};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(op.ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Operand of the A side (rows = M) or B side (rows = N).  For a batched GEMM
+// whose batch_stride is 0 the map has one batch entry and z is clamped.
+inline cudaError_t make_operand_map(CUtensorMap* m, const Operand& op, int mn_extent, int k_extent, int batch,
+                                    int box_mn) {
+  const int nb = op.batch_stride > 0 ? batch : 1;
+  if (op.kmajor) return make_map(m, op, k_extent, op.rows_per_batch, nb, box_mn);
+  return make_map(m, op, mn_extent, op.rows_per_batch, nb, 64);
+}
+
+template <int NACC, int BN, class Epi>
+cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
+                      cudaStream_t st, int* status) {
+  using C = Cfg<NACC, BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<NACC, BN, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  // Shared operands (batch_stride 0) always use batch coordinate 0.
+  if ((A.batch_stride == 0 || B.batch_stride == 0) && s.batch > 1) return cudaErrorInvalidValue;
+  CUtensorMap ma, ma2, mb;
+  cudaError_t e;
+  // For K-major operands rows_per_batch is the MN extent in memory; for
+  // MN-major ones it is the K extent (rows of the buffer per batch entry).
+  e = make_operand_map(&ma, A, s.M, s.K, s.batch, BM);
+  if (e != cudaSuccess) return e;
+  if (NACC == 2) {
+    e = make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
+    if (e != cudaSuccess) return e;
+  } else {
+    ma2 = ma;
+  }
+  e = make_operand_map(&mb, B, s.N, s.K, s.batch, BN);
+  if (e != cudaSuccess) return e;
+  TcParams p;
+  p.s = s;
+  p.a_mn = A.kmajor ? 0 : 1;
+  p.b_mn = B.kmajor ? 0 : 1;
+  p.tiles_m = (s.M + BM - 1) / BM;
+  p.tiles_n = (s.N + BN - 1) / BN;
+  p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
+  p.num_kb = (s.K + BK - 1) / BK;
+  p.status = status;
+  const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
+  gemm_tc_kernel<NACC, BN, Epi><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
+  return cudaGetLastError();
+}
+
+// Fraction of the machine a GEMM keeps busy with N tile `bn`: tiles over
+// (waves x SMs), discounted for N=128 tiles, which need 4/3 more operand
+// bytes per FLOP than N=256 (128x128: 128 B/clk of TMA feed at full MMA rate,
+// 128x256: 96 B/clk); the 0.78 factor is the measured ratio on B200.
+inline double tile_efficiency(const GemmShape& s, int bn) {
+  const int sms = num_sms();
+  const long tiles = (long)((s.M + BM - 1) / BM) * ((s.N + bn - 1) / bn) * s.batch;
+  const long waves = (tiles + sms - 1) / sms;
+  return (double)tiles / (double)(waves * sms) * (bn == 128 ? 0.78 : 1.0);
+}
+
 template <int NACC, class Epi>
 cudaError_t launch_gemm_tc(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B,
-                           const Epi& epi, cudaStream_t st, int*) {
-  return launch_gemm_simt<__nv_bfloat16, NACC, Epi>(s, A, A2, B, epi, st);
+                           const Epi& epi, cudaStream_t st, int* status) {
+  if (s.M <= 0 || s.N <= 0 || s.batch <= 0 || s.K <= 0) return cudaSuccess;
+  if constexpr (NACC == 2) {
+    return launch_tc<2, 128, Epi>(s, A, A2, B, epi, st, status);
+  } else if constexpr (Epi::kFixedHeadTile) {
+    return launch_tc<1, HEAD_BN, Epi>(s, A, A2, B, epi, st, status);
+  } else {
+    if (tile_efficiency(s, 128) > tile_efficiency(s, 256)) return launch_tc<1, 128, Epi>(s, A, A2, B, epi, st, status);
+    return launch_tc<1, 256, Epi>(s, A, A2, B, epi, st, status);
+  }
 }
-}}
+
+}  // namespace tc
+}  // namespace ttt

@@ -9,6 +9,19 @@
 
 namespace ttt {
 
+template <typename T>
+__device__ __forceinline__ void store4(T* p, float4 x);
+template <>
+__device__ __forceinline__ void store4<float>(float* p, float4 x) { *reinterpret_cast<float4*>(p) = x; }
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 x) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
 // ---------------------------------------------------------------------------
 // Gather chunk c of every sequence: resid[s*b + i] = hidden[s, c*b + i] and
 // its operand copy.
@@ -23,8 +36,7 @@ __global__ void gather_chunk_kernel(const float* __restrict__ hidden, int T_, in
     int64_t s = r / b, i = r - s * b;
     const float4 x = reinterpret_cast<const float4*>(hidden + ((s * T_ + (int64_t)chunk * b + i) * d))[c4];
     reinterpret_cast<float4*>(resid + r * d)[c4] = x;
-    T* a = act + r * d + c4 * 4;
-    a[0] = from_f<T>(x.x); a[1] = from_f<T>(x.y); a[2] = from_f<T>(x.z); a[3] = from_f<T>(x.w);
+    store4<T>(act + r * d + c4 * 4, x);
   }
 }
 
@@ -106,35 +118,45 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dz, const float* __
 }
 
 // ---------------------------------------------------------------------------
-// Cross-entropy reduction: one block per sequence.  Combines each row's
-// per-tile (max, sum exp) partials into lse, forms l_t = lse - logit[y_t],
-// and writes the chunk's mean loss.  Fixed thread-to-row mapping and a fixed
-// reduction tree: the result does not depend on scheduling.
+// Cross-entropy reduction, one warp per row: combine the row's online-softmax
+// partials (max, sum exp) into lse and form l_t = lse - logit[y_t].
 // ---------------------------------------------------------------------------
-__global__ void ce_reduce_kernel(const float* __restrict__ part, const float* __restrict__ tgt, int ntn,
-                                 const int* __restrict__ tokens, TokenMap tm, int V,
-                                 float* __restrict__ lse, float* __restrict__ chunk_loss, int nchunks,
-                                 int* status) {
-  __shared__ float red[32];
-  const int s = blockIdx.x;
-  const int b = tm.b;
-  float acc = 0.f;
-  for (int i = threadIdx.x; i < b; i += blockDim.x) {
-    int r = s * b + i;
-    const float* p = part + (int64_t)r * ntn * 2;
-    float m = -INFINITY;
-    for (int t = 0; t < ntn; ++t) m = fmaxf(m, p[2 * t]);
-    float sum = 0.f;
-    for (int t = 0; t < ntn; ++t) sum += p[2 * t + 1] * expf(p[2 * t] - m);
+__global__ void ce_rows_kernel(const float* __restrict__ part, const float* __restrict__ tgt, int ntn,
+                               const int* __restrict__ tokens, TokenMap tm, int V, int64_t n,
+                               float* __restrict__ lse, float* __restrict__ ltok, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= n) return;
+  const float2* p = reinterpret_cast<const float2*>(part + r * ntn * 2);
+  float m = -INFINITY;
+  for (int t = lane; t < ntn; t += 32) m = fmaxf(m, p[t].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+  for (int t = lane; t < ntn; t += 32) { float2 q = p[t]; sum += q.y * expf(q.x - m); }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) {
     float l = m + logf(sum);
     lse[r] = l;
-    int y = tokens[tm.index(r)];
+    int y = tokens[tm.index((int)r)];
     if (y < 0 || y >= V) {
       record_error(status, TTT_ERR_TOKEN_RANGE);
-      continue;
+      ltok[r] = 0.f;
+    } else {
+      ltok[r] = l - tgt[r];
     }
-    acc += l - tgt[r];
   }
+}
+
+// Chunk mean of the token losses, one block per sequence, fixed reduction
+// order (the result does not depend on scheduling).
+__global__ void ce_mean_kernel(const float* __restrict__ ltok, int b, float* __restrict__ chunk_loss, int chunk,
+                               int nchunks, int* status) {
+  __shared__ float red[32];
+  const int s = blockIdx.x;
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < b; i += blockDim.x) acc += ltok[(int64_t)s * b + i];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
@@ -146,7 +168,7 @@ __global__ void ce_reduce_kernel(const float* __restrict__ part, const float* __
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (threadIdx.x == 0) {
       float mean = v / (float)b;
-      chunk_loss[(int64_t)s * nchunks + tm.chunk] = mean;
+      chunk_loss[(int64_t)s * nchunks + chunk] = mean;
       if (!isfinite(mean)) record_error(status, TTT_ERR_NONFINITE);
     }
   }
@@ -161,17 +183,18 @@ template <typename T>
 __global__ void build_shadow_kernel(const float* __restrict__ W, T* __restrict__ sh, int64_t count,
                                     int h, int d, int swiglu) {
   const int64_t blk = (swiglu ? 3 : 2) * (int64_t)h * d;
-  const int64_t total = count * blk;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    int64_t o = e % blk, base = e - o;
+  const int64_t total4 = count * blk / 4;   // d % 16 == 0: a group of 4 never crosses a row
+  for (int64_t e4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < total4;
+       e4 += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = 4 * e4;
+    const int64_t o = e % blk, base = e - o;
     int64_t src = e;
     if (swiglu && o < 2 * (int64_t)h * d) {
-      int p = (int)(o / d);
-      int64_t c = o - (int64_t)p * d;
+      const int p = (int)(o / d);
+      const int64_t c = o - (int64_t)p * d;
       src = base + (int64_t)swiglu_row_of_pos(p, h) * d + c;
     }
-    sh[e] = from_f<T>(W[src]);
+    store4<T>(sh + e, *reinterpret_cast<const float4*>(W + src));
   }
 }
 

@@ -92,13 +92,18 @@ struct Plan {
   float kscale;  // 1/b for the mean reduction, 1 for the sum
   bool swiglu, has_static;
   size_t esz;  // operand element size
-  size_t KW, KM, consts, Wsh, resid, actin, act, fac, z, rstd, part, tgt, lse, P, dz, dout, dout_a,
+  size_t KW, KM, consts, Wsh, resid, actin, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
       doutW[2], doutM[2], dU, dUW, dUM, total;
 };
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-static int head_tile_n(int precision) { return precision == TTT_PREC_FP32 ? simt::BN : tc::HEAD_BN; }
+// Online-softmax partials per row: one per N tile (fp32 engine) or per column
+// part of an N tile (tcgen05 engine).
+static int head_parts(int precision, int V) {
+  if (precision == TTT_PREC_FP32) return (V + simt::BN - 1) / simt::BN;
+  return (V + tc::HEAD_BN - 1) / tc::HEAD_BN * tc::EPI_PARTS;
+}
 
 static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   Plan p{};
@@ -109,7 +114,7 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.nM = p.L * (p.has_static ? 2 : 1);
   p.esz = c.precision == TTT_PREC_FP32 ? 4 : 2;
   p.kscale = (c.loss_reduction == TTT_REDUCE_MEAN && b > 0) ? 1.0f / (float)b : 1.0f;
-  p.ntn = (p.V + head_tile_n(c.precision) - 1) / head_tile_n(c.precision);
+  p.ntn = head_parts(c.precision, p.V);
   // vocabulary slab: the [n, Vs] slab of dl/dlogits is the only per-vocabulary
   // buffer; capped at 32 MiB so it stays resident in L2.
   const size_t cap = 32ull << 20;
@@ -136,6 +141,7 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.part = take(8 * n * p.ntn);
   p.tgt = take(4 * n);
   p.lse = take(4 * n);
+  p.ltok = take(4 * n);
   p.P = take(e * n * p.Vs);
   p.dz = take(4 * n * d);
   p.dout = take(4 * n * d);
@@ -189,6 +195,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   float* part = reinterpret_cast<float*>(ws + p.part);
   float* tgt = reinterpret_cast<float*>(ws + p.tgt);
   float* lse = reinterpret_cast<float*>(ws + p.lse);
+  float* ltok = reinterpret_cast<float*>(ws + p.ltok);
   T* P = reinterpret_cast<T*>(ws + p.P);
   float* dz = reinterpret_cast<float*>(ws + p.dz);
   float* dout = reinterpret_cast<float*>(ws + p.dout);
@@ -261,7 +268,9 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       Operand Be = opnd(E, d, 0, 1, V);
       TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status)));
     }
-    ce_reduce_kernel<<<B, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, lse, chunk_loss, p.nchunks, status);
+    ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status);
+    TRY(cudaGetLastError());
+    ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status);
     TRY(cudaGetLastError());
     // ---- CE pass B and dz, one vocabulary slab at a time ----
     for (int sl = 0; sl < p.nslabs; ++sl) {
@@ -529,6 +538,27 @@ ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* 
   if (batch == 0 || T == 0) return TTT_OK;
   if (!eta || !beta || !gamma || !KW || !KM || !consts) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
   TTT_CUDA_TRY(launch_scalar_scan(eta, beta, gamma, batch, T, b, KW, KM, consts, static_cast<cudaStream_t>(stream)));
+  return TTT_OK;
+}
+
+ttt_status ttt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
+                         int64_t strideA, int32_t a_kmajor, const void* B, int64_t ldb, int64_t strideB,
+                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || batch < 0) return fail(TTT_ERR_SHAPE, "negative size");
+  if (M == 0 || N == 0 || K == 0 || batch == 0) return TTT_OK;
+  if (!A || !B || !D) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) % 16 || lda % 8 || ldb % 8 ||
+      strideA % 8 || strideB % 8)
+    return fail(TTT_ERR_UNSUPPORTED, "operands need 16-byte aligned bases and strides multiple of 8 elements");
+  if (lda < (a_kmajor ? K : M) || ldb < (b_kmajor ? K : N) || ldd < N)
+    return fail(TTT_ERR_SHAPE, "leading dimension smaller than the matrix");
+  if (batch > 1 && (strideA == 0 || strideB == 0))
+    return fail(TTT_ERR_UNSUPPORTED, "batched operands need nonzero strides");
+  GemmShape s{M, N, K, batch};
+  Operand a = opnd(A, lda, strideA, a_kmajor ? 1 : 0, a_kmajor ? M : K);
+  Operand b = opnd(B, ldb, strideB, b_kmajor ? 1 : 0, b_kmajor ? N : K);
+  EpiStoreBatched e{D, ldd, strideD};
+  TTT_CUDA_TRY((tc::launch_gemm_tc<1, EpiStoreBatched>(s, a, a, b, e, static_cast<cudaStream_t>(stream), nullptr)));
   return TTT_OK;
 }
 

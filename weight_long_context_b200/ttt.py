@@ -24,7 +24,7 @@ MLP = {"gelu": 0, "swiglu": 1}
 PRECISION = {"fp32": 0, "bf16": 1}
 REDUCTION = {"mean": 0, "sum": 1}
 
-EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_scalar_kernels",
+EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_scalar_kernels", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
 
@@ -65,6 +65,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill.restype = I32
     lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
     lib.ttt_scalar_kernels.restype = I32
+    I64 = ctypes.c_int64
+    lib.ttt_gemm_bf16.argtypes = [I32, I32, I32, I32, P, I64, I64, I32, P, I64, I64, I32, P, I64, I64, P]
+    lib.ttt_gemm_bf16.restype = I32
     lib.ttt_get_device_status.argtypes = [P, P]
     lib.ttt_get_device_status.restype = I32
     lib.ttt_selftest_bounded_wait.argtypes = [P, ctypes.c_uint32, P]
@@ -137,6 +140,28 @@ def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tenso
                                              _ptr(KM), _ptr(consts), _stream_ptr(stream)),
            "ttt_scalar_kernels")
     return KW, KM, consts
+
+
+def ttt_gemm_bf16(A: torch.Tensor, B: torch.Tensor, a_kmajor: bool = True, b_kmajor: bool = True,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """D[z] = A[z] B[z]^T on the tcgen05 engine.  A, B: bf16 CUDA tensors of shape
+    [batch, M, K] / [batch, N, K] when K-major, [batch, K, M] / [batch, K, N] when
+    MN-major (2-D inputs are batch 1).  Returns fp32 [batch, M, N]."""
+    A3 = A if A.dim() == 3 else A.unsqueeze(0)
+    B3 = B if B.dim() == 3 else B.unsqueeze(0)
+    _dev(A3, torch.bfloat16, "A", A.device)
+    _dev(B3, torch.bfloat16, "B", A.device)
+    batch = A3.shape[0]
+    M, K = (A3.shape[1], A3.shape[2]) if a_kmajor else (A3.shape[2], A3.shape[1])
+    N = B3.shape[1] if b_kmajor else B3.shape[2]
+    if out is None:
+        out = torch.empty((batch, M, N), dtype=torch.float32, device=A.device)
+    sA = A3.shape[1] * A3.shape[2] if batch > 1 else 0
+    sB = B3.shape[1] * B3.shape[2] if batch > 1 else 0
+    _check(load_library().ttt_gemm_bf16(M, N, K, batch, _ptr(A3), A3.shape[2], sA, int(a_kmajor), _ptr(B3),
+                                        B3.shape[2], sB, int(b_kmajor), _ptr(out), N, M * N,
+                                        _stream_ptr(stream)), "ttt_gemm_bf16")
+    return out if A.dim() == 3 else out[0]
 
 
 def ttt_status_string(code: int) -> str:
