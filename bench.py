@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""Benchmark of the TTT-E2E inner loop with the E2-TTT chunk update on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one full prefill call (every chunk of every sequence of the
+workload: gather, MLP forward, fused LM-head cross-entropy, backward and the
+closed-form weight/momentum update) on inputs already resident in HBM.
+Metric: inner-loop tokens per second over the whole job (all GPUs), and the
+algorithmic FLOP rate against the measured bf16 tensor-core peak.
+
+Multi-GPU (launched by torch.distributed.run): every rank processes its own
+independent sequences (the workload with seed = rank); there is no
+data-path collective, only a barrier around the timed region and a max of the
+elapsed time over ranks (weak scaling).
+
+--impl reference times the CPU oracle (numpy, float32 BLAS on the host cores)
+on a bounded sample of the same workload: it is a baseline, not the target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_long_context_b200 import inputs as I  # noqa: E402
+
+METRIC = "TTT inner-loop tokens/sec at 1 B200; % of bf16 tensor-core peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "stack_128k"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# Workload arithmetic (algorithmic work per token; a restatement of the
+# method's FLOP count, not a measurement)
+# ---------------------------------------------------------------------------
+
+def flops_per_token(w: I.Workload) -> float:
+    """Algorithmic FLOPs per token of one inner-loop pass.
+
+    Each MLP forward 2 m d h; LM head 4 d V (logits + dz, the head is frozen);
+    backward to every dynamic MLP's activation 2 d h, plus 2 (m-1) d h for dX
+    when a dynamic MLP lies below, plus 2 m d h per static MLP above the lowest
+    dynamic one; aggregation 2 m d h per dynamic MLP per kernel (x2 for K_W and
+    K_M, x1 for plain SGD where M_C = eta_C G_C is a rank-1 write).  The
+    logits recompute of the cross-entropy backward is not counted.
+    """
+    d, h, V, L, m = w.d, w.hidden, w.vocab, w.n_blocks, w.n_mats
+    n_static = L if w.has_static else 0
+    fwd = (L + n_static) * 2 * m * d * h
+    head = 4 * d * V
+    bwd = L * 2 * d * h + (L - 1) * 2 * (m - 1) * d * h + (max(n_static - 1, 0)) * 2 * m * d * h
+    agg = L * 2 * m * d * h * (1 if w.scalars == "sgd" else 2)
+    return float(fwd + head + bwd + agg)
+
+
+def state_bytes(w: I.Workload) -> int:
+    return w.batch * w.n_blocks * w.block_params * 4 * 2
+
+
+def input_bytes(w: I.Workload) -> int:
+    return w.batch * w.T * (w.d * 4 + 4 + 12)
+
+
+def measured_peaks() -> dict:
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {}
+
+
+def peaks():
+    m = measured_peaks()
+    if m.get("bf16_tflops") and m.get("hbm_gbs"):
+        return dict(tflops=float(m["bf16_tflops"]), tflops_sustained=float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                    hbm=float(m["hbm_gbs"]), source="measured")
+    return dict(tflops=1590.0, tflops_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="ttt_clocks_", suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             + ",".join("clocks_event_reasons." + r for r in REASONS))
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 5 + len(REASONS):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for r, v in zip(REASONS, f[5:5 + len(REASONS)]):
+                if v.lower() == "active":
+                    reasons.add(r)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": sorted(reasons), "samples": 0}
+        # samples under load: power above the midpoint of the observed range
+        pmin, pmax = min(power), max(power)
+        load = [s for s, p in zip(sm, power) if p >= pmin + 0.5 * (pmax - pmin)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------------------
+# Multi-rank helpers (tested on CPU with gloo)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(backend: str, timeout_s: int = 180):
+    import datetime
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    return units_per_rank * world / max_seconds if max_seconds > 0 else 0.0
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for dp, _, fs in sorted(os.walk(os.path.join(ROOT, "weight_long_context_b200", "csrc"))):
+        for f in sorted(fs):
+            h.update(open(os.path.join(dp, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m_h = re.search(r"kernel_source_hash:\s*(\w+)", txt)
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not (m_h and m_t) or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline of our arm; the whole reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_chunks(w: I.Workload, n_chunks: int, seed: int = 0):
+    """Run the oracle on the first n_chunks chunks of one sequence; returns seconds."""
+    import oracle  # test infrastructure: the CPU baseline only
+    ws = w.with_(T=n_chunks * w.b, batch=1)
+    x = I.make_inputs(ws, seed=seed)
+    dtype = np.float64 if w.precision == "fp32" else np.float32
+    model = oracle.make_model(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.rms_eps, x["lm_head"], x["rms_gain"],
+                              x["static_w"], dtype=dtype)
+    t0 = time.perf_counter()
+    oracle.prefill(model, x["W0"], x["M0"], x["hidden"], x["tokens"], x["eta"], x["beta"], x["gamma"], w.b,
+                   dtype=dtype, reduction=w.reduction)
+    return time.perf_counter() - t0
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: I.Workload, budget_s: float = 12.0) -> dict:
+    """Oracle tokens/s on a bounded sample: whole chunks of one sequence until
+    about budget_s of CPU work (at least one chunk)."""
+    t1 = oracle_chunks(w, 1)
+    k = max(1, min(w.n_chunks, int(budget_s / max(t1, 1e-3))))
+    tk = oracle_chunks(w, k) if k > 1 else t1
+    prec = "float64" if w.precision == "fp32" else "float32"
+    return {"value": k * w.b / tk, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"first {k} chunk(s) ({k * w.b} tokens) of one sequence of {w.name}, numpy {prec} "
+                      f"BLAS, {tk:.1f} s"}
+
+
+def run_reference(args, w: I.Workload):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    per = oracle_chunks(w, 1)
+    k_chunks = max(1, min(w.n_chunks, int(15.0 / max(per * (args.steps + args.warmup), 1e-3))))
+    for _ in range(args.warmup):
+        oracle_chunks(w, k_chunks)
+    times = [oracle_chunks(w, k_chunks) for _ in range(args.steps)]
+    tok = k_chunks * w.b
+    value = tok * args.steps / sum(times)
+    cb = {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+          "sample": f"each step: first {k_chunks} chunk(s) ({tok} tokens) of one sequence of {w.name}, "
+                    f"numpy float32 BLAS"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32" if w.precision != "fp32" else "f64",
+            "data": "synthetic", "impl": "reference", "config": workload_config(w),
+            "cpu_baseline": cb, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                         "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: I.Workload) -> dict:
+    big = input_bytes(w) + state_bytes(w) > 2 * L2_BYTES
+    return {"workload": w.name, "d": w.d, "hidden": w.hidden, "vocab": w.vocab, "blocks": w.n_blocks,
+            "mlp": w.mlp, "static_mlp": w.has_static, "T": w.T, "chunk_b": w.b, "sequences_per_gpu": w.batch,
+            "scalars": w.scalars, "loss_reduction": w.reduction,
+            "precision": "fp32" if w.precision == "fp32" else "bf16 GEMM operands, fp32 accumulate/state",
+            "l2": ("inputs larger than L2 (hidden + fast-weight state %.2f GiB per step)" % ((input_bytes(w) + state_bytes(w)) / 2 ** 30))
+                  if big else "L2 flushed between timed steps (write of a 256 MiB buffer)"}
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w: I.Workload):
+    import torch
+    from weight_long_context_b200 import ttt
+
+    rank, world, local = dist_env()
+    if world > 1:
+        init_dist("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    st = torch.cuda.current_stream(dev)
+
+    x = I.make_inputs(w, seed=rank)
+    T = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    h = ttt.Handle(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.has_static, w.precision, T(x["lm_head"]),
+                   T(x["rms_gain"]), T(x["static_w"]) if x["static_w"] is not None else None, w.rms_eps,
+                   w.reduction)
+    hidden, tokens = T(x["hidden"]), T(x["tokens"], torch.int32)
+    W, M = T(x["W0"]), T(x["M0"])
+    eta, beta, gamma = T(x["eta"]), T(x["beta"]), T(x["gamma"])
+    flush = None
+    if input_bytes(w) + state_bytes(w) <= 2 * L2_BYTES:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        return h.prefill(hidden, tokens, W, M, eta, beta, gamma, w.b, stream=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert h.device_status() == 0, "device status after warm-up"
+
+    # ---- timed region: K steps, per-step CUDA events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        ev[i][0].record(st)
+        step()
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    status = h.device_status()
+    mean_ms = reduce_max(statistics.mean(step_ms), dev)
+    tokens_per_step = w.batch * w.T
+    value = whole_job_rate(tokens_per_step, world, mean_ms / 1e3)
+
+    # ---- per-kernel breakdown from one profiled replay (same launches, eager, events per launch)
+    W2, M2 = W.clone(), M.clone()
+    _, stats = h.prefill_profiled(hidden, tokens, W2, M2, eta, beta, gamma, w.b, stream=st)
+    del W2, M2
+    launches_per_step = sum(s["launches"] for s in stats)
+    pk = peaks()
+    gemms = [s for s in stats if s["flops"] > 0]
+    dom = max(gemms, key=lambda s: s["ms"])
+    t_tensor = dom["flops"] / (pk["tflops_sustained"] * 1e12)
+    t_hbm = dom["bytes"] / (pk["hbm"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    per_launch_ms = dom["ms"] / dom["launches"]
+    if bound == "tensor":
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        peak, unit = pk["tflops_sustained"], "TFLOP/s"
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        peak, unit = pk["hbm"], "GB/s"
+    traffic = profiled_traffic(dom["name"], w.name)
+    step_total = sum(s["ms"] for s in stats)
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic, "kernel": dom["name"], "launches_per_step": dom["launches"],
+                "ms_per_launch": per_launch_ms, "share_of_step": dom["ms"] / step_total,
+                "algorithmic_flops_per_launch": dom["flops"] / dom["launches"],
+                "algorithmic_bytes_per_launch": dom["bytes"] / dom["launches"],
+                "peak_source": f"{pk['source']} (bf16 sustained; HBM copy)"}
+
+    # ---- end to end through the public API with host buffers
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    hx = [pin(x["hidden"]), pin(x["tokens"].astype(np.int32)), pin(x["W0"]), pin(x["M0"]), pin(x["eta"]),
+          pin(x["beta"]), pin(x["gamma"])]
+    h2d = sum(t.numel() * t.element_size() for t in hx)
+    d2h = 2 * hx[2].numel() * 4 + w.batch * w.n_chunks * 4
+    del hidden, tokens, W, M, eta, beta, gamma
+    torch.cuda.empty_cache()
+    h.prefill_host(*hx, b=w.b, stream=st)    # warm the host path once
+    e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e_steps):
+        h.prefill_host(*hx, b=w.b, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e_steps, dev)
+    e2e = {"value": whole_job_rate(tokens_per_step, world, e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e_steps}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        fl = flops_per_token(w)
+        tflops = value * fl / 1e12
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.precision == "bf16" else "f32", "data": "synthetic",
+                "config": workload_config(w),
+                "algorithmic_tflops": tflops,
+                "pct_of_bf16_peak": {"burst": tflops / world / pk["tflops"],
+                                     "sustained": tflops / world / pk["tflops_sustained"], "source": pk["source"]},
+                "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+                "roofline": roofline, "device_status": status}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    w = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -138,6 +138,24 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
                        const float* eta, const float* beta, const float* gamma,
                        float* chunk_loss, void* workspace, size_t ws_bytes, void* stream);
 
+/* Per-kernel-class record of one profiled prefill. */
+typedef struct ttt_kernel_stat {
+  char name[24];     /* kernel class, e.g. "agg_update", "mlp_up", "ce_logits_lse" */
+  int64_t launches;  /* launches of this class in the call */
+  double ms;         /* summed device time, CUDA events around each launch */
+  double flops;      /* executed tensor-core FLOPs (2 M N K per GEMM), 0 for row kernels */
+  double bytes;      /* algorithmic bytes: each operand, state and output moved once */
+} ttt_kernel_stat;
+
+/* The same computation as ttt_prefill (same arguments, same results), run
+ * without the CUDA graph and with CUDA events around every launch, for
+ * tracing.  Synchronises `stream` before returning.  Fills stats[0..n) with
+ * one record per kernel class that ran (at most max_stats). */
+ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                                const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
+                                const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
+                                void* stream, ttt_kernel_stat* stats, int32_t max_stats, int32_t* n_stats);
+
 /* The scalar kernels of Proposition 3.1 for every chunk, on the device
  * ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1; computed in the division-free form
  * K_W_t = eta_t sum_{j>=t} (prod_{i=t+1}^{j} beta_i) gtilde_j, float64 inside).

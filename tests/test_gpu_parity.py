@@ -273,3 +273,25 @@ def test_bounded_wait_times_out_cleanly(dev):
     Wg, Mg, Lg, st = H.run_gpu(w, x, dev, handle=h)
     assert st == 0 and np.all(np.isfinite(Wg))
     h.close()
+
+
+def test_profiled_path_matches_graph_path(dev):
+    """ttt_prefill_profiled runs the same kernels eagerly with events: results
+    are bit-identical to the graph path and every launch is accounted for."""
+    w = I.Workload("prof", 128, 256, 544, 2, "swiglu", True, "bf16", 256, 64, 2, "e2ttt")
+    x = I.make_inputs(w, seed=4, m0_scale=1e-3)
+    Wa, Ma, La, st, h = H.run_gpu(w, x, dev, return_handle=True)
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    W, M = t(x["W0"]), t(x["M0"])
+    loss, stats = h.prefill_profiled(t(x["hidden"]), t(x["tokens"], torch.int32), W, M, t(x["eta"]),
+                                     t(x["beta"]), t(x["gamma"]), w.b)
+    assert np.array_equal(W.cpu().numpy(), Wa) and np.array_equal(M.cpu().numpy(), Ma)
+    assert np.array_equal(loss.cpu().numpy(), La)
+    names = {s["name"] for s in stats}
+    assert {"agg_update", "mlp_up", "mlp_down", "ce_logits_lse", "ce_dz", "mlp_bwd_dA"} <= names
+    assert all(s["ms"] > 0 and s["launches"] > 0 for s in stats)
+    upd = next(s for s in stats if s["name"] == "agg_update")
+    # two aggregation GEMMs per dynamic MLP per chunk, 2 x 2 x rows x cols x b x batch FLOPs
+    assert upd["launches"] == 2 * w.n_blocks * w.n_chunks
+    assert upd["flops"] == pytest.approx(4.0 * 3 * w.hidden * w.d * w.b * w.batch * w.n_blocks * w.n_chunks)
+    h.close()

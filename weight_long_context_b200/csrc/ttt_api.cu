@@ -80,6 +80,7 @@ struct ttt_handle {
   ttt::GraphKey key;
   bool have_key = false;
   bool use_graph = true;
+  int64_t launches = 0;     // kernel launches of the last prefill
 };
 
 namespace ttt {
@@ -175,12 +176,53 @@ static Operand opnd(const void* p, int64_t ld, int64_t bs, int kmajor, int64_t r
 }
 
 // ---------------------------------------------------------------------------
+// Launch recorder: counts launches always; with timing on (the profiled
+// entry point, eager launches) brackets every launch with CUDA events and
+// accumulates per-class time, executed MMA FLOPs and algorithmic bytes.
+// ---------------------------------------------------------------------------
+enum KernelClass {
+  K_SCAN, K_SHADOW, K_GATHER, K_MLP_UP, K_MLP_DOWN, K_RMS_FWD, K_CE_LSE, K_CE_ROWS, K_CE_MEAN,
+  K_CE_GRAD, K_CE_DZ, K_RMS_BWD, K_BWD_DA, K_BWD_DX, K_AGG_UPDATE, K_NCLASS
+};
+static const char* kClassName[K_NCLASS] = {
+    "scalar_scan", "w_shadow", "gather", "mlp_up", "mlp_down", "rmsnorm_fwd", "ce_logits_lse", "ce_rows",
+    "ce_mean", "ce_logits_grad", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update"};
+
+struct Prof {
+  bool timing = false;
+  int64_t launches = 0;
+  struct Rec { int cls; cudaEvent_t a, b; double flops, bytes; };
+  std::vector<Rec> recs;
+  int cur = -1;
+  void begin(int cls, cudaStream_t st) {
+    ++launches;
+    if (!timing) return;
+    Rec r{cls, nullptr, nullptr, 0, 0};
+    cudaEventCreate(&r.a);
+    cudaEventCreate(&r.b);
+    cudaEventRecord(r.a, st);
+    recs.push_back(r);
+  }
+  void end(double flops, double bytes, cudaStream_t st) {
+    if (!timing) return;
+    Rec& r = recs.back();
+    r.flops = flops;
+    r.bytes = bytes;
+    cudaEventRecord(r.b, st);
+  }
+  ~Prof() {
+    for (auto& r : recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+  }
+};
+
+// ---------------------------------------------------------------------------
 // Enqueue one prefill (all chunks) on `st`.
 // ---------------------------------------------------------------------------
 template <typename T>
 static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
                                    float* W, float* M, const float* eta, const float* beta,
-                                   const float* gamma, float* chunk_loss, char* ws, cudaStream_t st) {
+                                   const float* gamma, float* chunk_loss, char* ws, cudaStream_t st,
+                                   Prof& prof) {
   const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, V = p.V, L = p.L;
   float* KW = reinterpret_cast<float*>(ws + p.KW);
   float* KM = reinterpret_cast<float*>(ws + p.KM);
@@ -210,12 +252,14 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   int* status = hd->status;
   cudaError_t err;
 #define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
+#define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
+  const double e = (double)p.esz;
 
   // K1 for all chunks (depends only on the scalars).
-  TRY(launch_scalar_scan(eta, beta, gamma, B, p.T, b, KW, KM, consts, st));
+  LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T, TRY(launch_scalar_scan(eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
   // Operand shadow of W_0.
-  build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0);
-  TRY(cudaGetLastError());
+  LAUNCH(K_SHADOW, 0, (4.0 + e) * B * L * p.m * h * d,
+         (build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0)));
 
   const int64_t blk = (int64_t)p.m * h * d;          // params per block
   const int64_t seqW = (int64_t)L * blk;             // params per sequence
@@ -228,8 +272,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
 
   for (int c = 0; c < p.nchunks; ++c) {
     TokenMap tm{b, p.T, c};
-    gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin);
-    TRY(cudaGetLastError());
+    LAUNCH(K_GATHER, 0, (8.0 + e) * n * d, (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin)));
 
     // ---- forward through the blocks ----
     for (int i = 0; i < p.nM; ++i) {
@@ -247,31 +290,35 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         Operand A = opnd(ain, d, (int64_t)Mz * d, 1, Mz);
         Operand Bw = opnd(w1, d, wstride, 1, H2);
         T* fptr = (i >= i_min) ? fi : nullptr;
-        if (sw) TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status)));
-        else TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status)));
+        const double fl = 2.0 * Mz * H2 * d * Bz;
+        const double by = e * ((double)n * d + (double)H2 * d * Bz + (double)n * h + (fptr ? (double)n * H2 : 0.0));
+        if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status))));
+        else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status))));
       }
       {
         GemmShape s{Mz, d, h, Bz};
         Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
         Operand Bw = opnd(w2, h, wstride, 1, d);
         T* next = (i + 1 < p.nM) ? actin + (int64_t)(i + 1) * n * d : nullptr;
-        TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, d, Mz}, st, status)));
+        LAUNCH(K_MLP_DOWN, 2.0 * Mz * d * h * Bz,
+               e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0)) + 8.0 * n * d,
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, d, Mz}, st, status))));
       }
     }
 
     // ---- head: RMSNorm, CE pass A, reduce ----
-    rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd);
-    TRY(cudaGetLastError());
+    LAUNCH(K_RMS_FWD, 0, (4.0 + e) * n * d,
+           (rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd)));
     {
       GemmShape s{n, V, d, 1};
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E, d, 0, 1, V);
-      TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status)));
+      LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status))));
     }
-    ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status);
-    TRY(cudaGetLastError());
-    ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status);
-    TRY(cudaGetLastError());
+    LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
+           (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
+    LAUNCH(K_CE_MEAN, 0, 4.0 * n, (ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status)));
     // ---- CE pass B and dz, one vocabulary slab at a time ----
     for (int sl = 0; sl < p.nslabs; ++sl) {
       const int v0 = sl * p.Vs;
@@ -280,20 +327,22 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         GemmShape s{n, vs, d, 1};
         Operand A = opnd(z, d, 0, 1, n);
         Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
-        TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status)));
+        LAUNCH(K_CE_GRAD, 2.0 * n * vs * d, e * ((double)n * d + (double)vs * d + (double)n * vs),
+               TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status))));
       }
       {
         GemmShape s{n, d, vs, 1};
         Operand A = opnd(P, p.Vs, 0, 1, n);
         Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 0, vs);
-        TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status)));
+        LAUNCH(K_CE_DZ, 2.0 * n * d * vs, e * ((double)n * vs + (double)vs * d) + (sl > 0 ? 8.0 : 4.0) * n * d,
+               TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status))));
       }
     }
     {
       const int top = p.nM - 1;  // always dynamic
-      rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
-                                                         doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm);
-      TRY(cudaGetLastError());
+      LAUNCH(K_RMS_BWD, 0, (12.0 + 3.0 * e) * n * d,
+             (rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
+                                                                 doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm)));
     }
 
     // ---- backward, top down ----
@@ -313,8 +362,10 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         T* du = need_dx ? dU : nullptr;
         T* dw = dyn ? dUW : nullptr;
         T* dm = dyn ? dUM : nullptr;
-        if (sw) TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status)));
-        else TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status)));
+        const double fl = 2.0 * Mz * h * d * Bz;
+        const double by = e * ((double)n * d + (double)d * h * Bz + (double)n * H2 * (1 + (du ? 1 : 0) + (dw ? 2 : 0)));
+        if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status))));
+        else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status))));
       }
       if (need_dx) {  // B2: dout += dU W1
         GemmShape s{Mz, d, H2, Bz};
@@ -323,7 +374,9 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         const bool below_dyn = is_dyn(i - 1);
         T* ow = below_dyn ? doutW[(i - 1) & 1] : nullptr;
         T* om = below_dyn ? doutM[(i - 1) & 1] : nullptr;
-        TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status)));
+        LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
+               e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status))));
       }
       if (dyn) {
         T* ain = actin + (int64_t)i * n * d;
@@ -336,21 +389,26 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
           Operand A = opnd(dUW, H2, (int64_t)b * H2, 0, b);
           Operand A2 = opnd(dUM, H2, (int64_t)b * H2, 0, b);
           Operand Bx = opnd(ain, d, (int64_t)b * d, 0, b);
-          EpiUpdate<T> e{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
-          TRY((gemm<T, 2>(s, A, A2, Bx, e, st, status)));
+          EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+          LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B,
+                 (16.0 + e) * H2 * d * B + e * ((double)n * H2 * 2 + (double)n * d),
+                 TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
         }
         {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
           GemmShape s{d, h, b, B};
           Operand A = opnd(doutW[i & 1], d, (int64_t)b * d, 0, b);
           Operand A2 = opnd(doutM[i & 1], d, (int64_t)b * d, 0, b);
           Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
-          EpiUpdate<T> e{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
-                         consts, c, p.nchunks, h, 0};
-          TRY((gemm<T, 2>(s, A, A2, Bx, e, st, status)));
+          EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
+                          consts, c, p.nchunks, h, 0};
+          LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B,
+                 (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
+                 TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
         }
       }
     }
   }
+#undef LAUNCH
 #undef TRY
   return cudaSuccess;
 }
@@ -497,15 +555,17 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
+  Prof prof;
   auto enqueue = [&](cudaStream_t q) -> cudaError_t {
     if (h->cfg.precision == TTT_PREC_FP32)
-      return enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q);
-    return enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q);
+      return enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
+    return enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
   };
 
   if (!h->use_graph) {
     cudaError_t e = enqueue(st);
     if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    h->launches = prof.launches;
     return TTT_OK;
   }
   GraphKey key{batch, T, b, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, workspace, ws_bytes};
@@ -526,8 +586,56 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
     if (e != cudaSuccess) { h->exec = nullptr; set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
     h->key = key;
     h->have_key = true;
+    h->launches = prof.launches;
   }
   TTT_CUDA_TRY(cudaGraphLaunch(h->exec, st));
+  return TTT_OK;
+}
+
+ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                                const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
+                                const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
+                                void* stream, ttt_kernel_stat* stats, int32_t max_stats, int32_t* n_stats) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (!stats || !n_stats || max_stats < 0) return fail(TTT_ERR_INVALID_ARG, "stats / n_stats missing");
+  *n_stats = 0;
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
+    return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  Plan p = make_plan(h->cfg, batch, T, b);
+  if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  Prof prof;
+  prof.timing = true;
+  prof.recs.reserve(1 << 16);
+  cudaError_t e = h->cfg.precision == TTT_PREC_FP32
+                      ? enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
+                      : enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
+  if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+  TTT_CUDA_TRY(cudaStreamSynchronize(st));
+  ttt_kernel_stat agg[K_NCLASS];
+  memset(agg, 0, sizeof(agg));
+  for (const auto& r : prof.recs) {
+    float ms = 0.f;
+    TTT_CUDA_TRY(cudaEventElapsedTime(&ms, r.a, r.b));
+    ttt_kernel_stat& a = agg[r.cls];
+    a.launches += 1;
+    a.ms += ms;
+    a.flops += r.flops;
+    a.bytes += r.bytes;
+  }
+  int32_t k = 0;
+  for (int c = 0; c < K_NCLASS && k < max_stats; ++c) {
+    if (agg[c].launches == 0) continue;
+    stats[k] = agg[c];
+    snprintf(stats[k].name, sizeof(stats[k].name), "%s", kClassName[c]);
+    ++k;
+  }
+  *n_stats = k;
+  h->launches = prof.launches;
   return TTT_OK;
 }
 

@@ -24,7 +24,8 @@ MLP = {"gelu": 0, "swiglu": 1}
 PRECISION = {"fp32": 0, "bf16": 1}
 REDUCTION = {"mean": 0, "sum": 1}
 
-EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_scalar_kernels", "ttt_gemm_bf16",
+EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_profiled",
+            "ttt_scalar_kernels", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
 
@@ -41,6 +42,11 @@ class ttt_config(ctypes.Structure):
                 ("n_blocks", ctypes.c_int32), ("mlp", ctypes.c_int32), ("has_static", ctypes.c_int32),
                 ("precision", ctypes.c_int32), ("loss_reduction", ctypes.c_int32),
                 ("rms_eps", ctypes.c_float)]
+
+
+class ttt_kernel_stat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 24), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 _lib = None
@@ -63,6 +69,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_workspace_size.restype = I32
     lib.ttt_prefill.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill.restype = I32
+    lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
+                                         ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
+    lib.ttt_prefill_profiled.restype = I32
     lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
     lib.ttt_scalar_kernels.restype = I32
     I64 = ctypes.c_int64
@@ -231,6 +240,23 @@ class Handle:
                                           _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(chunk_loss),
                                           _ptr(ws), ws.numel(), _stream_ptr(stream)), "ttt_prefill")
         return chunk_loss
+
+    def prefill_profiled(self, hidden, tokens, W, M, eta, beta, gamma, b: int, stream=None):
+        """ttt_prefill_profiled: same results as prefill (W, M updated in place),
+        plus per-kernel-class stats.  Returns (chunk_loss, [dict, ...])."""
+        B, T, d = hidden.shape
+        nc = T // b if b > 0 else 0
+        loss = torch.empty((B, nc), dtype=torch.float32, device=self.device)
+        ws = self.workspace(B, T, b)
+        stats = (ttt_kernel_stat * 32)()
+        n = ctypes.c_int32()
+        _check(load_library().ttt_prefill_profiled(self._h, B, T, b, _ptr(hidden), _ptr(tokens), _ptr(W), _ptr(M),
+                                                   _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(loss), _ptr(ws),
+                                                   ws.numel(), _stream_ptr(stream), stats, 32, ctypes.byref(n)),
+               "ttt_prefill_profiled")
+        out = [dict(name=stats[i].name.decode(), launches=stats[i].launches, ms=stats[i].ms,
+                    flops=stats[i].flops, bytes=stats[i].bytes) for i in range(n.value)]
+        return loss, out
 
     def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None):
         """End-to-end call on HOST tensors: copies the inputs to the device,
