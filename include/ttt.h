@@ -138,6 +138,27 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
                        const float* eta, const float* beta, const float* gamma,
                        float* chunk_loss, void* workspace, size_t ws_bytes, void* stream);
 
+/* ttt_prefill without a caller-provided workspace and without allocating:
+ * for callers that must not allocate device memory while they run (memory
+ * budgeted once at start-up, a host that owns the allocator, or a loop that
+ * cannot afford the implicit device synchronisation of cudaMalloc/cudaFree).
+ * The pages have no counterpart; this is a deployment variant of ttt_prefill.
+ * Same arguments and results as ttt_prefill minus workspace/ws_bytes; the
+ * caller still passes every input and output.  Its scratch is a 16 MiB
+ * file-scope device array inside the library, held by every GPU that loads
+ * the library until the process exits; calls needing more scratch than that
+ * (ttt_workspace_size() > 16 MiB) return TTT_ERR_WORKSPACE with the sizes in
+ * ttt_last_error().  Launches run directly on `stream` (no CUDA graph).  The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array: calls whose work
+ * overlaps on the GPU (other streams, other threads, other handles) race and
+ * corrupt each other's results; serialise them.  Nothing in the array needs
+ * to start at zero (every buffer is written before it is read in a call). */
+ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                               const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
+                               const float* gamma, float* chunk_loss, void* stream);
+
 /* Per-kernel-class record of one profiled prefill. */
 typedef struct ttt_kernel_stat {
   char name[24];     /* kernel class, e.g. "agg_update", "mlp_up", "ce_logits_lse" */

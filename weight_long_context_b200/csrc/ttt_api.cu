@@ -449,6 +449,39 @@ static ttt_status check_shape(const ttt_handle* h, int batch, int T, int b) {
 using namespace ttt;
 
 // ---------------------------------------------------------------------------
+// Allocation-free prefill: scratch in a file-scope device array.
+//
+// For callers that must not allocate device memory while they run: programs
+// whose device memory is budgeted once at start-up, hosts that own the
+// allocator and forbid raw cudaMalloc, and latency-critical loops where the
+// implicit device synchronisation of cudaMalloc / cudaFree is not acceptable.
+// The scratch is kNoAllocScratchBytes of static device memory that every GPU
+// loading this library holds until the process exits.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_ptr[64] = {};   // device address of the scratch, per device ordinal
+
+// Device address of the scratch for the current device.  In host code the
+// array's name is only a stand-in, so the address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static ttt_status noalloc_scratch(void** out) {
+  int dev = 0;
+  TTT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(TTT_ERR_UNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    TTT_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TTT_OK;
+}
+
+// ---------------------------------------------------------------------------
 // C ABI
 // ---------------------------------------------------------------------------
 extern "C" {
@@ -646,6 +679,40 @@ ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* 
   if (batch == 0 || T == 0) return TTT_OK;
   if (!eta || !beta || !gamma || !KW || !KM || !consts) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
   TTT_CUDA_TRY(launch_scalar_scan(eta, beta, gamma, batch, T, b, KW, KM, consts, static_cast<cudaStream_t>(stream)));
+  return TTT_OK;
+}
+
+ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                               const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
+                               const float* gamma, float* chunk_loss, void* stream) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
+    return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (reinterpret_cast<uintptr_t>(hidden) % 16) return fail(TTT_ERR_INVALID_ARG, "hidden must be 16-byte aligned");
+  Plan p = make_plan(h->cfg, batch, T, b);
+  if (p.total > kNoAllocScratchBytes) {
+    static thread_local char msg[160];
+    snprintf(msg, sizeof(msg), "ttt_prefill_noalloc needs %zu bytes of scratch; its static scratch holds %zu bytes",
+             p.total, kNoAllocScratchBytes);
+    return fail(TTT_ERR_WORKSPACE, msg);
+  }
+  int dev = 0;
+  TTT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != h->device) return fail(TTT_ERR_INVALID_ARG, "the current device is not the handle's device");
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != TTT_OK) return s;
+  // Every buffer of the plan is written before it is read within the call,
+  // so the scratch needs no clearing between calls.
+  Prof prof;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(scratch);
+  cudaError_t e = h->cfg.precision == TTT_PREC_FP32
+                      ? enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
+                      : enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
+  if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
   return TTT_OK;
 }
 

@@ -24,7 +24,8 @@ MLP = {"gelu": 0, "swiglu": 1}
 PRECISION = {"fp32": 0, "bf16": 1}
 REDUCTION = {"mean": 0, "sum": 1}
 
-EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_profiled",
+EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
+            "ttt_prefill_profiled",
             "ttt_scalar_kernels", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
@@ -69,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_workspace_size.restype = I32
     lib.ttt_prefill.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill.restype = I32
+    lib.ttt_prefill_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P]
+    lib.ttt_prefill_noalloc.restype = I32
     lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
     lib.ttt_prefill_profiled.restype = I32
