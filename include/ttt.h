@@ -195,10 +195,13 @@ ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* 
  * (row-major, leading dimension ldd, batch stride strideD, in elements).
  * A(m, k) is at A + z*strideA + (a_kmajor ? m*lda + k : k*lda + m); same for
  * B(n, k).  lda, ldb, strideA, strideB: multiples of 8 elements; strides are
- * nonzero when batch > 1.  Asynchronous on `stream`. */
+ * nonzero when batch > 1.  workspace (256-byte aligned, >= 1 MiB, or NULL)
+ * lets the engine split K across CTA pairs when the output has too few tiles
+ * to fill the GPU; its contents are not preserved.  Asynchronous on `stream`. */
 ttt_status ttt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
                          int64_t strideA, int32_t a_kmajor, const void* B, int64_t ldb, int64_t strideB,
-                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* stream);
+                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* workspace,
+                         size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, return the first device-side error recorded by this
  * handle's kernels since the last call (TTT_OK if none) and clear it. */

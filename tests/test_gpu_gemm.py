@@ -43,3 +43,27 @@ def test_gemm_rejects_unaligned_strides(dev):
     with pytest.raises(ttt.TTTError) as ei:
         ttt.ttt_gemm_bf16(A, B, False, True)
     assert ei.value.code == 3
+
+
+SPLITK = [(1024, 2048, 5632, 1), (1024, 2048, 11264, 1), (512, 520, 4096, 2), (296, 264, 1000, 1)]
+
+
+@pytest.mark.parametrize("b_k", [True, False])
+@pytest.mark.parametrize("shape", SPLITK, ids=[f"{m}x{n}x{k}b{z}" for m, n, k, z in SPLITK])
+def test_gemm_split_k(dev, shape, b_k):
+    """With a workspace the engine may split K across CTA pairs and reduce the
+    fp32 partials in a fixed order: same result as without, bit for bit."""
+    from weight_long_context_b200 import ttt
+    M, N, K, Z = shape
+    g = torch.Generator(device="cpu").manual_seed(M + N + K)
+    A = torch.randn(Z, M, K, generator=g).to(dev, torch.bfloat16)
+    B = torch.randn(Z, N, K, generator=g).to(dev, torch.bfloat16)
+    Bin = B if b_k else B.transpose(1, 2).contiguous()
+    ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    D = ttt.ttt_gemm_bf16(A, Bin, True, b_k, workspace=ws)
+    D2 = ttt.ttt_gemm_bf16(A, Bin, True, b_k, workspace=ws)
+    torch.cuda.synchronize()
+    ref = torch.matmul(A.float(), B.float().transpose(1, 2))
+    err = (D - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 1e-5, err
+    assert torch.equal(D, D2)

@@ -152,7 +152,10 @@ struct EpiF1 {
 };
 
 // ---------------------------------------------------------------------------
-// F2: residual add.  resid += A W2^T; optional operand copy of the new stream.
+// F2: residual add.  resid += A W2^T; optional operand copy of the new stream
+// and, when the next MLP is dynamic, its K-scaled negated copies
+// -kscale K_W x and -kscale K_M x: the B operands of that MLP's first-matrix
+// aggregation (sum_t dU_t (x) (-K_t x_t) = sum_t K_t G_t).
 // ---------------------------------------------------------------------------
 template <typename T>
 struct EpiResid {
@@ -160,37 +163,50 @@ struct EpiResid {
   using RowState = NoRowState;
   float* resid;   // [rows, d]
   T* act_next;    // [rows, d] or nullptr
+  T* aw_next;     // [rows, d] or nullptr
+  T* am_next;
+  const float* KW;
+  const float* KM;
+  float kscale;
+  TokenMap tm;
   int d;
   int rows_per_z;
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
     int64_t grow = (int64_t)z * rows_per_z + r;
+    float kw = 0.f, km = 0.f;
+    if (aw_next) {
+      int64_t ti = tm.index((int)grow);
+      kw = -KW[ti] * kscale;
+      km = -KM[ti] * kscale;
+    }
     float* p = resid + grow * d + c0;
-    T* q = act_next ? act_next + grow * d + c0 : nullptr;
+    const int64_t o = grow * d + c0;
     if (nv == 32) {
       float x[32];
       vld<32>(p, x);
 #pragma unroll
       for (int j = 0; j < 32; ++j) x[j] += v[j];
       vst<32>(p, x);
-      if (q) vst<32>(q, x);
+      if (act_next) vst<32>(act_next + o, x);
+      if (aw_next) { vst_scaled<32>(aw_next + o, x, kw); vst_scaled<32>(am_next + o, x, km); }
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) if (j < nv) {
         float x = p[j] + v[j];
         p[j] = x;
-        if (q) q[j] = from_f<T>(x);
+        if (act_next) act_next[o + j] = from_f<T>(x);
+        if (aw_next) { aw_next[o + j] = from_f<T>(kw * x); am_next[o + j] = from_f<T>(km * x); }
       }
     }
   }
 };
 
 // ---------------------------------------------------------------------------
-// B1: dA = dOut W2 ([n,h]); dU = dA * factor at the U positions; for a
-// dynamic MLP also the K-scaled negated copies -K_W dU and -K_M dU that are
-// the A operands of the aggregation (so the aggregation GEMM yields
-// sum_t K_t G_t directly, G_t being the negative gradient).
+// B1: dA = dOut W2 ([n,h]); dU = dA * factor at the U positions.  dU feeds
+// the dX GEMM and, for a dynamic MLP, is the shared A operand of its
+// first-matrix aggregation.
 // SwiGLU: the 32 dA columns [c0, c0+32) own the 64 contiguous interleaved
 // positions [2 c0, 2 c0 + 64) (gate/up groups of 16).
 // ---------------------------------------------------------------------------
@@ -199,13 +215,7 @@ struct EpiB1 {
   static constexpr bool kFixedHeadTile = false;
   using RowState = NoRowState;
   const T* fac;   // [rows, H2]
-  T* dU;          // [rows, H2] or nullptr
-  T* dUW;         // [rows, H2] or nullptr (static MLP)
-  T* dUM;
-  const float* KW;
-  const float* KM;
-  float kscale;   // 1/b (mean reduction) or 1 (sum)
-  TokenMap tm;
+  T* dU;          // [rows, H2]
   int h;
   int rows_per_z;
   __device__ void row_begin(RowState&, int, int) const {}
@@ -213,12 +223,6 @@ struct EpiB1 {
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
     int64_t grow = (int64_t)z * rows_per_z + r;
     const int64_t H2 = SWIGLU ? 2 * (int64_t)h : h;
-    float kw = 0.f, km = 0.f;
-    if (dUW) {
-      int64_t ti = tm.index((int)grow);
-      kw = -KW[ti] * kscale;
-      km = -KM[ti] * kscale;
-    }
     const int64_t ob = grow * H2;
     if (!SWIGLU) {
       if (nv == 32) {
@@ -226,15 +230,12 @@ struct EpiB1 {
         vld<32>(fac + ob + c0, f);
 #pragma unroll
         for (int j = 0; j < 32; ++j) du[j] = v[j] * f[j];
-        if (dU) vst<32>(dU + ob + c0, du);
-        if (dUW) { vst_scaled<32>(dUW + ob + c0, du, kw); vst_scaled<32>(dUM + ob + c0, du, km); }
+        vst<32>(dU + ob + c0, du);
       } else {
-  #pragma unroll
-      for (int j = 0; j < 32; ++j) if (j < nv) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) if (j < nv) {
           int c = c0 + j;
-          float du = v[j] * to_f<T>(fac[ob + c]);
-          if (dU) dU[ob + c] = from_f<T>(du);
-          if (dUW) { dUW[ob + c] = from_f<T>(kw * du); dUM[ob + c] = from_f<T>(km * du); }
+          dU[ob + c] = from_f<T>(v[j] * to_f<T>(fac[ob + c]));
         }
       }
     } else {
@@ -249,13 +250,8 @@ struct EpiB1 {
         du[gi] = v[j] * f[gi];
         du[gi + 16] = v[j] * f[gi + 16];
       }
-      if (nv == 32) {
-        if (dU) vst<64>(dU + p0, du);
-        if (dUW) { vst_scaled<64>(dUW + p0, du, kw); vst_scaled<64>(dUM + p0, du, km); }
-      } else {
-        if (dU) vst<32>(dU + p0, du);
-        if (dUW) { vst_scaled<32>(dUW + p0, du, kw); vst_scaled<32>(dUM + p0, du, km); }
-      }
+      if (nv == 32) vst<64>(dU + p0, du);
+      else vst<32>(dU + p0, du);
     }
   }
 };
@@ -421,8 +417,12 @@ struct EpiStoreBatched {
   __device__ void row_end(RowState&, int, int, int) const {}
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
     float* o = out + (int64_t)z * zstride + (int64_t)r * ld + c0;
+    if (nv == 32 && ((reinterpret_cast<uintptr_t>(o) & 15) == 0)) {
+      vst<32>(o, v);
+    } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) if (j < nv) o[j] = v[j];
+      for (int j = 0; j < 32; ++j) if (j < nv) o[j] = v[j];
+    }
   }
 };
 

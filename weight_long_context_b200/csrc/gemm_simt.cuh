@@ -24,9 +24,12 @@ __device__ __forceinline__ float simt_load(const Operand& op, int z, int mn, int
   return to_f<T>(p[off]);
 }
 
+// NACC == 2: dualb = 0 -> acc_j = A_j B^T (A2 is a second A operand);
+// dualb = 1 -> acc_j = A B_j^T (A2 carries the second B operand, staged in the
+// otherwise unused second A tile).
 template <typename T, int NACC, class Epi>
 __global__ void __launch_bounds__(simt::THREADS)
-gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi) {
+gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi, int dualb) {
   using namespace simt;
   __shared__ float As[NACC][BK][BM + 1];
   __shared__ float Bs[BK][BN + 1];
@@ -53,24 +56,28 @@ gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi) {
       int mm, kk;
       if (A.kmajor) { mm = idx / BK; kk = idx % BK; } else { kk = idx / BM; mm = idx % BM; }
       As[0][kk][mm] = simt_load<T>(A, z, m0 + mm, k0 + kk, s.M, s.K);
-      if (NACC == 2) As[NACC - 1][kk][mm] = simt_load<T>(A2, z, m0 + mm, k0 + kk, s.M, s.K);
+      if (NACC == 2 && !dualb) As[NACC - 1][kk][mm] = simt_load<T>(A2, z, m0 + mm, k0 + kk, s.M, s.K);
       int nn;
       if (B.kmajor) { nn = idx / BK; kk = idx % BK; } else { kk = idx / BN; nn = idx % BN; }
       Bs[kk][nn] = simt_load<T>(B, z, n0 + nn, k0 + kk, s.N, s.K);
+      if (NACC == 2 && dualb) As[NACC - 1][kk][nn] = simt_load<T>(A2, z, n0 + nn, k0 + kk, s.N, s.K);
     }
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
-      float b[4];
+      float b[NACC][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx * 4 + j];
+      for (int j = 0; j < 4; ++j) {
+        b[0][j] = Bs[kk][tx * 4 + j];
+        if (NACC == 2) b[NACC - 1][j] = dualb ? As[NACC - 1][kk][tx * 4 + j] : b[0][j];
+      }
 #pragma unroll
       for (int a = 0; a < NACC; ++a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float av = As[a][kk][ty * 4 + i];
+          float av = As[(NACC == 2 && dualb) ? 0 : a][kk][ty * 4 + i];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[a][i][j] = fmaf(av, b[j], acc[a][i][j]);
+          for (int j = 0; j < 4; ++j) acc[a][i][j] = fmaf(av, b[a][j], acc[a][i][j]);
         }
       }
     }
@@ -110,10 +117,10 @@ gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi) {
 
 template <typename T, int NACC, class Epi>
 cudaError_t launch_gemm_simt(const GemmShape& s, const Operand& A, const Operand& A2,
-                             const Operand& B, const Epi& epi, cudaStream_t st) {
+                             const Operand& B, const Epi& epi, cudaStream_t st, int dualb = 0) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0) return cudaSuccess;
   dim3 grid((s.N + simt::BN - 1) / simt::BN, (s.M + simt::BM - 1) / simt::BM, s.batch);
-  gemm_simt_kernel<T, NACC, Epi><<<grid, simt::THREADS, 0, st>>>(s, A, A2, B, epi);
+  gemm_simt_kernel<T, NACC, Epi><<<grid, simt::THREADS, 0, st>>>(s, A, A2, B, epi, dualb);
   return cudaGetLastError();
 }
 

@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+
 #include "common.cuh"
 #include "gemm_types.cuh"
 
@@ -176,8 +178,17 @@ struct Cfg {
 struct TcParams {
   GemmShape s;
   int a_mn, b_mn;       // 1 = MN-major operand
+  // Dual accumulators (NACC = 2, BN = 128, 1-SM kernel): dualb = 0 shares B
+  // (acc_j += A_j B^T, maps A, A2, B); dualb = 1 shares A (acc_j += A B_j^T,
+  // maps A, B, and A2 holding B_2).  Both use three 16 KiB slots per stage.
+  int dualb;
   int tiles_m, tiles_n, num_tiles, num_kb;
   int* status;
+  // Split-K (pair kernel): unit u = tile * splits + ks covers k-blocks
+  // [ks * kb_per_split, min(num_kb, (ks + 1) * kb_per_split)).
+  int splits, kb_per_split;
+  float* partial;   // [num_tiles][splits][2 CTAs][128 rows][BN] fp32 when splits > 1
+  int* counters;    // [num_tiles][2 CTAs][EPI_WARPS], zero on entry, left zero on exit
 };
 
 template <int NACC, int BN, class Epi>
@@ -232,21 +243,43 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           uint8_t* sb = sa + NACC * C::A_BYTES;
           mbar_expect_tx(&full[st], C::STAGE_BYTES);
           const int k0 = kb * BK;
-          if (!p.a_mn) {
-            tma_load_3d(sa, &mapA, &full[st], k0, m0, z);
-            if (NACC == 2) tma_load_3d(sa + C::A_BYTES, &mapA2, &full[st], k0, m0, z);
-          } else {
+          if (NACC == 2 && p.dualb) {
+            // slot 0: A, slot 1: B_1, slot 2: B_2 (BN == BM: all slots 16 KiB)
+            if (!p.a_mn) {
+              tma_load_3d(sa, &mapA, &full[st], k0, m0, z);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BM / 64; ++j) {
-              tma_load_3d(sa + j * 8192, &mapA, &full[st], m0 + 64 * j, k0, z);
-              if (NACC == 2) tma_load_3d(sa + C::A_BYTES + j * 8192, &mapA2, &full[st], m0 + 64 * j, k0, z);
+              for (int j = 0; j < BM / 64; ++j) tma_load_3d(sa + j * 8192, &mapA, &full[st], m0 + 64 * j, k0, z);
             }
-          }
-          if (!p.b_mn) {
-            tma_load_3d(sb, &mapB, &full[st], k0, n0, z);
-          } else {
+            uint8_t* sb1 = sa + C::A_BYTES;
+            uint8_t* sb2 = sb1 + C::B_BYTES;
+            if (!p.b_mn) {
+              tma_load_3d(sb1, &mapB, &full[st], k0, n0, z);
+              tma_load_3d(sb2, &mapA2, &full[st], k0, n0, z);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, &mapB, &full[st], n0 + 64 * j, k0, z);
+              for (int j = 0; j < BN / 64; ++j) {
+                tma_load_3d(sb1 + j * 8192, &mapB, &full[st], n0 + 64 * j, k0, z);
+                tma_load_3d(sb2 + j * 8192, &mapA2, &full[st], n0 + 64 * j, k0, z);
+              }
+            }
+          } else {
+            if (!p.a_mn) {
+              tma_load_3d(sa, &mapA, &full[st], k0, m0, z);
+              if (NACC == 2) tma_load_3d(sa + C::A_BYTES, &mapA2, &full[st], k0, m0, z);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BM / 64; ++j) {
+                tma_load_3d(sa + j * 8192, &mapA, &full[st], m0 + 64 * j, k0, z);
+                if (NACC == 2) tma_load_3d(sa + C::A_BYTES + j * 8192, &mapA2, &full[st], m0 + 64 * j, k0, z);
+              }
+            }
+            if (!p.b_mn) {
+              tma_load_3d(sb, &mapB, &full[st], k0, n0, z);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, &mapB, &full[st], n0 + 64 * j, k0, z);
+            }
           }
         }
       }
@@ -279,13 +312,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           for (int kk = 0; kk < BK / 16; ++kk) {
             // K-major: advance 16 elements = 32 bytes inside the swizzled row.
             // MN-major: advance 16 K-rows = two 8-row groups of 1024 bytes.
-            const uint64_t bdesc = p.b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
 #pragma unroll
             for (int a = 0; a < NACC; ++a) {
-              const uint32_t abase = sa + a * C::A_BYTES;
+              const bool db = NACC == 2 && p.dualb;
+              const uint32_t abase = db ? sa : sa + a * C::A_BYTES;
+              const uint32_t bbase = db ? sa + C::A_BYTES + a * C::B_BYTES : sb;
               const uint64_t adesc = p.a_mn ? smem_desc_sw128(abase + kk * 2048, 8192, 1024)
                                             : smem_desc_sw128(abase + kk * 32, 16, 1024);
+              const uint64_t bdesc = p.b_mn ? smem_desc_sw128(bbase + kk * 2048, 8192, 1024)
+                                            : smem_desc_sw128(bbase + kk * 32, 16, 1024);
               mma_bf16(d0 + a * BN, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
             }
           }
@@ -335,11 +370,336 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair (2-SM) variant: tcgen05.mma.cta_group::2, M = 256 per pair.
+//
+// Each CTA of a cluster pair holds 128 rows of A and BN/2 columns of B per
+// stage (no TMA multicast: each CTA loads its own halves); the leader CTA
+// (rank 0) issues M=256 x N=BN MMAs that read both CTAs' shared memory and
+// write each CTA's 128-row slice of the accumulator into that CTA's TMEM.
+// Per SM this halves the B bytes per FLOP against the 1-SM kernel (a 256x256
+// pair tile needs 64 B/clk of operand feed per SM instead of 96 B/clk).
+// Barriers: both CTAs' TMA loads complete on the leader's "full" barrier
+// (the leader arms it with both CTAs' bytes); the leader's tcgen05.commit
+// multicasts "empty" and "accumulator full" to both CTAs; both epilogues
+// release the leader's "accumulator empty" barrier (remote arrive).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load whose completion is signalled on a barrier that may live in the
+// peer CTA of the pair (cluster address); no multicast.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this shared offset in both CTAs of the pair once
+// the leader's prior MMAs are complete.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t mask = 0x3) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_m256(int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+template <int NACC, int BN>
+struct Cfg2 {
+  static constexpr int A_BYTES = BM * BK * 2;            // this CTA's 128 rows
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;      // this CTA's BN/2 columns
+  static constexpr int STAGE_BYTES = NACC * A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * NACC * BN;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(BN % 128 == 0, "each CTA loads whole 64-column boxes of B");
+};
+
+template <int NACC, int BN, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
+                const __grid_constant__ CUtensorMap mapB, const TcParams p, const Epi epi) {
+  using C = Cfg2<NACC, BN>;
+  constexpr int HBN = BN / 2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2 * 32 * EPI_WARPS); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const GemmShape& s = p.s;
+
+  if (warp == 0) {
+    // ------------------------------ producer (both CTAs) ------------------------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      const int num_units = p.num_tiles * p.splits;
+      for (int u = pair; u < num_units && ok; u += npairs) {
+        const int t = u / p.splits, ks = u - t * p.splits;
+        const int tm = t % p.tiles_m;
+        const int rest = t / p.tiles_m;
+        const int tn = rest % p.tiles_n;
+        const int z = rest / p.tiles_n;
+        const int m0 = tm * 2 * BM + (int)rank * BM;     // this CTA's 128 rows
+        const int n0 = tn * BN + (int)rank * HBN;        // this CTA's BN/2 columns
+        const int kb0 = ks * p.kb_per_split;
+        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* sa = smem + st * C::STAGE_BYTES;
+          uint8_t* sb = sa + NACC * C::A_BYTES;
+          if (leader) mbar_expect_tx(&full[st], 2 * C::STAGE_BYTES);
+          const uint32_t fb = mapa_shared(smem_u32(&full[st]), 0);
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tma_load_3d_pair(sa, &mapA, fb, k0, m0, z);
+            if (NACC == 2) tma_load_3d_pair(sa + C::A_BYTES, &mapA2, fb, k0, m0, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j) {
+              tma_load_3d_pair(sa + j * 8192, &mapA, fb, m0 + 64 * j, k0, z);
+              if (NACC == 2) tma_load_3d_pair(sa + C::A_BYTES + j * 8192, &mapA2, fb, m0 + 64 * j, k0, z);
+            }
+          }
+          if (!p.b_mn) {
+            tma_load_3d_pair(sb, &mapB, fb, k0, n0, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < HBN / 64; ++j) tma_load_3d_pair(sb + j * 8192, &mapB, fb, n0 + 64 * j, k0, z);
+          }
+        }
+      }
+      if (leader) {
+        const uint32_t issued = it;
+        const uint32_t first = issued > (uint32_t)C::STAGES ? issued - C::STAGES : 0;
+        for (uint32_t j = first; j < issued; ++j)
+          mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader) ------------------------------
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_m256(BN, p.a_mn, p.b_mn);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      const int num_units = p.num_tiles * p.splits;
+      for (int u = pair; u < num_units && ok; u += npairs, ++tcount) {
+        const int ks = u % p.splits;
+        const int kb0 = ks * p.kb_per_split;
+        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+        const uint32_t buf = tcount & 1u;
+        const uint32_t aph = (tcount >> 1) & 1u;
+        if (!mbar_wait(&tempty[buf], aph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * (NACC * BN);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
+          const uint32_t sb = sa + NACC * C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = p.b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
+#pragma unroll
+            for (int a = 0; a < NACC; ++a) {
+              const uint32_t abase = sa + a * C::A_BYTES;
+              const uint64_t adesc = p.a_mn ? smem_desc_sw128(abase + kk * 2048, 8192, 1024)
+                                            : smem_desc_sw128(abase + kk * 32, 16, 1024);
+              mma_bf16_pair(d0 + a * BN, adesc, bdesc, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit_pair(&empty[st]);
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[buf]);
+      }
+      mma_commit_pair(drain, 0x1);   // the leader's own barrier only
+      mbar_wait(drain, 0, nullptr, p.status);
+    }
+  } else {
+    // ------------------------------ epilogue (both CTAs) ------------------------------
+    const int q = warp & 3;
+    const int part = (warp - 2) >> 2;
+    constexpr int PART_COLS = BN / EPI_PARTS;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    uint32_t tcount = 0;
+    const int num_units = p.num_tiles * p.splits;
+    for (int u = pair; u < num_units; u += npairs, ++tcount) {
+      const int t = u / p.splits, ks = u - t * p.splits;
+      const int tm = t % p.tiles_m;
+      const int rest = t / p.tiles_m;
+      const int tn = rest % p.tiles_n;
+      const int z = rest / p.tiles_n;
+      const uint32_t buf = tcount & 1u;
+      const uint32_t aph = (tcount >> 1) & 1u;
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
+      if (!ready) break;
+      tc_fence_after();
+      const int r = tm * 2 * BM + (int)rank * BM + row_in_tile;
+      const bool row_ok = r < s.M;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
+      if (p.splits == 1) {
+        typename Epi::RowState rs;
+        if (row_ok) epi.row_begin(rs, z, r);
+#pragma unroll 1
+        for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
+          float v[32], v2[32];
+          tmem_ld32(tbase + c, v);
+          if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
+          const int c0 = tn * BN + c;
+          if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+        }
+        if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+        tc_fence_before();
+        mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+      } else {
+        // Split-K: park this split's fp32 partial, free the accumulator, and
+        // let the last split to arrive sum all partials in split order.
+        // Partial layout is warp-major: [unit][cta][epi warp][span][8 float4][lane],
+        // so each warp store / load instruction covers 512 contiguous bytes.
+        const size_t slab = (size_t)BM * BN;                 // one CTA's partial tile
+        const int ew = warp - 2;
+        float4* mine = reinterpret_cast<float4*>(p.partial + ((size_t)(t * p.splits + ks) * 2 + rank) * slab) +
+                       (size_t)ew * (PART_COLS / 4) * 32 + lane;
+#pragma unroll 1
+        for (int c = part * PART_COLS, sp = 0; c < (part + 1) * PART_COLS; c += 32, ++sp) {
+          float v[32];
+          tmem_ld32(tbase + c, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            mine[(sp * 8 + i) * 32] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+        // One arrival counter per epilogue-warp region (32 rows x PART_COLS):
+        // no barrier across warps, so an aborting warp cannot strand others.
+        int* ctr = p.counters + ((size_t)t * 2 + rank) * EPI_WARPS + (warp - 2);
+        __threadfence();
+        __syncwarp();
+        int old = 0;
+        if (lane == 0) old = atomicAdd(ctr, 1);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old == p.splits - 1) {
+          __threadfence();
+          typename Epi::RowState rs;
+          if (row_ok) epi.row_begin(rs, z, r);
+          const float4* base = reinterpret_cast<const float4*>(p.partial + ((size_t)t * p.splits * 2 + rank) * slab) +
+                               (size_t)ew * (PART_COLS / 4) * 32 + lane;
+#pragma unroll 1
+          for (int c = part * PART_COLS, sp = 0; c < (part + 1) * PART_COLS; c += 32, ++sp) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            for (int k2 = 0; k2 < p.splits; ++k2) {
+              const float4* src = base + (size_t)k2 * 2 * (slab / 4) + sp * 8 * 32;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 x = __ldcg(src + i * 32);
+                v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
+              }
+            }
+            const int c0 = tn * BN + c;
+            if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
+          }
+          if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+          __syncwarp();
+          if (lane == 0) *ctr = 0;
+        }
+      }
+    }
+  }
+
+  // On an abort, give copies issued by either CTA time to land before the
+  // pair synchronises and releases its shared memory and TMEM.
+  if (*abort_flag) {
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 200000ull) {}
+  }
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -403,7 +763,8 @@ inline cudaError_t make_operand_map(CUtensorMap* m, const Operand& op, int mn_ex
 
 template <int NACC, int BN, class Epi>
 cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
-                      cudaStream_t st, int* status) {
+                      cudaStream_t st, int* status, int dualb = 0) {
+  static_assert(NACC == 1 || BN == BM, "dual accumulators use equal A and B slots");
   using C = Cfg<NACC, BN>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -421,8 +782,10 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   e = make_operand_map(&ma, A, s.M, s.K, s.batch, BM);
   if (e != cudaSuccess) return e;
   if (NACC == 2) {
-    e = make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
+    // dual-B: the second operand is a B (N extent, B major-ness)
+    e = dualb ? make_operand_map(&ma2, A2, s.N, s.K, s.batch, BN) : make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
     if (e != cudaSuccess) return e;
+    if (dualb && A2.kmajor != B.kmajor) return cudaErrorInvalidValue;
   } else {
     ma2 = ma;
   }
@@ -430,6 +793,7 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   if (e != cudaSuccess) return e;
   TcParams p;
   p.s = s;
+  p.dualb = dualb;
   p.a_mn = A.kmajor ? 0 : 1;
   p.b_mn = B.kmajor ? 0 : 1;
   p.tiles_m = (s.M + BM - 1) / BM;
@@ -437,6 +801,10 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
   p.num_kb = (s.K + BK - 1) / BK;
   p.status = status;
+  p.splits = 1;
+  p.kb_per_split = p.num_kb;
+  p.partial = nullptr;
+  p.counters = nullptr;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
   gemm_tc_kernel<NACC, BN, Epi><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
@@ -453,18 +821,149 @@ inline double tile_efficiency(const GemmShape& s, int bn) {
   return (double)tiles / (double)(waves * sms) * (bn == 128 ? 0.78 : 1.0);
 }
 
+// Split count for a pair-kernel GEMM: minimise waves x (k-blocks per split +
+// a fixed cost for parking and reducing a partial), with no empty split and
+// within the partial-tile scratch.
+inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("TTT_GEMM_SPLITS");   // tuning knob: force a split count
+    forced = e ? atoi(e) : 0;
+  }
+  if (forced > 0) {
+    const int kbps = (num_kb + forced - 1) / forced;
+    const int s_eff = (num_kb + kbps - 1) / kbps;
+    const bool fits = forced == 1 || (ss.partial && ss.counters &&
+                                      (size_t)tiles * s_eff * 2 * BM * 256 * sizeof(float) <= ss.partial_bytes &&
+                                      (size_t)tiles * 2 * EPI_WARPS <= ss.counter_count);
+    return fits ? s_eff : 1;
+  }
+  const int pairs = num_sms() / 2;
+  // Measured on B200: splitting pays only when unsplit tiles leave most pairs
+  // idle; with 1-2 waves of tiles the partial round trip costs more than the
+  // quantisation it removes.
+  if (tiles >= (long)(0.6 * pairs)) return 1;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int S = 1; S <= 8 && S <= num_kb; ++S) {
+    const int kbps = (num_kb + S - 1) / S;
+    const int s_eff = (num_kb + kbps - 1) / kbps;
+    if (s_eff != S) continue;
+    if (S > 1) {
+      if (!ss.partial || !ss.counters) break;
+      if ((size_t)tiles * S * 2 * BM * 256 * sizeof(float) > ss.partial_bytes) break;
+      if ((size_t)tiles * 2 * EPI_WARPS > ss.counter_count) break;
+    }
+    const long units = tiles * S;
+    const long waves = (units + pairs - 1) / pairs;
+    const double cost = (double)waves * (kbps + (S > 1 ? 4 : 0));
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = S; }
+  }
+  return best;
+}
+
+template <int NACC, int BN, class Epi>
+cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
+                       cudaStream_t st, int* status, const SplitScratch& ss = SplitScratch()) {
+  using C = Cfg2<NACC, BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<NACC, BN, Epi>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if ((A.batch_stride == 0 || B.batch_stride == 0) && s.batch > 1) return cudaErrorInvalidValue;
+  CUtensorMap ma, ma2, mb;
+  cudaError_t e = make_operand_map(&ma, A, s.M, s.K, s.batch, BM);
+  if (e != cudaSuccess) return e;
+  if (NACC == 2) {
+    e = make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
+    if (e != cudaSuccess) return e;
+  } else {
+    ma2 = ma;
+  }
+  e = make_operand_map(&mb, B, s.N, s.K, s.batch, BN / 2);
+  if (e != cudaSuccess) return e;
+  TcParams p;
+  p.s = s;
+  p.dualb = 0;
+  p.a_mn = A.kmajor ? 0 : 1;
+  p.b_mn = B.kmajor ? 0 : 1;
+  p.tiles_m = (s.M + 2 * BM - 1) / (2 * BM);
+  p.tiles_n = (s.N + BN - 1) / BN;
+  p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
+  p.num_kb = (s.K + BK - 1) / BK;
+  p.status = status;
+  p.splits = (NACC == 1 && BN == 256) ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
+  p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
+  p.partial = ss.partial;
+  p.counters = ss.counters;
+  const int pairs = num_sms() / 2;
+  const int units = p.num_tiles * p.splits;
+  const int grid = 2 * (units < pairs ? units : pairs);
+  gemm_tc2_kernel<NACC, BN, Epi><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
+  return cudaGetLastError();
+}
+
+// 0: 1-SM kernel, 1: CTA-pair kernel (env TTT_GEMM_PAIR=0 forces 1-SM, for A/B timing).
+inline int pair_mode() {
+  static int m = -1;
+  if (m < 0) {
+    const char* e = getenv("TTT_GEMM_PAIR");
+    m = (e && e[0] == '0') ? 0 : 1;
+  }
+  return m;
+}
+
+// Pair tiles (256 x 256): fraction of the pairs kept busy; the pair kernel
+// needs 2/3 of the operand bytes per FLOP of the 1-SM 128x256 tile.
+inline double tile_efficiency2(const GemmShape& s) {
+  const int pairs = num_sms() / 2;
+  const long tiles = (long)((s.M + 2 * BM - 1) / (2 * BM)) * ((s.N + 255) / 256) * s.batch;
+  const long waves = (tiles + pairs - 1) / pairs;
+  return (double)tiles / (double)(waves * pairs);
+}
+
 template <int NACC, class Epi>
 cudaError_t launch_gemm_tc(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B,
-                           const Epi& epi, cudaStream_t st, int* status) {
+                           const Epi& epi, cudaStream_t st, int* status, const SplitScratch& ss = SplitScratch()) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0 || s.K <= 0) return cudaSuccess;
   if constexpr (NACC == 2) {
     return launch_tc<2, 128, Epi>(s, A, A2, B, epi, st, status);
-  } else if constexpr (Epi::kFixedHeadTile) {
-    return launch_tc<1, HEAD_BN, Epi>(s, A, A2, B, epi, st, status);
   } else {
-    if (tile_efficiency(s, 128) > tile_efficiency(s, 256)) return launch_tc<1, 128, Epi>(s, A, A2, B, epi, st, status);
-    return launch_tc<1, 256, Epi>(s, A, A2, B, epi, st, status);
+    // Expected throughput = fraction of the machine busy x relative rate of
+    // the tile shape under the operand-feed limit (pair 256x256: 1.3,
+    // 1-SM 128x256: 1.0, 1-SM 128x128: 0.78, already in tile_efficiency).
+    // The pair kernel may split K, which lifts its occupancy.
+    double s_pair = 0.0;
+    if (pair_mode() && s.M > BM) {
+      const long tiles = (long)((s.M + 2 * BM - 1) / (2 * BM)) * ((s.N + 255) / 256) * s.batch;
+      const int num_kb = (s.K + BK - 1) / BK;
+      const int S = choose_splits(tiles, num_kb, ss);
+      const int pairs = num_sms() / 2;
+      const long units = tiles * S;
+      const long waves = (units + pairs - 1) / pairs;
+      const int kbps = (num_kb + S - 1) / S;
+      // useful k-blocks over issued k-block slots (with the split overhead)
+      s_pair = 1.3 * (double)tiles * num_kb / ((double)waves * pairs * (kbps + (S > 1 ? 4 : 0)));
+    }
+    const double s256 = tile_efficiency(s, 256);
+    const double s128 = Epi::kFixedHeadTile ? 0.0 : tile_efficiency(s, 128);
+    if (s_pair >= s256 && s_pair >= s128) return launch_tc2<1, 256, Epi>(s, A, A2, B, epi, st, status, ss);
+    if constexpr (!Epi::kFixedHeadTile) {
+      if (s128 > s256) return launch_tc<1, 128, Epi>(s, A, A2, B, epi, st, status);
+    }
+    return launch_tc<1, HEAD_BN, Epi>(s, A, A2, B, epi, st, status);
   }
+}
+
+// Dual accumulators sharing A: acc_0 = A B1^T, acc_1 = A B2^T (B1, B2 same layout).
+template <class Epi>
+cudaError_t launch_gemm_tc_dualb(const GemmShape& s, const Operand& A, const Operand& B1, const Operand& B2,
+                                 const Epi& epi, cudaStream_t st, int* status) {
+  if (s.M <= 0 || s.N <= 0 || s.batch <= 0 || s.K <= 0) return cudaSuccess;
+  return launch_tc<2, 128, Epi>(s, A, B2, B1, epi, st, status, 1);
 }
 
 }  // namespace tc

@@ -24,4 +24,14 @@ struct Operand {
   int64_t rows_per_batch;
 };
 
+// Scratch for split-K partial tiles of the CTA-pair GEMM (both may be null:
+// no split-K).  counters must be zero before the first GEMM that uses them;
+// every GEMM leaves them zero.
+struct SplitScratch {
+  float* partial = nullptr;
+  size_t partial_bytes = 0;
+  int* counters = nullptr;
+  size_t counter_count = 0;
+};
+
 }  // namespace ttt

@@ -26,17 +26,27 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 x
 // Gather chunk c of every sequence: resid[s*b + i] = hidden[s, c*b + i] and
 // its operand copy.
 // ---------------------------------------------------------------------------
+// When the first MLP is dynamic, also its K-scaled negated input copies
+// (B operands of its first-matrix aggregation).
 template <typename T>
 __global__ void gather_chunk_kernel(const float* __restrict__ hidden, int T_, int b, int chunk, int d,
-                                    int64_t n, float* __restrict__ resid, T* __restrict__ act) {
+                                    int64_t n, float* __restrict__ resid, T* __restrict__ act,
+                                    T* __restrict__ aw, T* __restrict__ am, const float* __restrict__ KW,
+                                    const float* __restrict__ KM, float kscale) {
   const int64_t q = d >> 2;  // float4 per row (d % 16 == 0)
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n * q;
        e += (int64_t)gridDim.x * blockDim.x) {
     int64_t r = e / q, c4 = e - r * q;
     int64_t s = r / b, i = r - s * b;
-    const float4 x = reinterpret_cast<const float4*>(hidden + ((s * T_ + (int64_t)chunk * b + i) * d))[c4];
+    const int64_t ti = s * T_ + (int64_t)chunk * b + i;
+    const float4 x = reinterpret_cast<const float4*>(hidden + ti * d)[c4];
     reinterpret_cast<float4*>(resid + r * d)[c4] = x;
     store4<T>(act + r * d + c4 * 4, x);
+    if (aw) {
+      const float kw = -KW[ti] * kscale, km = -KM[ti] * kscale;
+      store4<T>(aw + r * d + c4 * 4, make_float4(kw * x.x, kw * x.y, kw * x.z, kw * x.w));
+      store4<T>(am + r * d + c4 * 4, make_float4(km * x.x, km * x.y, km * x.z, km * x.w));
+    }
   }
 }
 

@@ -93,8 +93,9 @@ struct Plan {
   float kscale;  // 1/b for the mean reduction, 1 for the sum
   bool swiglu, has_static;
   size_t esz;  // operand element size
-  size_t KW, KM, consts, Wsh, resid, actin, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
-      doutW[2], doutM[2], dU, dUW, dUM, total;
+  size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
+      doutW[2], doutM[2], dU, sk_partial, sk_counters, total;
+  size_t sk_partial_bytes, sk_counter_count;
 };
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -135,6 +136,8 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.Wsh = take(e * B * p.L * p.m * h * d);
   p.resid = take(4 * n * d);
   p.actin = take(e * p.nM * n * d);
+  p.aw = take(e * p.nM * n * d);
+  p.am = take(e * p.nM * n * d);
   p.act = take(e * p.nM * n * h);
   p.fac = take(e * p.nM * n * H2);
   p.z = take(e * n * d);
@@ -149,8 +152,11 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.dout_a = take(e * n * d);
   for (int i = 0; i < 2; ++i) { p.doutW[i] = take(e * n * d); p.doutM[i] = take(e * n * d); }
   p.dU = take(e * n * H2);
-  p.dUW = take(e * n * H2);
-  p.dUM = take(e * n * H2);
+  // split-K scratch of the CTA-pair GEMMs (only when 256-row pair tiles exist)
+  p.sk_partial_bytes = (c.precision == TTT_PREC_BF16 && n >= 256) ? std::min<size_t>(64ull << 20, 64ull * 1024 * n) : 0;
+  p.sk_counter_count = p.sk_partial_bytes ? 65536 : 0;
+  p.sk_partial = take(p.sk_partial_bytes);
+  p.sk_counters = take(4 * p.sk_counter_count);
   p.total = off;
   return p;
 }
@@ -160,12 +166,25 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
 // ---------------------------------------------------------------------------
 template <typename T, int NACC, class Epi>
 static cudaError_t gemm(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B,
-                        const Epi& epi, cudaStream_t st, int* status) {
+                        const Epi& epi, cudaStream_t st, int* status, const SplitScratch& ss = SplitScratch()) {
   if constexpr (std::is_same<T, float>::value) {
     (void)status;
+    (void)ss;
     return launch_gemm_simt<T, NACC, Epi>(s, A, A2, B, epi, st);
   } else {
-    return tc::launch_gemm_tc<NACC, Epi>(s, A, A2, B, epi, st, status);
+    return tc::launch_gemm_tc<NACC, Epi>(s, A, A2, B, epi, st, status, ss);
+  }
+}
+
+// Dual accumulators sharing the A operand: acc_0 = A B1^T, acc_1 = A B2^T.
+template <typename T, class Epi>
+static cudaError_t gemm_dualb(const GemmShape& s, const Operand& A, const Operand& B1, const Operand& B2,
+                              const Epi& epi, cudaStream_t st, int* status) {
+  if constexpr (std::is_same<T, float>::value) {
+    (void)status;
+    return launch_gemm_simt<T, 2, Epi>(s, A, B2, B1, epi, st, 1);
+  } else {
+    return tc::launch_gemm_tc_dualb<Epi>(s, A, B1, B2, epi, st, status);
   }
 }
 
@@ -230,6 +249,8 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
   float* resid = reinterpret_cast<float*>(ws + p.resid);
   T* actin = reinterpret_cast<T*>(ws + p.actin);
+  T* aw = reinterpret_cast<T*>(ws + p.aw);
+  T* am = reinterpret_cast<T*>(ws + p.am);
   T* act = reinterpret_cast<T*>(ws + p.act);
   T* fac = reinterpret_cast<T*>(ws + p.fac);
   T* z = reinterpret_cast<T*>(ws + p.z);
@@ -245,17 +266,23 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
   T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
   T* dU = reinterpret_cast<T*>(ws + p.dU);
-  T* dUW = reinterpret_cast<T*>(ws + p.dUW);
-  T* dUM = reinterpret_cast<T*>(ws + p.dUM);
   const T* E = static_cast<const T*>(hd->E);
   const T* S = static_cast<const T*>(hd->S);
   int* status = hd->status;
+  SplitScratch ss;
+  ss.partial = reinterpret_cast<float*>(ws + p.sk_partial);
+  ss.partial_bytes = p.sk_partial_bytes;
+  ss.counters = reinterpret_cast<int*>(ws + p.sk_counters);
+  ss.counter_count = p.sk_counter_count;
+  if (!p.sk_partial_bytes) ss = SplitScratch();
   cudaError_t err;
 #define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
 #define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
   const double e = (double)p.esz;
 
   // K1 for all chunks (depends only on the scalars).
+  // Split-K arrival counters start at zero (every GEMM leaves them zero).
+  if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
   LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T, TRY(launch_scalar_scan(eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
   // Operand shadow of W_0.
   LAUNCH(K_SHADOW, 0, (4.0 + e) * B * L * p.m * h * d,
@@ -272,7 +299,13 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
 
   for (int c = 0; c < p.nchunks; ++c) {
     TokenMap tm{b, p.T, c};
-    LAUNCH(K_GATHER, 0, (8.0 + e) * n * d, (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin)));
+    {
+      const bool first_dyn = is_dyn(0);
+      LAUNCH(K_GATHER, 0, (8.0 + e * (first_dyn ? 3 : 1)) * n * d,
+             (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin,
+                                                          first_dyn ? aw : nullptr, first_dyn ? am : nullptr,
+                                                          KW, KM, p.kscale)));
+    }
 
     // ---- forward through the blocks ----
     for (int i = 0; i < p.nM; ++i) {
@@ -292,17 +325,22 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         T* fptr = (i >= i_min) ? fi : nullptr;
         const double fl = 2.0 * Mz * H2 * d * Bz;
         const double by = e * ((double)n * d + (double)H2 * d * Bz + (double)n * h + (fptr ? (double)n * H2 : 0.0));
-        if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status))));
-        else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status))));
+        if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status, ss))));
+        else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status, ss))));
       }
       {
         GemmShape s{Mz, d, h, Bz};
         Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
         Operand Bw = opnd(w2, h, wstride, 1, d);
         T* next = (i + 1 < p.nM) ? actin + (int64_t)(i + 1) * n * d : nullptr;
+        const bool next_dyn = i + 1 < p.nM && is_dyn(i + 1);
+        T* nw = next_dyn ? aw + (int64_t)(i + 1) * n * d : nullptr;
+        T* nmm = next_dyn ? am + (int64_t)(i + 1) * n * d : nullptr;
         LAUNCH(K_MLP_DOWN, 2.0 * Mz * d * h * Bz,
-               e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0)) + 8.0 * n * d,
-               TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, d, Mz}, st, status))));
+               e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0) + (nw ? 2.0 * n * d : 0.0)) +
+                   8.0 * n * d,
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, nw, nmm, KW, KM, p.kscale, tm, d, Mz}, st,
+                                status, ss))));
       }
     }
 
@@ -314,7 +352,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E, d, 0, 1, V);
       LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status))));
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
     }
     LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
            (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
@@ -328,14 +366,14 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         Operand A = opnd(z, d, 0, 1, n);
         Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
         LAUNCH(K_CE_GRAD, 2.0 * n * vs * d, e * ((double)n * d + (double)vs * d + (double)n * vs),
-               TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status))));
+               TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status, ss))));
       }
       {
         GemmShape s{n, d, vs, 1};
         Operand A = opnd(P, p.Vs, 0, 1, n);
         Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 0, vs);
         LAUNCH(K_CE_DZ, 2.0 * n * d * vs, e * ((double)n * vs + (double)vs * d) + (sl > 0 ? 8.0 : 4.0) * n * d,
-               TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status))));
+               TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status, ss))));
       }
     }
     {
@@ -355,17 +393,14 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
       const bool need_dx = i > i_min;
       T* fi = fac + (int64_t)i * n * H2;
-      {  // B1: dA = dOut W2 -> dU (+ scaled copies)
+      {  // B1: dA = dOut W2 -> dU
         GemmShape s{Mz, h, d, Bz};
         Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
         Operand Bw = opnd(w2, h, wstride, 0, d);
-        T* du = need_dx ? dU : nullptr;
-        T* dw = dyn ? dUW : nullptr;
-        T* dm = dyn ? dUM : nullptr;
         const double fl = 2.0 * Mz * h * d * Bz;
-        const double by = e * ((double)n * d + (double)d * h * Bz + (double)n * H2 * (1 + (du ? 1 : 0) + (dw ? 2 : 0)));
-        if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status))));
-        else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, du, dw, dm, KW, KM, p.kscale, tm, h, Mz}, st, status))));
+        const double by = e * ((double)n * d + (double)d * h * Bz + 2.0 * n * H2);
+        if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, dU, h, Mz}, st, status, ss))));
+        else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, dU, h, Mz}, st, status, ss))));
       }
       if (need_dx) {  // B2: dout += dU W1
         GemmShape s{Mz, d, H2, Bz};
@@ -376,23 +411,23 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         T* om = below_dyn ? doutM[(i - 1) & 1] : nullptr;
         LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
                e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
-               TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status))));
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status, ss))));
       }
       if (dyn) {
-        T* ain = actin + (int64_t)i * n * d;
         T* aout = act + (int64_t)i * n * h;
         float* Wl = W + l * blk;
         float* Ml = M + l * blk;
         T* Sl = Wsh + l * blk;
-        {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens
+        {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens:
+           // sum_t dU_t (x) (-K_t x_t), A = dU shared by both accumulators
           GemmShape s{H2, d, b, B};
-          Operand A = opnd(dUW, H2, (int64_t)b * H2, 0, b);
-          Operand A2 = opnd(dUM, H2, (int64_t)b * H2, 0, b);
-          Operand Bx = opnd(ain, d, (int64_t)b * d, 0, b);
+          Operand A = opnd(dU, H2, (int64_t)b * H2, 0, b);
+          Operand B1 = opnd(aw + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+          Operand B2 = opnd(am + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
           EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
           LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B,
-                 (16.0 + e) * H2 * d * B + e * ((double)n * H2 * 2 + (double)n * d),
-                 TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+                 (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
+                 TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
         }
         {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
           GemmShape s{d, h, b, B};
@@ -704,8 +739,9 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != TTT_OK) return s;
-  // Every buffer of the plan is written before it is read within the call,
-  // so the scratch needs no clearing between calls.
+  // Every buffer of the plan is written before it is read within the call
+  // (the split-K counters are cleared by the call itself), so the scratch
+  // needs no clearing between calls.
   Prof prof;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(scratch);
@@ -718,7 +754,8 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
 
 ttt_status ttt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
                          int64_t strideA, int32_t a_kmajor, const void* B, int64_t ldb, int64_t strideB,
-                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* stream) {
+                         int32_t b_kmajor, float* D, int64_t ldd, int64_t strideD, void* workspace,
+                         size_t ws_bytes, void* stream) {
   if (M < 0 || N < 0 || K < 0 || batch < 0) return fail(TTT_ERR_SHAPE, "negative size");
   if (M == 0 || N == 0 || K == 0 || batch == 0) return TTT_OK;
   if (!A || !B || !D) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
@@ -733,7 +770,17 @@ ttt_status ttt_gemm_bf16(int32_t M, int32_t N, int32_t K, int32_t batch, const v
   Operand a = opnd(A, lda, strideA, a_kmajor ? 1 : 0, a_kmajor ? M : K);
   Operand b = opnd(B, ldb, strideB, b_kmajor ? 1 : 0, b_kmajor ? N : K);
   EpiStoreBatched e{D, ldd, strideD};
-  TTT_CUDA_TRY((tc::launch_gemm_tc<1, EpiStoreBatched>(s, a, a, b, e, static_cast<cudaStream_t>(stream), nullptr)));
+  SplitScratch ss;
+  if (workspace && ws_bytes >= (size_t(1) << 20)) {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    // counters first (zeroed here), the rest holds split-K partial tiles
+    ss.counters = static_cast<int*>(workspace);
+    ss.counter_count = 65536;
+    ss.partial = reinterpret_cast<float*>(static_cast<char*>(workspace) + 4 * ss.counter_count);
+    ss.partial_bytes = ws_bytes - 4 * ss.counter_count;
+    TTT_CUDA_TRY(cudaMemsetAsync(ss.counters, 0, 4 * ss.counter_count, static_cast<cudaStream_t>(stream)));
+  }
+  TTT_CUDA_TRY((tc::launch_gemm_tc<1, EpiStoreBatched>(s, a, a, b, e, static_cast<cudaStream_t>(stream), nullptr, ss)));
   return TTT_OK;
 }
 

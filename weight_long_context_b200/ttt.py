@@ -78,7 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
     lib.ttt_scalar_kernels.restype = I32
     I64 = ctypes.c_int64
-    lib.ttt_gemm_bf16.argtypes = [I32, I32, I32, I32, P, I64, I64, I32, P, I64, I64, I32, P, I64, I64, P]
+    lib.ttt_gemm_bf16.argtypes = [I32, I32, I32, I32, P, I64, I64, I32, P, I64, I64, I32, P, I64, I64, P, SZ, P]
     lib.ttt_gemm_bf16.restype = I32
     lib.ttt_get_device_status.argtypes = [P, P]
     lib.ttt_get_device_status.restype = I32
@@ -155,7 +155,8 @@ def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tenso
 
 
 def ttt_gemm_bf16(A: torch.Tensor, B: torch.Tensor, a_kmajor: bool = True, b_kmajor: bool = True,
-                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                  out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
     """D[z] = A[z] B[z]^T on the tcgen05 engine.  A, B: bf16 CUDA tensors of shape
     [batch, M, K] / [batch, N, K] when K-major, [batch, K, M] / [batch, K, N] when
     MN-major (2-D inputs are batch 1).  Returns fp32 [batch, M, N]."""
@@ -172,6 +173,7 @@ def ttt_gemm_bf16(A: torch.Tensor, B: torch.Tensor, a_kmajor: bool = True, b_kma
     sB = B3.shape[1] * B3.shape[2] if batch > 1 else 0
     _check(load_library().ttt_gemm_bf16(M, N, K, batch, _ptr(A3), A3.shape[2], sA, int(a_kmajor), _ptr(B3),
                                         B3.shape[2], sB, int(b_kmajor), _ptr(out), N, M * N,
+                                        _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                         _stream_ptr(stream)), "ttt_gemm_bf16")
     return out if A.dim() == 3 else out[0]
 
