@@ -95,6 +95,14 @@ __device__ __forceinline__ void vst_scaled(T* p, const float* v, float s) {
   vst<N>(p, t);
 }
 
+// Four consecutive elements from float values (8 bytes for bf16, 16 for fp32).
+__device__ __forceinline__ void store_x4(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store_x4(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
 // ---------------------------------------------------------------------------
 // F1: U = a W1^T (GELU: [n,h]; SwiGLU: [n,2h] in the interleaved layout).
 // Writes the activation A (input of the second matrix) and the factors the
@@ -104,6 +112,8 @@ __device__ __forceinline__ void vst_scaled(T* p, const float* v, float s) {
 template <typename T, bool SWIGLU>
 struct EpiF1 {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   T* act;        // [rows, h]
   T* fac;        // [rows, H2] or nullptr when no backward passes through
@@ -160,6 +170,8 @@ struct EpiF1 {
 template <typename T>
 struct EpiResid {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   float* resid;   // [rows, d]
   T* act_next;    // [rows, d] or nullptr
@@ -213,6 +225,8 @@ struct EpiResid {
 template <typename T, bool SWIGLU>
 struct EpiB1 {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   const T* fac;   // [rows, H2]
   T* dU;          // [rows, H2]
@@ -263,6 +277,8 @@ struct EpiB1 {
 template <typename T>
 struct EpiB2 {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   float* dout;    // [rows, d]
   T* dout_a;      // [rows, d]
@@ -312,6 +328,8 @@ struct EpiB2 {
 // ---------------------------------------------------------------------------
 struct EpiCEPartial {
   static constexpr bool kFixedHeadTile = true;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   struct RowState { float m, s; int y; };
   float* part;        // [rows, ntn, 2]
   float* tgt;         // [rows]
@@ -351,6 +369,8 @@ struct EpiCEPartial {
 template <typename T>
 struct EpiCEGrad {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = int;  // the row's label
   T* P;               // [rows, Vs]
   const float* lse;   // [rows]
@@ -381,6 +401,8 @@ struct EpiCEGrad {
 // ---------------------------------------------------------------------------
 struct EpiStoreF32 {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   float* out;
   int ld;
@@ -409,6 +431,8 @@ struct EpiStoreF32 {
 // Batched fp32 store: out[z](r, c) at out + z * zstride + r * ld + c.
 struct EpiStoreBatched {
   static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
   using RowState = NoRowState;
   float* out;
   int64_t ld;
@@ -435,7 +459,15 @@ struct EpiStoreBatched {
 template <typename T>
 struct EpiUpdate {
   static constexpr bool kFixedHeadTile = false;
-  using RowState = NoRowState;
+  static constexpr bool kPreload = true;
+  // The tcgen05 engine stages each warp's 32 x 32 accumulator span through
+  // shared memory and calls span_warp(): the warp then walks the span row by
+  // row, 8 lanes x 4 columns per row, so every W / M / shadow access of an
+  // instruction covers whole 128-byte rows (the CUDA-core engine uses span()).
+  static constexpr bool kWarpRows = true;
+  // The span's W and M values, loaded by preload() before the engine reads
+  // the accumulators from TMEM, so the state reads overlap the TMEM reads.
+  struct RowState { float w[32], m[32]; };
   float* W;            // this matrix, sequence 0 (rows of the packed layout)
   float* M;
   T* Wsh;              // shadow of this matrix, sequence 0 (library row order)
@@ -448,7 +480,88 @@ struct EpiUpdate {
   int h;               // > 0: rows are SwiGLU [gate; up] positions to remap
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
-  __device__ void span(RowState&, int z, int r, int c0, const float* v, const float* v2, int nv) const {
+  // Row-walking epilogue (used by the tcgen05 engine): a warp updates a span
+  // of 32 rows x 32 columns, 8 lanes x 4 columns per row, so every W / M /
+  // shadow access of an instruction covers whole 128-byte rows.  load_span()
+  // issues the span's W and M loads into registers; finish_span() combines
+  // them with the accumulators staged in shared memory (sv / sv2: element
+  // (row i, column j) at [i * 32 + ((j + i) & 31)], rotated so both the
+  // staging writes and these reads are conflict-free) and stores the results.
+  // The engine calls them per half span (16 rows), 8 warps per CTA.
+  struct SpanRegs { float4 w[4], m[4]; };
+  // half: rows [16 half, 16 half + 16) of the span (8 lanes x 4 rows per step).
+  __device__ void load_span(SpanRegs& R, int half, int z, int row0, int c0, int nv, int nrows, int lane) const {
+    const int sub = lane >> 3, cj = (lane & 7) * 4;
+    if (cj + 4 > nv) return;
+    const float* Wz = W + z * seq_stride + c0 + cj;
+    const float* Mz = M + z * seq_stride + c0 + cj;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 16 * half + 4 * k + sub;
+      if (i < nrows) {
+        const int r = row0 + i;
+        const int64_t off = (int64_t)(h > 0 ? swiglu_row_of_pos(r, h) : r) * cols;
+        R.w[k] = *reinterpret_cast<const float4*>(Wz + off);
+        R.m[k] = *reinterpret_cast<const float4*>(Mz + off);
+      }
+    }
+  }
+  __device__ void finish_span(const SpanRegs& R, int half, int z, int row0, int c0, const float* sv,
+                              const float* sv2, int nv, int nrows, int lane) const {
+    const float4 cs = *reinterpret_cast<const float4*>(consts + ((int64_t)z * nchunks + chunk) * 4);
+    const float g0 = cs.x, b0 = cs.y, cM = cs.z;
+    const int sub = lane >> 3, cj = (lane & 7) * 4;
+    const bool vec = cj + 4 <= nv;
+    float* const Wz = W + z * seq_stride + c0 + cj;
+    float* const Mz = M + z * seq_stride + c0 + cj;
+    T* const Sz = Wsh + z * sh_stride + c0 + cj;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = 16 * half + 4 * k + sub;
+      if (i >= nrows || cj >= nv) continue;
+      const int r = row0 + i;
+      const int64_t off = (int64_t)(h > 0 ? swiglu_row_of_pos(r, h) : r) * cols;
+      float a[4], a2[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a[j] = sv[i * 32 + ((cj + j + i) & 31)];
+        a2[j] = sv2[i * 32 + ((cj + j + i) & 31)];
+      }
+      T* sp = Sz + (int64_t)r * cols;
+      if (vec) {
+        float wn[4] = {R.w[k].x, R.w[k].y, R.w[k].z, R.w[k].w};
+        float mn[4] = {R.m[k].x, R.m[k].y, R.m[k].z, R.m[k].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float wv = fmaf(g0, wn[j], fmaf(cM, mn[j], a[j]));
+          mn[j] = fmaf(b0, mn[j], a2[j]);
+          wn[j] = wv;
+        }
+        *reinterpret_cast<float4*>(Wz + off) = make_float4(wn[0], wn[1], wn[2], wn[3]);
+        *reinterpret_cast<float4*>(Mz + off) = make_float4(mn[0], mn[1], mn[2], mn[3]);
+        store_x4(sp, wn);
+      } else {
+        float* wq = Wz + off;
+        float* mq = Mz + off;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (cj + j < nv) {
+            const float wv = fmaf(g0, wq[j], fmaf(cM, mq[j], a[j]));
+            mq[j] = fmaf(b0, mq[j], a2[j]);
+            wq[j] = wv;
+            sp[j] = from_f<T>(wv);
+          }
+        }
+      }
+    }
+  }
+  __device__ void preload(RowState& st, int z, int r, int c0, int nv) const {
+    if (nv != 32) return;
+    int fr = h > 0 ? swiglu_row_of_pos(r, h) : r;
+    vld<32>(W + z * seq_stride + (int64_t)fr * cols + c0, st.w);
+    vld<32>(M + z * seq_stride + (int64_t)fr * cols + c0, st.m);
+  }
+  __device__ void span(RowState& st, int z, int r, int c0, const float* v, const float* v2, int nv) const {
     const float4 cs = *reinterpret_cast<const float4*>(consts + ((int64_t)z * nchunks + chunk) * 4);
     const float g0 = cs.x, b0 = cs.y, cM = cs.z;
     int fr = h > 0 ? swiglu_row_of_pos(r, h) : r;
@@ -457,20 +570,14 @@ struct EpiUpdate {
     T* sp = Wsh + z * sh_stride + (int64_t)r * cols + c0;
     if (nv == 32) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {   // two halves of 16 keep register use bounded
-        float w[16], m[16];
-        vld<16>(wp + 16 * q, w);
-        vld<16>(mp + 16 * q, m);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          float wn = fmaf(g0, w[j], fmaf(cM, m[j], v[16 * q + j]));
-          m[j] = fmaf(b0, m[j], v2[16 * q + j]);
-          w[j] = wn;
-        }
-        vst<16>(wp + 16 * q, w);
-        vst<16>(mp + 16 * q, m);
-        vst<16>(sp + 16 * q, w);
+      for (int j = 0; j < 32; ++j) {
+        float wn = fmaf(g0, st.w[j], fmaf(cM, st.m[j], v[j]));
+        st.m[j] = fmaf(b0, st.m[j], v2[j]);
+        st.w[j] = wn;
       }
+      vst<32>(wp, st.w);
+      vst<32>(mp, st.m);
+      vst<32>(sp, st.w);
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) if (j < nv) {

@@ -108,6 +108,7 @@ gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi, int dua
           v[j] = Cs[0][tid][sp * 32 + j];
           v2[j] = Cs[NACC - 1][tid][sp * 32 + j];
         }
+        if constexpr (Epi::kPreload) epi.preload(st, z, r, c0, nv);
         epi.span(st, z, r, c0, v, v2, nv);
       }
       epi.row_end(st, z, r, blockIdx.x);

@@ -163,16 +163,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
 // ---------------------------------------------------------------------------
 // Kernel configuration per (accumulators, N tile)
 // ---------------------------------------------------------------------------
-template <int NACC, int BN>
+template <int NACC, int BN, bool WARPROWS = false>
 struct Cfg {
+  // Epilogue warps: two per TMEM lane quarter, splitting the tile's columns.
+  static constexpr int EW = EPI_WARPS;
+  static constexpr int PARTS = EW / 4;
+  static constexpr int NTHREADS = 64 + 32 * EW;
   static constexpr int A_BYTES = BM * BK * 2;            // 16 KiB
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = NACC * A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  // Epilogues that walk rows per warp stage each warp's 32x32 span(s) in
+  // shared memory: NACC x 4 KiB per epilogue warp.
+  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EW * NACC * 32 * 32 * 4 : 0;
+  static constexpr int STAGES = ((WARPROWS ? 220 : 200) * 1024 - ROWSTAGE_BYTES) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * NACC * BN;         // two accumulator buffers
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ROWSTAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(SMEM_BYTES <= 232448, "shared memory above the 227 KiB per-CTA limit");
 };
 
 struct TcParams {
@@ -192,13 +200,14 @@ struct TcParams {
 };
 
 template <int NACC, int BN, class Epi>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Cfg<NACC, BN, Epi::kWarpRows>::NTHREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
                const __grid_constant__ CUtensorMap mapB, const TcParams p, const Epi epi) {
-  using C = Cfg<NACC, BN>;
+  using C = Cfg<NACC, BN, Epi::kWarpRows>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* rowstage = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::ROWSTAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -211,7 +220,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 32 * EPI_WARPS); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 32 * C::EW); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -337,7 +346,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // ------------------------------ epilogue ------------------------------
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int part = (warp - 2) >> 2;       // which column part of the tile
-    constexpr int PART_COLS = BN / EPI_PARTS;
+    constexpr int PART_COLS = BN / C::PARTS;
     const int row_in_tile = q * 32 + lane;
     uint32_t tcount = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
@@ -356,15 +365,48 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       typename Epi::RowState rs;
       if (row_ok) epi.row_begin(rs, z, r);
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
+      if constexpr (Epi::kWarpRows) {
+        float* sv = rowstage + (warp - 2) * (NACC * 1024);
+        float* sv2 = sv + (NACC - 1) * 1024;
+        const int row0 = tm * BM + q * 32;
+        const int nrows = min(32, s.M - row0);
 #pragma unroll 1
-      for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
-        float v[32], v2[32];
-        tmem_ld32(tbase + c, v);
-        if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
-        const int c0 = tn * BN + c;
-        if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+        for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
+          const int c0 = tn * BN + c;
+          float v[32], v2[32];
+          tmem_ld32(tbase + c, v);
+          if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            sv[lane * 32 + ((j + lane) & 31)] = v[j];
+            if (NACC == 2) sv2[lane * 32 + ((j + lane) & 31)] = v2[j];
+          }
+          __syncwarp();
+          if (nrows > 0 && c0 < s.N) {
+            const int nv = min(32, s.N - c0);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              typename Epi::SpanRegs R;
+              epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
+              epi.finish_span(R, half, z, row0, c0, sv, sv2, nv, nrows, lane);
+            }
+          }
+          __syncwarp();
+        }
+      } else {
+#pragma unroll 1
+        for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
+          float v[32], v2[32];
+          const int c0 = tn * BN + c;
+          if constexpr (Epi::kPreload) {
+            if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
+          }
+          tmem_ld32(tbase + c, v);
+          if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
+          if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+        }
       }
-      if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+      if (row_ok) epi.row_end(rs, z, r, tn * C::PARTS + part);
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
@@ -623,9 +665,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
 #pragma unroll 1
         for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
           float v[32], v2[32];
+          const int c0 = tn * BN + c;
+          if constexpr (Epi::kPreload) {
+            if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
+          }
           tmem_ld32(tbase + c, v);
           if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
-          const int c0 = tn * BN + c;
           if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
         }
         if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
@@ -678,6 +723,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
               }
             }
             const int c0 = tn * BN + c;
+            if constexpr (Epi::kPreload) {
+              if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
+            }
             if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
           }
           if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
@@ -765,7 +813,7 @@ template <int NACC, int BN, class Epi>
 cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
                       cudaStream_t st, int* status, int dualb = 0) {
   static_assert(NACC == 1 || BN == BM, "dual accumulators use equal A and B slots");
-  using C = Cfg<NACC, BN>;
+  using C = Cfg<NACC, BN, Epi::kWarpRows>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<NACC, BN, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -806,7 +854,7 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   p.partial = nullptr;
   p.counters = nullptr;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  gemm_tc_kernel<NACC, BN, Epi><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
+  gemm_tc_kernel<NACC, BN, Epi><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
 }
 
