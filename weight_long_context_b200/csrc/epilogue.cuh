@@ -254,18 +254,20 @@ struct EpiB1 {
       }
     } else {
       // h % 16 == 0 and c0 % 32 == 0: nv is 16 or 32, whole groups of 16.
-      const int64_t p0 = ob + 2 * (int64_t)c0;
-      float f[64], du[64];
-      if (nv == 32) vld<64>(fac + p0, f);
-      else vld<32>(fac + p0, f);
+      // dA columns c0 + 16 g + k own positions 2 c0 + 32 g + k (gate) and + 16 (up).
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int gi = (j >> 4) * 32 + (j & 15);   // gate position within the 64
-        du[gi] = v[j] * f[gi];
-        du[gi + 16] = v[j] * f[gi + 16];
+      for (int g = 0; g < 2; ++g) {
+        if (16 * g >= nv) break;
+        const int64_t p0 = ob + 2 * (int64_t)c0 + 32 * g;
+        float f[32], du[32];
+        vld<32>(fac + p0, f);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          du[k] = v[16 * g + k] * f[k];
+          du[16 + k] = v[16 * g + k] * f[16 + k];
+        }
+        vst<32>(dU + p0, du);
       }
-      if (nv == 32) vst<64>(dU + p0, du);
-      else vst<32>(dU + p0, du);
     }
   }
 };
