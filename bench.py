@@ -420,10 +420,15 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="profiling captures only: run the first N chunks of each sequence instead of the full T "
+                         "(every launch keeps its full-size shape; the line's config names the reduced T)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     w = I.WORKLOADS[args.workload]
+    if args.chunks > 0:
+        w = w.with_(T=min(w.T, args.chunks * w.b))
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
