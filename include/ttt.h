@@ -130,7 +130,8 @@ ttt_status ttt_workspace_size(const ttt_handle* h, int32_t batch, int32_t T, int
  *                             taken at that chunk's start weights
  *   workspace  device scratch of at least ttt_workspace_size() bytes, 256-byte
  *              aligned; its contents are not preserved
- * W and M are updated in place.  T must be a multiple of b (TTT_ERR_SHAPE
+ * W and M are updated in place.  hidden, W and M must be 16-byte aligned
+ * (TTT_ERR_INVALID_ARG otherwise).  T must be a multiple of b (TTT_ERR_SHAPE
  * otherwise); T == 0 or batch == 0 is a no-op.  hidden, tokens and the
  * scalars must not alias W, M, chunk_loss or the workspace. */
 ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,

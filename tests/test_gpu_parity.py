@@ -295,3 +295,27 @@ def test_profiled_path_matches_graph_path(dev):
     assert upd["launches"] == 2 * w.n_blocks * w.n_chunks
     assert upd["flops"] == pytest.approx(4.0 * 3 * w.hidden * w.d * w.b * w.batch * w.n_blocks * w.n_chunks)
     h.close()
+
+
+def test_misaligned_state_rejected(dev):
+    """W and M must be 16-byte aligned: a 4-byte offset is rejected before any launch."""
+    import ctypes
+    from weight_long_context_b200 import ttt
+    w = I.Workload("e", 32, 32, 32, 1, "gelu", False, "bf16", 16, 8, 1, "e2ttt")
+    x = I.make_inputs(w, seed=0)
+    h = H.make_handle(w, x, dev)
+    t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    n = ttt.ttt_workspace_size(h._h, 1, 16, 8)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    loss = torch.empty((1, 2), device=dev)
+    Wbig = torch.zeros(x["W0"].size + 4, device=dev)
+    p = lambda a: ctypes.c_void_p(a.data_ptr())
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    hid, tok, M0 = t(x["hidden"]), t(x["tokens"], torch.int32), t(x["M0"])
+    sc = [t(x["eta"]), t(x["beta"]), t(x["gamma"])]
+    for Wp, Mp in ((Wbig[1:], M0), (t(x["W0"]), Wbig[1:])):
+        code = ttt.load_library().ttt_prefill(h._h, 1, 16, 8, p(hid), p(tok), p(Wp), p(Mp), *[p(a) for a in sc],
+                                              p(loss), p(ws), n, st)
+        assert code == 1
+    assert h.device_status() == 0
+    h.close()

@@ -619,7 +619,8 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   Plan p = make_plan(h->cfg, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  if (reinterpret_cast<uintptr_t>(hidden) % 16) return fail(TTT_ERR_INVALID_ARG, "hidden must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "hidden, W and M must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
@@ -674,6 +675,8 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
   Plan p = make_plan(h->cfg, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "hidden, W and M must be 16-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   Prof prof;
@@ -725,7 +728,8 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  if (reinterpret_cast<uintptr_t>(hidden) % 16) return fail(TTT_ERR_INVALID_ARG, "hidden must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "hidden, W and M must be 16-byte aligned");
   Plan p = make_plan(h->cfg, batch, T, b);
   if (p.total > kNoAllocScratchBytes) {
     static thread_local char msg[160];
