@@ -319,7 +319,7 @@ def scalar_kernels_ratio_form(eta, beta, gamma):
 # ---------------------------------------------------------------------------
 
 def chunk_update_closed(W, M, grads, eta, beta, gamma, gscale=1.0):
-    """Algorithm 1 lines 2 and 4-7: aggregate with K_W and K_M, then
+    """Algorithm 1, the scalar-kernel and update steps: aggregate with K_W and K_M, then
     W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + dW and M_C = btilde_0 M_0 + dM.
 
     G_t = -gscale * outer(L[t], R[t]) (gscale = 1/b for the mean reduction),
@@ -394,9 +394,9 @@ def prefill_sequence(model: Model, W0, M0, hidden, tokens, eta, beta, gamma, b,
         s = slice(c * b, (c + 1) * b)
         X = hidden[s]
         y = tokens[s]
-        loss, fwd = chunk_forward(model, W, X, y)     # line 1: at chunk-start weights
+        loss, fwd = chunk_forward(model, W, X, y)     # forward at the chunk-start weights
         losses[c] = float(np.mean(loss))
-        grads = chunk_backward(model, W, y, fwd)      # line 3: single backward
+        grads = chunk_backward(model, W, y, fwd)      # one backward for the whole chunk
         W, M = step(W, M, grads, eta[s], beta[s], gamma[s], gscale)
     return W, M, losses
 

@@ -11,7 +11,7 @@
 //   forward MLP activations ("Rethinking Expressivity and Efficiency in
 //   Test-Time Training", 快速权重网络实例化), residual adds, the online-softmax
 //   pieces of the next-token cross-entropy, the backward factors, and the
-//   Proposition 3.1 state update (same page, 命题3.1 and Algorithm 1 lines 6-7).
+//   Proposition 3.1 state update (same page, 命题3.1 and Algorithm 1).
 #pragma once
 
 #include "common.cuh"
@@ -453,7 +453,7 @@ struct EpiStoreBatched {
 };
 
 // ---------------------------------------------------------------------------
-// Aggregation + in-place update (Algorithm 1 lines 4-7): v = sum_t K_W_t G_t,
+// Aggregation + in-place update (Algorithm 1, update step): v = sum_t K_W_t G_t,
 // v2 = sum_t K_M_t G_t for this element;
 //   W <- gtilde_0 W + btilde_0 R_1 M + v,   M <- btilde_0 M + v2,
 // and the operand shadow of the new W.  Batch z = sequence.

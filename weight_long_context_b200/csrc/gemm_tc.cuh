@@ -143,6 +143,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// 32 lanes x 16 columns of 32-bit (same lane mapping as tmem_ld32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1
 // at bit 46, layout type 2 at bits 61-63).  Addresses and offsets in bytes.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -198,6 +213,68 @@ struct TcParams {
   float* partial;   // [num_tiles][splits][2 CTAs][128 rows][BN] fp32 when splits > 1
   int* counters;    // [num_tiles][2 CTAs][EPI_WARPS], zero on entry, left zero on exit
 };
+
+// Row-walking epilogue loop shared by both kernels: each 32 x 32 span of the
+// warp's accumulators is staged in shared memory (sv / sv2, rotated so the
+// staging writes and the row reads are conflict-free) and finished half a span
+// (16 rows) at a time, 8 lanes x 4 columns per row.  The tiles this CTA
+// processes are first, first + step, ...; tile rows start at
+// tm * rows_per_tile + row_off.  release(buf) frees the accumulator buffer once
+// every span of the tile is staged.  Epilogues of this kind keep no per-row state.
+template <int NACC, int BN, int PART_COLS, class Epi, class Release>
+__device__ __forceinline__ void warp_rows_loop(const Epi& epi, const TcParams& p, int first, int step,
+                                               int rows_per_tile, int row_off, uint32_t tmem_base,
+                                               uint64_t* tfull, float* sv, float* sv2, int q, int part, int lane,
+                                               volatile int* abort_flag, Release release) {
+  constexpr int NSP = PART_COLS / 32;
+  const GemmShape& s = p.s;
+  uint32_t tcount = 0;
+  for (int t = first; t < p.num_tiles; t += step, ++tcount) {
+    const uint32_t buf = tcount & 1u;
+    const uint32_t aph = (tcount >> 1) & 1u;
+    const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
+    if (!ready) break;
+    tc_fence_after();
+    const int tm = t % p.tiles_m;
+    const int rest = t / p.tiles_m;
+    const int tn = rest % p.tiles_n;
+    const int z = rest / p.tiles_n;
+    const int row0 = tm * rows_per_tile + row_off + q * 32;
+    const int nrows = min(32, s.M - row0);
+    const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
+#pragma unroll 1
+    for (int spi = 0; spi < NSP; ++spi) {
+      const int c = part * PART_COLS + spi * 32;
+      const int c0 = tn * BN + c;
+      const int nv = min(32, s.N - c0);
+#pragma unroll
+      for (int hc = 0; hc < 32; hc += 16) {
+        float v[16], v2[16];
+        tmem_ld16(tbase + c + hc, v);
+        if (NACC == 2) tmem_ld16(tbase + BN + c + hc, v2);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          sv[lane * 32 + ((hc + j + lane) & 31)] = v[j];
+          if (NACC == 2) sv2[lane * 32 + ((hc + j + lane) & 31)] = v2[j];
+        }
+      }
+      if (spi == NSP - 1) {  // every accumulator of this tile is staged: free the buffer
+        tc_fence_before();
+        release(buf);
+      }
+      __syncwarp();
+      if (nrows > 0 && nv > 0) {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          typename Epi::SpanRegs R;
+          epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
+          epi.finish_span(R, half, z, row0, c0, sv, sv2, nv, nrows, lane);
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
 
 template <int NACC, int BN, class Epi>
 __global__ void __launch_bounds__(Cfg<NACC, BN, Epi::kWarpRows>::NTHREADS, 1)
@@ -302,6 +379,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     // ------------------------------ MMA issuer ----------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(BN, p.a_mn, p.b_mn);
+      // Descriptors: a fixed high part (layout, strides) | the slot address in
+      // 16-byte units; each k-step / accumulator slot adds a constant to the
+      // address field (no carry: shared addresses stay below 256 KiB).
+      const uint64_t a_hi = smem_desc_sw128(0, p.a_mn ? 8192 : 16, 1024);
+      const uint64_t b_hi = smem_desc_sw128(0, p.b_mn ? 8192 : 16, 1024);
+      const uint32_t a_ks = p.a_mn ? 2048 >> 4 : 32 >> 4;   // one k-step of 16
+      const uint32_t b_ks = p.b_mn ? 2048 >> 4 : 32 >> 4;
+      const bool db = NACC == 2 && p.dualb;
+      const uint32_t a_slot = db ? 0u : (uint32_t)(C::A_BYTES >> 4);   // accumulator a's A slot step
+      const uint32_t b_slot = db ? (uint32_t)(C::B_BYTES >> 4) : 0u;   // accumulator a's B slot step
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++tcount) {
@@ -316,22 +403,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
-          const uint32_t sb = sa + NACC * C::A_BYTES;
+          const uint32_t sb = sa + (db ? C::A_BYTES : NACC * C::A_BYTES);
+          const uint64_t ad = a_hi | (uint64_t)((sa >> 4) & 0x3FFFu);
+          const uint64_t bd = b_hi | (uint64_t)((sb >> 4) & 0x3FFFu);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             // K-major: advance 16 elements = 32 bytes inside the swizzled row.
             // MN-major: advance 16 K-rows = two 8-row groups of 1024 bytes.
 #pragma unroll
-            for (int a = 0; a < NACC; ++a) {
-              const bool db = NACC == 2 && p.dualb;
-              const uint32_t abase = db ? sa : sa + a * C::A_BYTES;
-              const uint32_t bbase = db ? sa + C::A_BYTES + a * C::B_BYTES : sb;
-              const uint64_t adesc = p.a_mn ? smem_desc_sw128(abase + kk * 2048, 8192, 1024)
-                                            : smem_desc_sw128(abase + kk * 32, 16, 1024);
-              const uint64_t bdesc = p.b_mn ? smem_desc_sw128(bbase + kk * 2048, 8192, 1024)
-                                            : smem_desc_sw128(bbase + kk * 32, 16, 1024);
-              mma_bf16(d0 + a * BN, adesc, bdesc, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int a = 0; a < NACC; ++a)
+              mma_bf16(d0 + a * BN, ad + (kk * a_ks + a * a_slot), bd + (kk * b_ks + a * b_slot), idesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[st]);   // frees the stage once these MMAs have read it
         }
@@ -348,52 +430,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     const int part = (warp - 2) >> 2;       // which column part of the tile
     constexpr int PART_COLS = BN / C::PARTS;
     const int row_in_tile = q * 32 + lane;
-    uint32_t tcount = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
-      const int tm = t % p.tiles_m;
-      const int rest = t / p.tiles_m;
-      const int tn = rest % p.tiles_n;
-      const int z = rest / p.tiles_n;
-      const uint32_t buf = tcount & 1u;
-      const uint32_t aph = (tcount >> 1) & 1u;
-      // Warp-uniform decision: tcgen05.ld below is .sync.aligned.
-      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
-      if (!ready) break;
-      tc_fence_after();
-      const int r = tm * BM + row_in_tile;
-      const bool row_ok = r < s.M;
-      typename Epi::RowState rs;
-      if (row_ok) epi.row_begin(rs, z, r);
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
-      if constexpr (Epi::kWarpRows) {
-        float* sv = rowstage + (warp - 2) * (NACC * 1024);
-        float* sv2 = sv + (NACC - 1) * 1024;
-        const int row0 = tm * BM + q * 32;
-        const int nrows = min(32, s.M - row0);
-#pragma unroll 1
-        for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
-          const int c0 = tn * BN + c;
-          float v[32], v2[32];
-          tmem_ld32(tbase + c, v);
-          if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            sv[lane * 32 + ((j + lane) & 31)] = v[j];
-            if (NACC == 2) sv2[lane * 32 + ((j + lane) & 31)] = v2[j];
-          }
-          __syncwarp();
-          if (nrows > 0 && c0 < s.N) {
-            const int nv = min(32, s.N - c0);
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-              typename Epi::SpanRegs R;
-              epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
-              epi.finish_span(R, half, z, row0, c0, sv, sv2, nv, nrows, lane);
-            }
-          }
-          __syncwarp();
-        }
-      } else {
+    if constexpr (Epi::kWarpRows) {
+      float* sv = rowstage + (warp - 2) * (NACC * 1024);
+      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, blockIdx.x, gridDim.x, BM, 0, tmem_base, tfull, sv,
+                                          sv + (NACC - 1) * 1024, q, part, lane, abort_flag,
+                                          [&](uint32_t b) { mbar_arrive(&tempty[b]); });
+    } else {
+      uint32_t tcount = 0;
+      for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
+        const int tm = t % p.tiles_m;
+        const int rest = t / p.tiles_m;
+        const int tn = rest % p.tiles_n;
+        const int z = rest / p.tiles_n;
+        const uint32_t buf = tcount & 1u;
+        const uint32_t aph = (tcount >> 1) & 1u;
+        // Warp-uniform decision: tcgen05.ld below is .sync.aligned.
+        const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
+        if (!ready) break;
+        tc_fence_after();
+        const int r = tm * BM + row_in_tile;
+        const bool row_ok = r < s.M;
+        typename Epi::RowState rs;
+        if (row_ok) epi.row_begin(rs, z, r);
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
 #pragma unroll 1
         for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
           float v[32], v2[32];
@@ -405,10 +464,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
           if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
           if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
         }
+        if (row_ok) epi.row_end(rs, z, r, tn * C::PARTS + part);
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
       }
-      if (row_ok) epi.row_end(rs, z, r, tn * C::PARTS + part);
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
     }
   }
 
@@ -493,27 +552,38 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m256(int n, int a_mn, int b_mn
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
-template <int NACC, int BN>
+// DUALB (NACC = 2 only): the two accumulators share A and take two B
+// operands; stage layout [A | B] where CTA 0's B slot holds the whole B1 tile
+// and CTA 1's the whole B2 tile; otherwise [A1 | (A2) | B half].
+template <int NACC, int BN, bool WARPROWS = false, bool DUALB = false>
 struct Cfg2 {
   static constexpr int A_BYTES = BM * BK * 2;            // this CTA's 128 rows
   static constexpr int B_BYTES = (BN / 2) * BK * 2;      // this CTA's BN/2 columns
-  static constexpr int STAGE_BYTES = NACC * A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES;
+  static constexpr int NA = DUALB ? 1 : NACC;            // A slots per stage
+  static constexpr int NB = DUALB ? 2 : 1;               // B slots per stage
+  static constexpr int STAGE_BYTES = NA * A_BYTES + NB * B_BYTES;
+  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EPI_WARPS * NACC * 32 * 32 * 4 : 0;
+  static constexpr int STAGES = ((WARPROWS ? 220 : 200) * 1024 - ROWSTAGE_BYTES) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * NACC * BN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ROWSTAGE_BYTES + 1024 + 256;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(BN % 128 == 0, "each CTA loads whole 64-column boxes of B");
+  static_assert(!DUALB || NACC == 2, "dual B operands need two accumulators");
+  static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(SMEM_BYTES <= 232448, "shared memory above the 227 KiB per-CTA limit");
 };
 
-template <int NACC, int BN, class Epi>
+// mapA2: the second A operand, or with DUALB the second B operand.
+template <int NACC, int BN, class Epi, bool DUALB = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
                 const __grid_constant__ CUtensorMap mapB, const TcParams p, const Epi epi) {
-  using C = Cfg2<NACC, BN>;
+  using C = Cfg2<NACC, BN, Epi::kWarpRows, DUALB>;
   constexpr int HBN = BN / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* rowstage = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::ROWSTAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -563,21 +633,34 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
           const uint32_t ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
           uint8_t* sa = smem + st * C::STAGE_BYTES;
-          uint8_t* sb = sa + NACC * C::A_BYTES;
+          uint8_t* sb = sa + C::NA * C::A_BYTES;
           if (leader) mbar_expect_tx(&full[st], 2 * C::STAGE_BYTES);
           const uint32_t fb = mapa_shared(smem_u32(&full[st]), 0);
           const int k0 = kb * BK;
+          constexpr bool A2 = NACC == 2 && !DUALB;
           if (!p.a_mn) {
             tma_load_3d_pair(sa, &mapA, fb, k0, m0, z);
-            if (NACC == 2) tma_load_3d_pair(sa + C::A_BYTES, &mapA2, fb, k0, m0, z);
+            if (A2) tma_load_3d_pair(sa + C::A_BYTES, &mapA2, fb, k0, m0, z);
           } else {
 #pragma unroll
             for (int j = 0; j < BM / 64; ++j) {
               tma_load_3d_pair(sa + j * 8192, &mapA, fb, m0 + 64 * j, k0, z);
-              if (NACC == 2) tma_load_3d_pair(sa + C::A_BYTES + j * 8192, &mapA2, fb, m0 + 64 * j, k0, z);
+              if (A2) tma_load_3d_pair(sa + C::A_BYTES + j * 8192, &mapA2, fb, m0 + 64 * j, k0, z);
             }
           }
-          if (!p.b_mn) {
+          if constexpr (DUALB) {
+            // CTA 0 stages the whole B1 tile, CTA 1 the whole B2 tile: the
+            // pair's N = 2 BN MMA then reads [B1 | B2] and fills both
+            // accumulators (columns [0, BN) and [BN, 2 BN)) at once.
+            const CUtensorMap* mb = rank == 0 ? &mapB : &mapA2;
+            const int nb0 = tn * BN;
+            if (!p.b_mn) {
+              tma_load_3d_pair(sb, mb, fb, k0, nb0, z);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j) tma_load_3d_pair(sb + j * 8192, mb, fb, nb0 + 64 * j, k0, z);
+            }
+          } else if (!p.b_mn) {
             tma_load_3d_pair(sb, &mapB, fb, k0, n0, z);
           } else {
 #pragma unroll
@@ -595,7 +678,14 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------ MMA issuer (leader) ------------------------------
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_bf16_m256(BN, p.a_mn, p.b_mn);
+      const uint32_t idesc = idesc_bf16_m256(DUALB ? 2 * BN : BN, p.a_mn, p.b_mn);
+      // Descriptors as in the 1-SM kernel: fixed high part | slot address.
+      const uint64_t a_hi = smem_desc_sw128(0, p.a_mn ? 8192 : 16, 1024);
+      const uint64_t b_hi = smem_desc_sw128(0, p.b_mn ? 8192 : 16, 1024);
+      const uint32_t a_ks = p.a_mn ? 2048 >> 4 : 32 >> 4;
+      const uint32_t b_ks = p.b_mn ? 2048 >> 4 : 32 >> 4;
+      constexpr uint32_t a_slot = (uint32_t)(C::A_BYTES >> 4);
+      constexpr int NMMA = DUALB ? 1 : NACC;   // MMAs per k-step
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       const int num_units = p.num_tiles * p.splits;
@@ -614,18 +704,15 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
           if (!mbar_wait(&full[st], ph, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + st * C::STAGE_BYTES);
-          const uint32_t sb = sa + NACC * C::A_BYTES;
+          const uint32_t sb = sa + C::NA * C::A_BYTES;
+          const uint64_t ad = a_hi | (uint64_t)((sa >> 4) & 0x3FFFu);
+          const uint64_t bd = b_hi | (uint64_t)((sb >> 4) & 0x3FFFu);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t bdesc = p.b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
 #pragma unroll
-            for (int a = 0; a < NACC; ++a) {
-              const uint32_t abase = sa + a * C::A_BYTES;
-              const uint64_t adesc = p.a_mn ? smem_desc_sw128(abase + kk * 2048, 8192, 1024)
-                                            : smem_desc_sw128(abase + kk * 32, 16, 1024);
-              mma_bf16_pair(d0 + a * BN, adesc, bdesc, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
-            }
+            for (int a = 0; a < NMMA; ++a)
+              mma_bf16_pair(d0 + a * BN, ad + (kk * a_ks + a * a_slot), bd + kk * b_ks, idesc,
+                            (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty[st]);
         }
@@ -645,6 +732,13 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     uint32_t tcount = 0;
     const int num_units = p.num_tiles * p.splits;
+    if constexpr (Epi::kWarpRows) {   // never split: the launcher keeps splits == 1
+      float* sv = rowstage + (warp - 2) * (NACC * 1024);
+      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, pair, npairs, 2 * BM, (int)rank * BM, tmem_base, tfull, sv,
+                                          sv + (NACC - 1) * 1024, q, part, lane, abort_flag, [&](uint32_t b) {
+                                            mbar_arrive_remote(b ? tempty_leader1 : tempty_leader0);
+                                          });
+    } else
     for (int u = pair; u < num_units; u += npairs, ++tcount) {
       const int t = u / p.splits, ks = u - t * p.splits;
       const int tm = t % p.tiles_m;
@@ -910,13 +1004,14 @@ inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
   return best;
 }
 
-template <int NACC, int BN, class Epi>
+// DUALB: A2 is the second B operand (same layout as B).
+template <int NACC, int BN, class Epi, bool DUALB = false>
 cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
                        cudaStream_t st, int* status, const SplitScratch& ss = SplitScratch()) {
-  using C = Cfg2<NACC, BN>;
+  using C = Cfg2<NACC, BN, Epi::kWarpRows, DUALB>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<NACC, BN, Epi>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<NACC, BN, Epi, DUALB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -926,16 +1021,17 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   cudaError_t e = make_operand_map(&ma, A, s.M, s.K, s.batch, BM);
   if (e != cudaSuccess) return e;
   if (NACC == 2) {
-    e = make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
+    if (DUALB && A2.kmajor != B.kmajor) return cudaErrorInvalidValue;
+    e = DUALB ? make_operand_map(&ma2, A2, s.N, s.K, s.batch, BN) : make_operand_map(&ma2, A2, s.M, s.K, s.batch, BM);
     if (e != cudaSuccess) return e;
   } else {
     ma2 = ma;
   }
-  e = make_operand_map(&mb, B, s.N, s.K, s.batch, BN / 2);
+  e = make_operand_map(&mb, B, s.N, s.K, s.batch, DUALB ? BN : BN / 2);
   if (e != cudaSuccess) return e;
   TcParams p;
   p.s = s;
-  p.dualb = 0;
+  p.dualb = DUALB ? 1 : 0;
   p.a_mn = A.kmajor ? 0 : 1;
   p.b_mn = B.kmajor ? 0 : 1;
   p.tiles_m = (s.M + 2 * BM - 1) / (2 * BM);
@@ -943,14 +1039,14 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
   p.num_kb = (s.K + BK - 1) / BK;
   p.status = status;
-  p.splits = (NACC == 1 && BN == 256) ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
+  p.splits = (NACC == 1 && BN == 256 && !Epi::kWarpRows) ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
   p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
   p.partial = ss.partial;
   p.counters = ss.counters;
   const int pairs = num_sms() / 2;
   const int units = p.num_tiles * p.splits;
   const int grid = 2 * (units < pairs ? units : pairs);
-  gemm_tc2_kernel<NACC, BN, Epi><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
+  gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
 }
 
@@ -978,6 +1074,8 @@ cudaError_t launch_gemm_tc(const GemmShape& s, const Operand& A, const Operand& 
                            const Epi& epi, cudaStream_t st, int* status, const SplitScratch& ss = SplitScratch()) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0 || s.K <= 0) return cudaSuccess;
   if constexpr (NACC == 2) {
+    // Pair tiles (M = 256) halve the B bytes per FLOP; both shapes quantise alike.
+    if (pair_mode() && s.M > BM) return launch_tc2<2, 128, Epi>(s, A, A2, B, epi, st, status);
     return launch_tc<2, 128, Epi>(s, A, A2, B, epi, st, status);
   } else {
     // Expected throughput = fraction of the machine busy x relative rate of
@@ -1011,6 +1109,7 @@ template <class Epi>
 cudaError_t launch_gemm_tc_dualb(const GemmShape& s, const Operand& A, const Operand& B1, const Operand& B2,
                                  const Epi& epi, cudaStream_t st, int* status) {
   if (s.M <= 0 || s.N <= 0 || s.batch <= 0 || s.K <= 0) return cudaSuccess;
+  if (pair_mode() && s.M > BM) return launch_tc2<2, 128, Epi, true>(s, A, B2, B1, epi, st, status);
   return launch_tc<2, 128, Epi>(s, A, B2, B1, epi, st, status, 1);
 }
 
