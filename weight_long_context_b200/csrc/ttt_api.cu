@@ -93,7 +93,7 @@ struct Plan {
   float kscale;  // 1/b for the mean reduction, 1 for the sum
   bool swiglu, has_static;
   size_t esz;  // operand element size
-  size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
+  size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, logits, P, dz, dout, dout_a,
       doutW[2], doutM[2], dU, sk_partial, sk_counters, total;
   size_t sk_partial_bytes, sk_counter_count;
 };
@@ -146,6 +146,9 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.tgt = take(4 * n);
   p.lse = take(4 * n);
   p.ltok = take(4 * n);
+  // bf16 path: the head GEMM of CE pass A also keeps the fp32 logits [n, V],
+  // so pass B is elementwise instead of a second head GEMM.
+  p.logits = take(c.precision == TTT_PREC_BF16 ? 4ull * n * p.V : 0);
   p.P = take(e * n * p.Vs);
   p.dz = take(4 * n * d);
   p.dout = take(4 * n * d);
@@ -205,7 +208,7 @@ enum KernelClass {
 };
 static const char* kClassName[K_NCLASS] = {
     "scalar_scan", "w_shadow", "gather", "mlp_up", "mlp_down", "rmsnorm_fwd", "ce_logits_lse", "ce_rows",
-    "ce_mean", "ce_logits_grad", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update"};
+    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update"};
 
 struct Prof {
   bool timing = false;
@@ -260,6 +263,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   float* lse = reinterpret_cast<float*>(ws + p.lse);
   float* ltok = reinterpret_cast<float*>(ws + p.ltok);
   T* P = reinterpret_cast<T*>(ws + p.P);
+  float* logits = std::is_same<T, float>::value ? nullptr : reinterpret_cast<float*>(ws + p.logits);
   float* dz = reinterpret_cast<float*>(ws + p.dz);
   float* dout = reinterpret_cast<float*>(ws + p.dout);
   T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
@@ -352,7 +356,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E, d, 0, 1, V);
       LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, logits, V}, st, status, ss))));
     }
     LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
            (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
@@ -361,7 +365,12 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
     for (int sl = 0; sl < p.nslabs; ++sl) {
       const int v0 = sl * p.Vs;
       const int vs = V - v0 < p.Vs ? V - v0 : p.Vs;
-      {
+      if (logits) {   // softmax - onehot from the kept logits
+        const int64_t work = (int64_t)n * ((vs + 7) / 8);
+        LAUNCH(K_CE_GRAD, 0, (4.0 + e) * n * vs,
+               (ce_dlogits_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(logits, V, lse, tokens, tm, P,
+                                                                                    p.Vs, v0, vs, n)));
+      } else {        // fp32 path: recompute the slab's logits
         GemmShape s{n, vs, d, 1};
         Operand A = opnd(z, d, 0, 1, n);
         Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
