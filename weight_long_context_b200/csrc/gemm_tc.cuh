@@ -210,6 +210,10 @@ struct TcParams {
   // Split-K (pair kernel): unit u = tile * splits + ks covers k-blocks
   // [ks * kb_per_split, min(num_kb, (ks + 1) * kb_per_split)).
   int splits, kb_per_split;
+  // pair_finish (two splits, every unit resident at once): split 0 finishes
+  // the rows of TMEM lane quarters 0-1, split 1 those of quarters 2-3; a warp
+  // parks only the partial its partner finishes, in [num_tiles][2 CTAs][128 rows][BN].
+  int pair_finish;
   float* partial;   // [num_tiles][splits][2 CTAs][128 rows][BN] fp32 when splits > 1
   int* counters;    // [num_tiles][2 CTAs][EPI_WARPS], zero on entry, left zero on exit
 };
@@ -770,6 +774,73 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
         tc_fence_before();
         mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+      } else if (p.pair_finish) {
+        // Two splits resident at once: each finishes half of the tile's rows.
+        // The warp whose rows the partner finishes parks its fp32 partial and
+        // raises a flag; the finishing warp waits for the flag (bounded), adds
+        // its own accumulator and the partial (two terms: the same sum as
+        // partial 0 + partial 1) and runs the epilogue on its 32 rows.
+        const bool finisher = (ks == 0) == (q < 2);
+        const size_t slab = (size_t)BM * BN;
+        const int ew = warp - 2;
+        float4* region = reinterpret_cast<float4*>(p.partial + ((size_t)t * 2 + rank) * slab) +
+                         (size_t)ew * (PART_COLS / 4) * 32 + lane;
+        int* flag = p.counters + ((size_t)t * 2 + rank) * EPI_WARPS + ew;
+        if (!finisher) {
+#pragma unroll 1
+          for (int c = part * PART_COLS, sp = 0; c < (part + 1) * PART_COLS; c += 32, ++sp) {
+            float v[32];
+            tmem_ld32(tbase + c, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              region[(sp * 8 + i) * 32] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+          tc_fence_before();
+          mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicExch(flag, 1);
+        } else {
+          int ok = 1;
+          if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            while (*reinterpret_cast<volatile int*>(flag) == 0) {
+              if (global_ns() - t0 > WAIT_NS || *abort_flag) {
+                record_error(p.status, TTT_ERR_TIMEOUT);
+                *abort_flag = 1;
+                ok = 0;
+                break;
+              }
+              __nanosleep(100);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          __threadfence();
+          if (ok) {
+            typename Epi::RowState rs;
+            if (row_ok) epi.row_begin(rs, z, r);
+#pragma unroll 1
+            for (int c = part * PART_COLS, sp = 0; c < (part + 1) * PART_COLS; c += 32, ++sp) {
+              float v[32];
+              tmem_ld32(tbase + c, v);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 x = __ldcg(region + (sp * 8 + i) * 32);
+                v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
+              }
+              const int c0 = tn * BN + c;
+              if constexpr (Epi::kPreload) {
+                if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
+              }
+              if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
+            }
+            if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+          }
+          tc_fence_before();
+          mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+          __syncwarp();
+          if (lane == 0) *flag = 0;
+        }
       } else {
         // Split-K: park this split's fp32 partial, free the accumulator, and
         // let the last split to arrive sum all partials in split order.
@@ -945,6 +1016,7 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   p.status = status;
   p.splits = 1;
   p.kb_per_split = p.num_kb;
+  p.pair_finish = 0;
   p.partial = nullptr;
   p.counters = nullptr;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
@@ -1004,6 +1076,17 @@ inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
   return best;
 }
 
+// 1: two-split GEMMs finish half of each tile per split (env TTT_GEMM_PAIRFINISH=0
+// keeps the last-arriver reduction, for A/B timing).
+inline int pair_finish_mode() {
+  static int m = -1;
+  if (m < 0) {
+    const char* e = getenv("TTT_GEMM_PAIRFINISH");
+    m = (e && e[0] == '0') ? 0 : 1;
+  }
+  return m;
+}
+
 // DUALB: A2 is the second B operand (same layout as B).
 template <int NACC, int BN, class Epi, bool DUALB = false>
 cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
@@ -1045,6 +1128,9 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   p.counters = ss.counters;
   const int pairs = num_sms() / 2;
   const int units = p.num_tiles * p.splits;
+  // Finishing warps wait for their partner split, so both splits of every
+  // tile must be resident together: one wave of units, two splits.
+  p.pair_finish = (p.splits == 2 && units <= pairs && pair_finish_mode()) ? 1 : 0;
   const int grid = 2 * (units < pairs ? units : pairs);
   gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
