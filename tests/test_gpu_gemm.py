@@ -45,14 +45,17 @@ def test_gemm_rejects_unaligned_strides(dev):
     assert ei.value.code == 3
 
 
-SPLITK = [(1024, 2048, 5632, 1), (1024, 2048, 11264, 1), (512, 520, 4096, 2), (296, 264, 1000, 1)]
+SPLITK = [(1024, 2048, 5632, 1), (1024, 2048, 11264, 1), (512, 520, 4096, 2), (296, 264, 1000, 1),
+          # whole waves of tiles plus a last wave finished as paired halves
+          (1024, 11264, 2048, 1), (1024, 5632, 2048, 1), (1000, 5600, 1000, 1)]
 
 
 @pytest.mark.parametrize("b_k", [True, False])
 @pytest.mark.parametrize("shape", SPLITK, ids=[f"{m}x{n}x{k}b{z}" for m, n, k, z in SPLITK])
 def test_gemm_split_k(dev, shape, b_k):
-    """With a workspace the engine may split K across CTA pairs and reduce the
-    fp32 partials in a fixed order: same result as without, bit for bit."""
+    """With a workspace the engine may split K across CTA pairs (every tile, or
+    only the tiles of the last wave) and add the fp32 partials in a fixed
+    order: accurate, and the same bits on every run."""
     from weight_long_context_b200 import ttt
     M, N, K, Z = shape
     g = torch.Generator(device="cpu").manual_seed(M + N + K)

@@ -210,13 +210,44 @@ struct TcParams {
   // Split-K (pair kernel): unit u = tile * splits + ks covers k-blocks
   // [ks * kb_per_split, min(num_kb, (ks + 1) * kb_per_split)).
   int splits, kb_per_split;
-  // pair_finish (two splits, every unit resident at once): split 0 finishes
-  // the rows of TMEM lane quarters 0-1, split 1 those of quarters 2-3; a warp
-  // parks only the partial its partner finishes, in [num_tiles][2 CTAs][128 rows][BN].
-  int pair_finish;
+  // pair_finish: tiles [0, full_tiles) run whole, the remaining tiles as two
+  // halves of the k-blocks (units full_tiles + 2 i, + 1), all of them in the
+  // last wave so both halves of a tile are resident at once; half 0 finishes
+  // the rows of TMEM lane quarters 0-1, half 1 those of quarters 2-3, and a
+  // warp parks only the partial its partner finishes, in
+  // [tile - full_tiles][2 CTAs][128 rows][BN].
+  int pair_finish, full_tiles, num_units;
   float* partial;   // [num_tiles][splits][2 CTAs][128 rows][BN] fp32 when splits > 1
   int* counters;    // [num_tiles][2 CTAs][EPI_WARPS], zero on entry, left zero on exit
 };
+
+// Work unit u of the pair kernel: tile t, k-blocks [kb0, kb1), split index ks.
+struct Unit {
+  int t, ks, kb0, kb1;
+  bool split;
+};
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
+  Unit x;
+  if (p.pair_finish) {
+    if (u < p.full_tiles) {
+      x.t = u; x.ks = 0; x.kb0 = 0; x.kb1 = p.num_kb; x.split = false;
+    } else {
+      const int v = u - p.full_tiles;
+      x.t = p.full_tiles + (v >> 1);
+      x.ks = v & 1;
+      x.kb0 = x.ks ? p.kb_per_split : 0;
+      x.kb1 = x.ks ? p.num_kb : p.kb_per_split;
+      x.split = true;
+    }
+  } else {
+    x.t = u / p.splits;
+    x.ks = u - x.t * p.splits;
+    x.kb0 = x.ks * p.kb_per_split;
+    x.kb1 = min(p.num_kb, x.kb0 + p.kb_per_split);
+    x.split = p.splits > 1;
+  }
+  return x;
+}
 
 // Row-walking epilogue loop shared by both kernels: each 32 x 32 span of the
 // warp's accumulators is staged in shared memory (sv / sv2, rotated so the
@@ -621,18 +652,16 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      const int num_units = p.num_tiles * p.splits;
-      for (int u = pair; u < num_units && ok; u += npairs) {
-        const int t = u / p.splits, ks = u - t * p.splits;
+      for (int u = pair; u < p.num_units && ok; u += npairs) {
+        const Unit un = decode_unit(p, u);
+        const int t = un.t;
         const int tm = t % p.tiles_m;
         const int rest = t / p.tiles_m;
         const int tn = rest % p.tiles_n;
         const int z = rest / p.tiles_n;
         const int m0 = tm * 2 * BM + (int)rank * BM;     // this CTA's 128 rows
         const int n0 = tn * BN + (int)rank * HBN;        // this CTA's BN/2 columns
-        const int kb0 = ks * p.kb_per_split;
-        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
           const int st = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
@@ -692,11 +721,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       constexpr int NMMA = DUALB ? 1 : NACC;   // MMAs per k-step
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      const int num_units = p.num_tiles * p.splits;
-      for (int u = pair; u < num_units && ok; u += npairs, ++tcount) {
-        const int ks = u % p.splits;
-        const int kb0 = ks * p.kb_per_split;
-        const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+      for (int u = pair; u < p.num_units && ok; u += npairs, ++tcount) {
+        const Unit un = decode_unit(p, u);
+        const int kb0 = un.kb0, kb1 = un.kb1;
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
         if (!mbar_wait(&tempty[buf], aph ^ 1u, abort_flag, p.status)) { ok = false; break; }
@@ -735,7 +762,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     uint32_t tcount = 0;
-    const int num_units = p.num_tiles * p.splits;
     if constexpr (Epi::kWarpRows) {   // never split: the launcher keeps splits == 1
       float* sv = rowstage + (warp - 2) * (NACC * 1024);
       warp_rows_loop<NACC, BN, PART_COLS>(epi, p, pair, npairs, 2 * BM, (int)rank * BM, tmem_base, tfull, sv,
@@ -743,8 +769,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
                                             mbar_arrive_remote(b ? tempty_leader1 : tempty_leader0);
                                           });
     } else
-    for (int u = pair; u < num_units; u += npairs, ++tcount) {
-      const int t = u / p.splits, ks = u - t * p.splits;
+    for (int u = pair; u < p.num_units; u += npairs, ++tcount) {
+      const Unit un = decode_unit(p, u);
+      const int t = un.t, ks = un.ks;
       const int tm = t % p.tiles_m;
       const int rest = t / p.tiles_m;
       const int tn = rest % p.tiles_n;
@@ -757,7 +784,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       const int r = tm * 2 * BM + (int)rank * BM + row_in_tile;
       const bool row_ok = r < s.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
-      if (p.splits == 1) {
+      if (!un.split) {
         typename Epi::RowState rs;
         if (row_ok) epi.row_begin(rs, z, r);
 #pragma unroll 1
@@ -783,7 +810,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         const bool finisher = (ks == 0) == (q < 2);
         const size_t slab = (size_t)BM * BN;
         const int ew = warp - 2;
-        float4* region = reinterpret_cast<float4*>(p.partial + ((size_t)t * 2 + rank) * slab) +
+        float4* region = reinterpret_cast<float4*>(p.partial + ((size_t)(t - p.full_tiles) * 2 + rank) * slab) +
                          (size_t)ew * (PART_COLS / 4) * 32 + lane;
         int* flag = p.counters + ((size_t)t * 2 + rank) * EPI_WARPS + ew;
         if (!finisher) {
@@ -1017,6 +1044,8 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   p.splits = 1;
   p.kb_per_split = p.num_kb;
   p.pair_finish = 0;
+  p.full_tiles = p.num_tiles;
+  p.num_units = p.num_tiles;
   p.partial = nullptr;
   p.counters = nullptr;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
@@ -1033,6 +1062,41 @@ inline double tile_efficiency(const GemmShape& s, int bn) {
   const long tiles = (long)((s.M + BM - 1) / BM) * ((s.N + bn - 1) / bn) * s.batch;
   const long waves = (tiles + sms - 1) / sms;
   return (double)tiles / (double)(waves * sms) * (bn == 128 ? 0.78 : 1.0);
+}
+
+// 1: pair-kernel GEMMs may finish the tiles of their last wave as paired halves (env TTT_GEMM_PAIRFINISH=0
+// keeps the last-arriver reduction, for A/B timing).
+inline int pair_finish_mode() {
+  static int m = -1;
+  if (m < 0) {
+    const char* e = getenv("TTT_GEMM_PAIRFINISH");
+    m = (e && e[0] == '0') ? 0 : 1;
+  }
+  return m;
+}
+
+// Paired-finish schedule of a pair-kernel GEMM: the whole waves of tiles run
+// whole, the tiles of the last partial wave as two halves of the k-blocks
+// (2 x remainder <= pairs, so all halves are resident together and each pair
+// runs at most one).  Cost in k-blocks of one pair: whole waves x num_kb +
+// half a tile + PF_FIXUP_KB for parking and adding half a partial.  Returns
+// the number of whole tiles, or -1 when the plain whole-tile schedule is cheaper
+// or the scratch is missing.
+constexpr int PF_FIXUP_KB = 4;
+inline long paired_finish_plan(long tiles, int num_kb, const SplitScratch& ss, double* cost = nullptr) {
+  const int pairs = num_sms() / 2;
+  const long full = tiles / pairs * pairs;
+  const long rem = tiles - full;
+  const double whole = (double)((tiles + pairs - 1) / pairs) * num_kb;
+  if (cost) *cost = whole;
+  if (!pair_finish_mode() || rem == 0 || 2 * rem > pairs || num_kb < 2) return -1;
+  if (!ss.partial || !ss.counters) return -1;
+  if ((size_t)rem * 2 * BM * 256 * sizeof(float) > ss.partial_bytes) return -1;
+  if ((size_t)tiles * 2 * EPI_WARPS > ss.counter_count) return -1;
+  const double pf = (double)(full / pairs) * num_kb + (num_kb + 1) / 2 + PF_FIXUP_KB;
+  if (pf >= whole) return -1;
+  if (cost) *cost = pf;
+  return full;
 }
 
 // Split count for a pair-kernel GEMM: minimise waves x (k-blocks per split +
@@ -1076,17 +1140,6 @@ inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
   return best;
 }
 
-// 1: two-split GEMMs finish half of each tile per split (env TTT_GEMM_PAIRFINISH=0
-// keeps the last-arriver reduction, for A/B timing).
-inline int pair_finish_mode() {
-  static int m = -1;
-  if (m < 0) {
-    const char* e = getenv("TTT_GEMM_PAIRFINISH");
-    m = (e && e[0] == '0') ? 0 : 1;
-  }
-  return m;
-}
-
 // DUALB: A2 is the second B operand (same layout as B).
 template <int NACC, int BN, class Epi, bool DUALB = false>
 cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, const Operand& B, const Epi& epi,
@@ -1122,15 +1175,25 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
   p.num_kb = (s.K + BK - 1) / BK;
   p.status = status;
-  p.splits = (NACC == 1 && BN == 256 && !Epi::kWarpRows) ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
-  p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
+  const bool may_split = NACC == 1 && BN == 256 && !Epi::kWarpRows;
+  const long full = may_split ? paired_finish_plan(p.num_tiles, p.num_kb, ss) : -1;
+  if (full >= 0) {   // whole waves, then the last wave's tiles as paired halves
+    p.pair_finish = 1;
+    p.full_tiles = (int)full;
+    p.splits = 2;
+    p.kb_per_split = (p.num_kb + 1) / 2;
+    p.num_units = (int)full + 2 * (p.num_tiles - (int)full);
+  } else {
+    p.pair_finish = 0;
+    p.full_tiles = p.num_tiles;
+    p.splits = may_split ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
+    p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
+    p.num_units = p.num_tiles * p.splits;
+  }
   p.partial = ss.partial;
   p.counters = ss.counters;
   const int pairs = num_sms() / 2;
-  const int units = p.num_tiles * p.splits;
-  // Finishing warps wait for their partner split, so both splits of every
-  // tile must be resident together: one wave of units, two splits.
-  p.pair_finish = (p.splits == 2 && units <= pairs && pair_finish_mode()) ? 1 : 0;
+  const int units = p.num_units;
   const int grid = 2 * (units < pairs ? units : pairs);
   gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
@@ -1172,13 +1235,19 @@ cudaError_t launch_gemm_tc(const GemmShape& s, const Operand& A, const Operand& 
     if (pair_mode() && s.M > BM) {
       const long tiles = (long)((s.M + 2 * BM - 1) / (2 * BM)) * ((s.N + 255) / 256) * s.batch;
       const int num_kb = (s.K + BK - 1) / BK;
-      const int S = choose_splits(tiles, num_kb, ss);
       const int pairs = num_sms() / 2;
-      const long units = tiles * S;
-      const long waves = (units + pairs - 1) / pairs;
-      const int kbps = (num_kb + S - 1) / S;
-      // useful k-blocks over issued k-block slots (with the split overhead)
-      s_pair = 1.3 * (double)tiles * num_kb / ((double)waves * pairs * (kbps + (S > 1 ? 4 : 0)));
+      double cost = 0.0;
+      if (paired_finish_plan(tiles, num_kb, ss, &cost) >= 0) {
+        // useful k-blocks over issued k-block slots of the paired-finish schedule
+        s_pair = 1.3 * (double)tiles * num_kb / ((double)pairs * cost);
+      } else {
+        const int S = choose_splits(tiles, num_kb, ss);
+        const long units = tiles * S;
+        const long waves = (units + pairs - 1) / pairs;
+        const int kbps = (num_kb + S - 1) / S;
+        // useful k-blocks over issued k-block slots (with the split overhead)
+        s_pair = 1.3 * (double)tiles * num_kb / ((double)waves * pairs * (kbps + (S > 1 ? 4 : 0)));
+      }
     }
     const double s256 = tile_efficiency(s, 256);
     const double s128 = Epi::kFixedHeadTile ? 0.0 : tile_efficiency(s, 128);
