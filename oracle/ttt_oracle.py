@@ -365,6 +365,34 @@ def chunk_update_explicit(W, M, grads, eta, beta, gamma, gscale=1.0):
     return newW, newM
 
 
+def chunk_update_lact(W, M, grads, eta, beta, gamma, gscale=1.0):
+    """LaCT's chunk-wise rule ([E2-TTT] 高效的逐块（Chunk-wise）更新机制): a single
+    update direction for the chunk, the negative gradient of the eta-weighted
+    sum of the token losses at the chunk-start weights,
+      G = -grad sum_t eta_t l_t = sum_t eta_t G_t,
+    a momentum factor averaged over the chunk, and no decay:
+      M_C = (1/C sum_t beta_t) M_0 + G,   W_C = W_0 + M_C.
+    gamma is not used by this rule."""
+    bbar = float(np.mean(np.asarray(beta, dtype=np.float64)))
+    e = np.asarray(eta, dtype=np.float64)
+    newW, newM = [], []
+    for l in range(len(W)):
+        bw, bm = [], []
+        for j in range(len(W[l])):
+            Lf, Rf = grads[l][j]
+            dt = W[l][j].dtype
+            G = (-gscale * ((Lf * e[:, None].astype(Lf.dtype)).T @ Rf)).astype(dt)
+            Mn = (dt.type(bbar) * M[l][j] + G).astype(dt)
+            bw.append((W[l][j] + Mn).astype(dt))
+            bm.append(Mn)
+        newW.append(bw)
+        newM.append(bm)
+    return newW, newM
+
+
+UPDATE_RULES = ("closed", "explicit", "lact")
+
+
 # ---------------------------------------------------------------------------
 # The inner loop over a whole sequence
 # ---------------------------------------------------------------------------
@@ -389,7 +417,10 @@ def prefill_sequence(model: Model, W0, M0, hidden, tokens, eta, beta, gamma, b,
     W = [[m.copy() for m in blk] for blk in W0]
     M = [[m.copy() for m in blk] for blk in M0]
     losses = np.zeros(nc, dtype=np.float64)
-    step = chunk_update_closed if update == "closed" else chunk_update_explicit
+    if update not in UPDATE_RULES:
+        raise ValueError("update must be one of " + ", ".join(UPDATE_RULES))
+    # looked up at call time (the pins substitute planted mistakes)
+    step = {"closed": chunk_update_closed, "explicit": chunk_update_explicit, "lact": chunk_update_lact}[update]
     for c in range(nc):
         s = slice(c * b, (c + 1) * b)
         X = hidden[s]

@@ -249,6 +249,57 @@ def test_chunked_sgd_uses_chunk_start_gradients(red):
 
 
 # ---------------------------------------------------------------------------
+# 4b. LaCT's chunk-wise rule ([E2-TTT] 高效的逐块（Chunk-wise）更新机制)
+# ---------------------------------------------------------------------------
+
+def test_lact_without_momentum_matches_closed_form_w():
+    """beta = 0: LaCT's W_C = W_0 + sum_t eta_t G_t, which is also the E2-TTT
+    chunk end with beta = 0, gamma = 1; LaCT's M_C is the whole chunk step."""
+    s = tiny_setup(kind="swiglu", d=4, h=6, V=7, L=2, static=True, T=8, seed=3)
+    T = len(s["eta"])
+    Wl, Ml, _ = run_prefill(s, 4, update="lact", beta=np.zeros(T), gamma=s["gamma"])
+    Wc, _, _ = run_prefill(s, 4, update="closed", beta=np.zeros(T), gamma=np.ones(T))
+    assert rel(Wl, Wc) < 1e-12
+    # the last chunk's step is the last chunk's M
+    Wp, _, _ = run_prefill(s, 4, update="lact", beta=np.zeros(T), gamma=s["gamma"],
+                           X=s["X"][:4], y=s["y"][:4], eta=s["eta"][:4])
+    assert rel(Ml, Wl - Wp) < 1e-10
+
+
+@pytest.mark.parametrize("red", ["mean", "sum"])
+def test_lact_direction_is_gradient_of_weighted_loss(red):
+    """One chunk from M_0 = 0: M_C = -grad_W sum_t eta_t l_t (l_t / b for the
+    mean reduction) at W_0, taken by torch autograd of an independent model."""
+    s = tiny_setup(kind="gelu", d=5, h=7, V=9, L=1, static=False, T=6, seed=4, m0=0.0)
+    W, M, _ = run_prefill(s, 6, update="lact", reduction=red)
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    Wv = T_(s["W0"]).requires_grad_(True)
+    l = AM.losses("gelu", 5, 7, 1, 1e-6, T_(s["E"]), T_(s["g"]), None, Wv, T_(s["X"]), torch.tensor(s["y"]))
+    scale = 1.0 / 6 if red == "mean" else 1.0
+    (g,) = torch.autograd.grad((T_(s["eta"]) * l).sum() * scale, Wv)
+    assert rel(M, (-g).numpy()) < 1e-12
+    assert rel(W, (T_(s["W0"]) - g).numpy()) < 1e-12
+
+
+def test_lact_momentum_factor_is_the_chunk_average():
+    """beta alternating 0, 1 averages to 1/2 exactly (a product would give 0,
+    the last token's factor 1): M_C - M_C(M_0 = 0) = M_0 / 2."""
+    s = tiny_setup(kind="gelu", d=4, h=5, V=6, L=1, static=False, T=4, seed=5, m0=0.3)
+    beta = np.array([0.0, 1.0, 0.0, 1.0])
+    _, M, _ = run_prefill(s, 4, update="lact", beta=beta)
+    _, M0run, _ = run_prefill(s, 4, update="lact", beta=beta, M0=np.zeros_like(s["M0"]))
+    assert rel(M - M0run, 0.5 * s["M0"]) < 1e-12
+
+
+def test_lact_ignores_decay():
+    """LaCT's rule has no decay term: gamma does not change the result."""
+    s = tiny_setup(kind="gelu", d=4, h=5, V=6, L=1, static=False, T=8, seed=6)
+    W1, M1, _ = run_prefill(s, 4, update="lact", gamma=np.full(8, 0.5))
+    W2, M2, _ = run_prefill(s, 4, update="lact", gamma=np.ones(8))
+    assert rel(W1, W2) == 0.0 and rel(M1, M2) == 0.0
+
+
+# ---------------------------------------------------------------------------
 # 5. Cross-entropy closed forms
 # ---------------------------------------------------------------------------
 
@@ -391,6 +442,16 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "chunk_backward", _bwd_no_proj)
     _must_fail(test_gradients_match_finite_differences, "swiglu")
     monkeypatch.undo()
+
+    # (g) LaCT: the product of the momentum factors instead of their average
+    orig_lact = O.chunk_update_lact
+
+    def lact_prod(W, M, grads, eta, beta, gamma, gscale=1.0):
+        b = np.full(len(beta), np.prod(np.asarray(beta, dtype=np.float64)) ** (1.0 / len(beta)))
+        return orig_lact(W, M, grads, eta, b, gamma, gscale)
+    monkeypatch.setattr(O, "chunk_update_lact", lact_prod)
+    _must_fail(test_lact_momentum_factor_is_the_chunk_average)
+    monkeypatch.setattr(O, "chunk_update_lact", orig_lact)
 
     # (f) the residual dropped from the backward of a block
     orig_mb = O.mlp_backward
