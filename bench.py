@@ -216,7 +216,7 @@ def oracle_chunks(w: I.Workload, n_chunks: int, seed: int = 0):
                               x["static_w"], dtype=dtype)
     t0 = time.perf_counter()
     oracle.prefill(model, x["W0"], x["M0"], x["hidden"], x["tokens"], x["eta"], x["beta"], x["gamma"], w.b,
-                   dtype=dtype, reduction=w.reduction)
+                   dtype=dtype, reduction=w.reduction, update="lact" if w.update_rule == "lact" else "closed")
     return time.perf_counter() - t0
 
 
@@ -271,7 +271,7 @@ def workload_config(w: I.Workload) -> dict:
     big = input_bytes(w) + state_bytes(w) > 2 * L2_BYTES
     return {"workload": w.name, "d": w.d, "hidden": w.hidden, "vocab": w.vocab, "blocks": w.n_blocks,
             "mlp": w.mlp, "static_mlp": w.has_static, "T": w.T, "chunk_b": w.b, "sequences_per_gpu": w.batch,
-            "scalars": w.scalars, "loss_reduction": w.reduction,
+            "scalars": w.scalars, "loss_reduction": w.reduction, "update_rule": w.update_rule,
             "precision": "fp32" if w.precision == "fp32" else "bf16 GEMM operands, fp32 accumulate/state",
             "l2": ("inputs larger than L2 (hidden + fast-weight state %.2f GiB per step)" % ((input_bytes(w) + state_bytes(w)) / 2 ** 30))
                   if big else "L2 flushed between timed steps (write of a 256 MiB buffer)"}
@@ -296,7 +296,7 @@ def run_ours(args, w: I.Workload):
     T = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
     h = ttt.Handle(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.has_static, w.precision, T(x["lm_head"]),
                    T(x["rms_gain"]), T(x["static_w"]) if x["static_w"] is not None else None, w.rms_eps,
-                   w.reduction)
+                   w.reduction, w.update_rule)
     hidden, tokens = T(x["hidden"]), T(x["tokens"], torch.int32)
     W, M = T(x["W0"]), T(x["M0"])
     eta, beta, gamma = T(x["eta"]), T(x["beta"]), T(x["gamma"])
@@ -420,6 +420,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--update-rule", default="e2ttt", choices=["e2ttt", "lact"],
+                    help="chunk update rule: Proposition 3.1 (default) or LaCT's chunk-wise rule")
     ap.add_argument("--chunks", type=int, default=0,
                     help="profiling captures only: run the first N chunks of each sequence instead of the full T "
                          "(every launch keeps its full-size shape; the line's config names the reduced T)")
@@ -429,6 +431,8 @@ def main(argv=None):
     w = I.WORKLOADS[args.workload]
     if args.chunks > 0:
         w = w.with_(T=min(w.T, args.chunks * w.b))
+    if args.update_rule != w.update_rule:
+        w = w.with_(update_rule=args.update_rule)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -70,6 +70,7 @@ typedef enum ttt_status {
 enum { TTT_MLP_GELU = 0, TTT_MLP_SWIGLU = 1 };
 enum { TTT_PREC_FP32 = 0, TTT_PREC_BF16 = 1 };
 enum { TTT_REDUCE_MEAN = 0, TTT_REDUCE_SUM = 1 };
+enum { TTT_RULE_E2TTT = 0, TTT_RULE_LACT = 1 };
 
 /* Model shape.  d, hidden, vocab: multiples of 16, at least 16, and
  * d <= 16384, hidden <= 65536, vocab < 2^26.  n_blocks in [1, 64].
@@ -84,7 +85,13 @@ enum { TTT_REDUCE_MEAN = 0, TTT_REDUCE_SUM = 1 };
  * the recursion is l_t / b, so beta = 0, gamma = 1, eta = alpha is one SGD
  * step on the chunk's mean loss and b = 1 is online SGD.  TTT_REDUCE_SUM:
  * l_t itself (the second sketch's reduction='sum').  The reported chunk loss
- * is the mean either way. */
+ * is the mean either way.
+ * update_rule: how a chunk's per-token gradients G_t become the chunk-end
+ * state.  TTT_RULE_E2TTT: Proposition 3.1 of [E2-TTT] (命题3.1), the exact
+ * chunk end of M_t = beta_t M_{t-1} + eta_t G_t, W_t = gamma_t W_{t-1} + M_t.
+ * TTT_RULE_LACT: LaCT's chunk-wise rule as [E2-TTT] states it (高效的逐块
+ * 更新机制): G = sum_t eta_t G_t, M_C = (mean_t beta_t) M_0 + G,
+ * W_C = W_0 + M_C (gamma unused). */
 typedef struct ttt_config {
   int32_t d;
   int32_t hidden;
@@ -95,6 +102,7 @@ typedef struct ttt_config {
   int32_t precision;  /* TTT_PREC_FP32 or TTT_PREC_BF16 */
   int32_t loss_reduction; /* TTT_REDUCE_MEAN or TTT_REDUCE_SUM */
   float rms_eps;
+  int32_t update_rule; /* TTT_RULE_E2TTT or TTT_RULE_LACT */
 } ttt_config;
 
 typedef struct ttt_handle ttt_handle;
@@ -178,14 +186,22 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
                                 const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
                                 void* stream, ttt_kernel_stat* stats, int32_t max_stats, int32_t* n_stats);
 
-/* The scalar kernels of Proposition 3.1 for every chunk, on the device
- * ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1; computed in the division-free form
- * K_W_t = eta_t sum_{j>=t} (prod_{i=t+1}^{j} beta_i) gtilde_j, float64 inside).
+/* The per-token and per-chunk coefficients of a chunk update rule for every
+ * chunk, on the device.  rule = TTT_RULE_E2TTT: the scalar kernels of
+ * Proposition 3.1 ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1; computed in the
+ * division-free form K_W_t = eta_t sum_{j>=t} (prod_{i=t+1}^{j} beta_i)
+ * gtilde_j, float64 inside).  rule = TTT_RULE_LACT: K_W_t = K_M_t = eta_t and
+ * the chunk's mean momentum factor ([E2-TTT] 高效的逐块更新机制).
  *   eta, beta, gamma [batch, T]  in
- *   KW, KM [batch, T]            out: eta_t btilde_t R_t and eta_t btilde_t
- *   consts [batch, T/b, 4]       out: (gtilde_0, btilde_0, btilde_0 R_1, 0)
- * T % b == 0 required.  No handle needed; asynchronous on `stream`. */
-ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* eta,
+ *   KW, KM [batch, T]            out: E2TTT: eta_t btilde_t R_t and eta_t btilde_t;
+ *                                     LaCT: eta_t and eta_t
+ *   consts [batch, T/b, 4]       out: (coefficient of W_0 in W_C, of M_0 in M_C,
+ *                                     of M_0 in W_C, 0): E2TTT (gtilde_0,
+ *                                     btilde_0, btilde_0 R_1, 0); LaCT (1, mean
+ *                                     beta, mean beta, 0)
+ * T % b == 0 required; an unknown rule is TTT_ERR_INVALID_ARG.  No handle
+ * needed; asynchronous on `stream`. */
+ttt_status ttt_scalar_kernels(int32_t rule, int32_t batch, int32_t T, int32_t b, const float* eta,
                               const float* beta, const float* gamma, float* KW, float* KM,
                               float* consts, void* stream);
 

@@ -26,7 +26,8 @@ def oracle_model(w, x):
 def run_oracle(w, x, dtype=np.float64, n_chunks=None):
     model = oracle_model(w, x)
     return oracle.prefill(model, x["W0"], x["M0"], x["hidden"], x["tokens"], x["eta"], x["beta"],
-                          x["gamma"], w.b, dtype=dtype, n_chunks=n_chunks, reduction=w.reduction)
+                          x["gamma"], w.b, dtype=dtype, n_chunks=n_chunks, reduction=w.reduction,
+                          update="lact" if w.update_rule == "lact" else "closed")
 
 
 def make_handle(w, x, dev):
@@ -36,7 +37,7 @@ def make_handle(w, x, dev):
     return ttt.Handle(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.has_static, w.precision,
                       T(x["lm_head"]), T(x["rms_gain"]),
                       T(x["static_w"]) if x["static_w"] is not None else None, w.rms_eps,
-                      w.reduction)
+                      w.reduction, w.update_rule)
 
 
 def run_gpu(w, x, dev, handle=None, return_handle=False):

@@ -60,9 +60,17 @@ def test_config_validation_is_host_side(lib):
 
 def test_scalar_kernels_shape_validation(lib):
     z = ctypes.c_void_p(16)
-    assert lib.ttt_scalar_kernels(1, 10, 3, z, z, z, z, z, z, None) == 2
-    assert lib.ttt_scalar_kernels(1, 10, 0, z, z, z, z, z, z, None) == 2
-    assert lib.ttt_scalar_kernels(0, 0, 4, z, z, z, z, z, z, None) == 0
+    for rule in (0, 1):   # E2TTT, LaCT
+        assert lib.ttt_scalar_kernels(rule, 1, 10, 3, z, z, z, z, z, z, None) == 2
+        assert lib.ttt_scalar_kernels(rule, 1, 10, 0, z, z, z, z, z, z, None) == 2
+        assert lib.ttt_scalar_kernels(rule, 0, 0, 4, z, z, z, z, z, z, None) == 0
+    assert lib.ttt_scalar_kernels(2, 0, 0, 4, z, z, z, z, z, z, None) == 1   # unknown rule
+
+
+def test_create_rejects_unknown_update_rule(lib):
+    C = ttt.ttt_config
+    assert _create(lib, C(32, 32, 32, 1, 0, 0, 0, 0, 1e-6, 2)) == 1
+    assert b"update_rule" in lib.ttt_last_error()
 
 
 def test_prefill_rejects_null_handle(lib):

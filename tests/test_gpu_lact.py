@@ -1,0 +1,76 @@
+"""LaCT's chunk-wise update rule on the GPU ("Rethinking Expressivity and
+Efficiency in Test-Time Training", 高效的逐块（Chunk-wise）更新机制):
+G = sum_t eta_t G_t, M_C = (mean_t beta_t) M_0 + G, W_C = W_0 + M_C, against the
+oracle's direct statement of the rule."""
+import numpy as np
+import pytest
+import torch
+
+from tests import helpers as H
+from weight_long_context_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+@pytest.mark.parametrize("b", [1, 16, 64, 1024])
+def test_lact_coefficients(dev, b):
+    from weight_long_context_b200 import ttt
+    rng = np.random.default_rng(b + 7)
+    B, nc = 2, 3
+    T = b * nc
+    eta = (0.01 / (1 + np.exp(-rng.normal(size=(B, T))))).astype(np.float32)
+    beta = rng.uniform(0.8, 0.99, (B, T)).astype(np.float32)
+    gamma = rng.uniform(0.99, 1.0, (B, T)).astype(np.float32)
+    t = lambda a: torch.from_numpy(a).to(dev)
+    KW, KM, consts = ttt.ttt_scalar_kernels(t(eta), t(beta), t(gamma), b, rule="lact")
+    KW, KM, consts = KW.cpu().numpy(), KM.cpu().numpy(), consts.cpu().numpy()
+    assert np.array_equal(KW, eta) and np.array_equal(KM, eta)
+    for s in range(B):
+        for c in range(nc):
+            bbar = float(np.mean(beta[s, c * b:(c + 1) * b].astype(np.float64)))
+            np.testing.assert_allclose(consts[s, c], [1.0, bbar, bbar, 0.0], rtol=1e-6, atol=0)
+
+
+RAGGED = [
+    # name, d, h, V, L, mlp, static, T, b, batch
+    ("gelu_1blk", 80, 208, 528, 1, "gelu", False, 72, 24, 2),
+    ("swiglu_2blk_static", 48, 80, 272, 2, "swiglu", True, 60, 20, 2),
+]
+
+
+@pytest.mark.parametrize("precision", ["fp32", "bf16"])
+@pytest.mark.parametrize("case", RAGGED, ids=[c[0] for c in RAGGED])
+def test_lact_ragged_parity(dev, case, precision):
+    name, d, h, V, L, mlp, st, T, b, B = case
+    w = I.Workload(name, d, h, V, L, mlp, st, precision, T, b, B, "e2ttt", update_rule="lact")
+    x = I.make_inputs(w, seed=11, m0_scale=0.01, w0_per_sequence=True)
+    e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x))
+    print(name, precision, e)
+
+
+def test_lact_full_dims_first_chunks(dev):
+    """The 128K stack's shapes (the benchmark's launch configuration), first
+    two chunks, under the LaCT rule."""
+    w = I.WORKLOADS["stack_128k"]
+    w = w.with_(T=2 * w.b, update_rule="lact")
+    x = I.make_inputs(w, seed=0, m0_scale=1e-3)
+    e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x, dtype=np.float32))
+    print("stack_128k lact", e)
+
+
+def test_rules_differ(dev):
+    """The two rules are different updates of the same inputs (M_0 != 0)."""
+    name, d, h, V, L, mlp, st, T, b, B = RAGGED[0]
+    w = I.Workload(name, d, h, V, L, mlp, st, "fp32", T, b, B, "e2ttt")
+    x = I.make_inputs(w, seed=2, m0_scale=0.05)
+    Wa, Ma, _, sa = H.run_gpu(w, x, dev)
+    Wb, Mb, _, sb = H.run_gpu(w.with_(update_rule="lact"), x, dev)
+    assert sa == 0 and sb == 0
+    assert H.rel_fro(Ma, Mb) > 1e-3

@@ -105,14 +105,51 @@ __global__ void scalar_scan_kernel(const float* __restrict__ eta, const float* _
   }
 }
 
-inline cudaError_t launch_scalar_scan(const float* eta, const float* beta, const float* gamma,
+// LaCT's chunk-wise rule as "Rethinking Expressivity and Efficiency in
+// Test-Time Training" states it (高效的逐块（Chunk-wise）更新机制): one direction
+// G = sum_t eta_t G_t, M_C = (mean_t beta_t) M_0 + G, W_C = W_0 + M_C.  In the
+// update GEMM's terms K_W = K_M = eta and consts = (1, bbar, bbar, 0).  One warp
+// per chunk; the mean of beta is summed in float64 in a fixed order.
+__global__ void lact_scan_kernel(const float* __restrict__ eta, const float* __restrict__ beta, int T, int b,
+                                 int nchunks, float* __restrict__ KW, float* __restrict__ KM,
+                                 float* __restrict__ consts) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t job = (int64_t)blockIdx.x * warps + (threadIdx.x >> 5);
+  const int s = blockIdx.y;
+  if (job >= nchunks) return;
+  const int c = (int)job;
+  const int64_t base = (int64_t)s * T + (int64_t)c * b;
+  double sum = 0.0;
+  for (int k = lane; k < b; k += 32) {
+    const float e = eta[base + k];
+    KW[base + k] = e;
+    KM[base + k] = e;
+    sum += (double)beta[base + k];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane == 0) {
+    const float bbar = (float)(sum / (double)b);
+    float* o = consts + ((int64_t)s * nchunks + c) * 4;
+    o[0] = 1.f;
+    o[1] = bbar;
+    o[2] = bbar;
+    o[3] = 0.f;
+  }
+}
+
+inline cudaError_t launch_scalar_scan(int rule, const float* eta, const float* beta, const float* gamma,
                                       int batch, int T, int b, float* KW, float* KM,
                                       float* consts, cudaStream_t st) {
   if (batch <= 0 || T <= 0) return cudaSuccess;
   int nchunks = T / b;
   const int warps = 4;
   dim3 grid((nchunks + warps - 1) / warps, batch);
-  scalar_scan_kernel<<<grid, warps * 32, 0, st>>>(eta, beta, gamma, T, b, nchunks, KW, KM, consts);
+  if (rule == TTT_RULE_LACT)
+    lact_scan_kernel<<<grid, warps * 32, 0, st>>>(eta, beta, T, b, nchunks, KW, KM, consts);
+  else
+    scalar_scan_kernel<<<grid, warps * 32, 0, st>>>(eta, beta, gamma, T, b, nchunks, KW, KM, consts);
   return cudaGetLastError();
 }
 

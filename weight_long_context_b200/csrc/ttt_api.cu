@@ -287,7 +287,8 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   // K1 for all chunks (depends only on the scalars).
   // Split-K arrival counters start at zero (every GEMM leaves them zero).
   if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
-  LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T, TRY(launch_scalar_scan(eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
+  LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T,
+         TRY(launch_scalar_scan(hd->cfg.update_rule, eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
   // Operand shadow of W_0.
   LAUNCH(K_SHADOW, 0, (4.0 + e) * B * L * p.m * h * d,
          (build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0)));
@@ -468,6 +469,8 @@ static ttt_status check_config(const ttt_config* c) {
   if (c->has_static != 0 && c->has_static != 1) return fail(TTT_ERR_INVALID_ARG, "has_static must be 0 or 1");
   if (c->loss_reduction != TTT_REDUCE_MEAN && c->loss_reduction != TTT_REDUCE_SUM)
     return fail(TTT_ERR_INVALID_ARG, "loss_reduction must be MEAN or SUM");
+  if (c->update_rule != TTT_RULE_E2TTT && c->update_rule != TTT_RULE_LACT)
+    return fail(TTT_ERR_INVALID_ARG, "update_rule must be E2TTT or LACT");
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return fail(TTT_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
   if (c->d < 16 || c->hidden < 16 || c->vocab < 16 || c->n_blocks < 1)
     return fail(TTT_ERR_SHAPE, "d, hidden, vocab must be >= 16 and n_blocks >= 1");
@@ -719,13 +722,16 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
   return TTT_OK;
 }
 
-ttt_status ttt_scalar_kernels(int32_t batch, int32_t T, int32_t b, const float* eta, const float* beta,
-                              const float* gamma, float* KW, float* KM, float* consts, void* stream) {
+ttt_status ttt_scalar_kernels(int32_t rule, int32_t batch, int32_t T, int32_t b, const float* eta,
+                              const float* beta, const float* gamma, float* KW, float* KM, float* consts,
+                              void* stream) {
+  if (rule != TTT_RULE_E2TTT && rule != TTT_RULE_LACT) return fail(TTT_ERR_INVALID_ARG, "unknown update rule");
   if (batch < 0 || T < 0) return fail(TTT_ERR_SHAPE, "batch and T must be >= 0");
   if (b < 1 || T % b) return fail(TTT_ERR_SHAPE, "b >= 1 and T % b == 0 required");
   if (batch == 0 || T == 0) return TTT_OK;
   if (!eta || !beta || !gamma || !KW || !KM || !consts) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  TTT_CUDA_TRY(launch_scalar_scan(eta, beta, gamma, batch, T, b, KW, KM, consts, static_cast<cudaStream_t>(stream)));
+  TTT_CUDA_TRY(launch_scalar_scan(rule, eta, beta, gamma, batch, T, b, KW, KM, consts,
+                                  static_cast<cudaStream_t>(stream)));
   return TTT_OK;
 }
 

@@ -53,6 +53,7 @@ class Workload:
     token_dist: str = "zipf"
     rms_eps: float = 1e-6
     reduction: str = "mean"  # chunk objective: mean (default) or sum of token losses
+    update_rule: str = "e2ttt"  # chunk update: "e2ttt" (Proposition 3.1) or "lact" (chunk-wise rule)
 
     @property
     def n_mats(self) -> int:

@@ -23,6 +23,7 @@ STATUS_NAMES = ["TTT_OK", "TTT_ERR_INVALID_ARG", "TTT_ERR_SHAPE", "TTT_ERR_UNSUP
 MLP = {"gelu": 0, "swiglu": 1}
 PRECISION = {"fp32": 0, "bf16": 1}
 REDUCTION = {"mean": 0, "sum": 1}
+RULE = {"e2ttt": 0, "lact": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
             "ttt_prefill_profiled",
@@ -42,7 +43,7 @@ class ttt_config(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("n_blocks", ctypes.c_int32), ("mlp", ctypes.c_int32), ("has_static", ctypes.c_int32),
                 ("precision", ctypes.c_int32), ("loss_reduction", ctypes.c_int32),
-                ("rms_eps", ctypes.c_float)]
+                ("rms_eps", ctypes.c_float), ("update_rule", ctypes.c_int32)]
 
 
 class ttt_kernel_stat(ctypes.Structure):
@@ -75,7 +76,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
     lib.ttt_prefill_profiled.restype = I32
-    lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, P, P, P, P, P, P, P]
+    lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, I32, P, P, P, P, P, P, P]
     lib.ttt_scalar_kernels.restype = I32
     I64 = ctypes.c_int64
     lib.ttt_gemm_bf16.argtypes = [I32, I32, I32, I32, P, I64, I64, I32, P, I64, I64, I32, P, I64, I64, P, SZ, P]
@@ -140,7 +141,8 @@ def ttt_workspace_size(h, batch: int, T: int, b: int) -> int:
     return n.value
 
 
-def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tensor, b: int, stream=None):
+def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tensor, b: int, stream=None,
+                       rule: str = "e2ttt"):
     """K1 alone: returns (KW [B,T], KM [B,T], consts [B,T/b,4]) as new CUDA tensors."""
     B, T = eta.shape
     for t, nm in ((eta, "eta"), (beta, "beta"), (gamma, "gamma")):
@@ -148,7 +150,7 @@ def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tenso
     KW = torch.empty_like(eta)
     KM = torch.empty_like(eta)
     consts = torch.empty((B, T // b if b > 0 else 0, 4), dtype=torch.float32, device=eta.device)
-    _check(load_library().ttt_scalar_kernels(B, T, b, _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(KW),
+    _check(load_library().ttt_scalar_kernels(RULE[rule], B, T, b, _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(KW),
                                              _ptr(KM), _ptr(consts), _stream_ptr(stream)),
            "ttt_scalar_kernels")
     return KW, KM, consts
@@ -198,14 +200,14 @@ class Handle:
     def __init__(self, d: int, hidden: int, vocab: int, n_blocks: int, mlp: str, has_static: bool,
                  precision: str, lm_head: torch.Tensor, rms_gain: torch.Tensor,
                  static_w: Optional[torch.Tensor] = None, rms_eps: float = 1e-6,
-                 reduction: str = "mean"):
+                 reduction: str = "mean", update_rule: str = "e2ttt"):
         dev = lm_head.device
         _dev(lm_head, torch.float32, "lm_head", dev)
         _dev(rms_gain, torch.float32, "rms_gain", dev)
         if static_w is not None:
             _dev(static_w, torch.float32, "static_w", dev)
         self.cfg = ttt_config(d, hidden, vocab, n_blocks, MLP[mlp], int(bool(has_static)),
-                              PRECISION[precision], REDUCTION[reduction], rms_eps)
+                              PRECISION[precision], REDUCTION[reduction], rms_eps, RULE[update_rule])
         self.device = dev
         self.n_mats = 2 if mlp == "gelu" else 3
         with torch.cuda.device(dev):
