@@ -296,6 +296,26 @@ def scalar_kernels(eta, beta, gamma):
     return KW, KM, float(gt[0]), float(bt[0]), cM
 
 
+def scalar_heads(X, heads, bias, eta_base, alpha_base, tau):
+    """Input-dependent update scalars ([E2-TTT] 依赖于输入的动态参数化):
+      eta_t   = eta_base * sigmoid(w_eta . x_t + b_eta),
+      beta_t  = sigmoid(w_beta . x_t + b_beta) ** (1 / tau),
+      alpha_t = alpha_base * sigmoid(w_alpha . x_t + b_alpha),
+      gamma_t = 1 - eta_t * alpha_t.
+    X [..., d]; heads [3, d] rows (w_eta, w_beta, w_alpha); bias [3].
+    Reading: each Linear has a bias.  Evaluated in float64."""
+    X = np.asarray(X, dtype=np.float64)
+    Wh = np.asarray(heads, dtype=np.float64)
+    bh = np.asarray(bias, dtype=np.float64)
+    z = X @ Wh.T + bh                     # [..., 3]
+    sig = 1.0 / (1.0 + np.exp(-z))
+    eta = eta_base * sig[..., 0]
+    beta = sig[..., 1] ** (1.0 / tau)
+    alpha = alpha_base * sig[..., 2]
+    gamma = 1.0 - eta * alpha
+    return eta, beta, gamma
+
+
 def scalar_kernels_ratio_form(eta, beta, gamma):
     """The same coefficients through R_t = sum_{i>=t} gtilde_i / btilde_i.
 

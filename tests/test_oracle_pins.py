@@ -300,6 +300,52 @@ def test_lact_ignores_decay():
 
 
 # ---------------------------------------------------------------------------
+# 4c. Input-dependent scalars ([E2-TTT] 依赖于输入的动态参数化)
+# ---------------------------------------------------------------------------
+
+def test_scalar_heads_at_zero_logits():
+    """Zero weights and biases: every gate is sigmoid(0) = 1/2 exactly, so
+    eta = eta_base / 2, beta = 2^(-1/tau), gamma = 1 - eta_base alpha_base / 4."""
+    X = np.random.default_rng(0).normal(size=(5, 7))
+    eta, beta, gamma = O.scalar_heads(X, np.zeros((3, 7)), np.zeros(3), 0.02, 0.5, 8.0)
+    np.testing.assert_allclose(eta, 0.01, rtol=1e-15)
+    np.testing.assert_allclose(beta, 2.0 ** (-1.0 / 8.0), rtol=1e-15)
+    np.testing.assert_allclose(gamma, 1.0 - 0.02 * 0.5 / 4.0, rtol=1e-15)
+
+
+def test_scalar_heads_saturation_and_heads_are_separate():
+    """A large positive logit on one head only saturates that head's gate:
+    eta -> eta_base while beta and alpha stay at sigmoid(0) = 1/2."""
+    X = np.ones((1, 4))
+    heads = np.zeros((3, 4))
+    heads[0] = 50.0                       # eta head only
+    eta, beta, gamma = O.scalar_heads(X, heads, np.zeros(3), 0.01, 1.0, 4.0)
+    assert eta[0] == pytest.approx(0.01, rel=1e-15)
+    assert beta[0] == pytest.approx(0.5 ** 0.25, rel=1e-15)
+    assert gamma[0] == pytest.approx(1.0 - 0.01 * 0.5, rel=1e-15)
+    heads = np.zeros((3, 4))
+    heads[1] = -50.0                      # beta head only: sigmoid -> 0
+    _, beta, _ = O.scalar_heads(X, heads, np.zeros(3), 0.01, 1.0, 4.0)
+    assert beta[0] < 1e-20
+
+
+def test_scalar_heads_linear_in_x_and_bias():
+    """The gate logits are affine in x: moving x along w_beta by s changes
+    sigmoid^-1(beta^tau) by s |w_beta|^2, and the bias enters additively."""
+    rng = np.random.default_rng(1)
+    d = 6
+    heads = rng.normal(size=(3, d))
+    bias = rng.normal(size=3)
+    x = rng.normal(size=(1, d))
+    logit = lambda b: np.log(b ** 4.0 / (1.0 - b ** 4.0))
+    _, b1, _ = O.scalar_heads(x, heads, bias, 0.01, 1.0, 4.0)
+    _, b2, _ = O.scalar_heads(x + 0.1 * heads[1], heads, bias, 0.01, 1.0, 4.0)
+    assert logit(b2[0]) - logit(b1[0]) == pytest.approx(0.1 * float(heads[1] @ heads[1]), rel=1e-9)
+    _, b3, _ = O.scalar_heads(x, heads, bias + np.array([0.0, 0.3, 0.0]), 0.01, 1.0, 4.0)
+    assert logit(b3[0]) - logit(b1[0]) == pytest.approx(0.3, rel=1e-9)
+
+
+# ---------------------------------------------------------------------------
 # 5. Cross-entropy closed forms
 # ---------------------------------------------------------------------------
 
@@ -452,6 +498,15 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "chunk_update_lact", lact_prod)
     _must_fail(test_lact_momentum_factor_is_the_chunk_average)
     monkeypatch.setattr(O, "chunk_update_lact", orig_lact)
+
+    # (h) scalar heads: tau instead of 1 / tau as the momentum exponent
+    orig_heads = O.scalar_heads
+
+    def heads_tau(X, heads, bias, eta_base, alpha_base, tau):
+        return orig_heads(X, heads, bias, eta_base, alpha_base, 1.0 / tau)
+    monkeypatch.setattr(O, "scalar_heads", heads_tau)
+    _must_fail(test_scalar_heads_at_zero_logits)
+    monkeypatch.setattr(O, "scalar_heads", orig_heads)
 
     # (f) the residual dropped from the backward of a block
     orig_mb = O.mlp_backward
