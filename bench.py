@@ -304,7 +304,15 @@ def run_ours(args, w: I.Workload):
     if input_bytes(w) + state_bytes(w) <= 2 * L2_BYTES:
         flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
 
+    heads = None
+    if args.scalar_heads:
+        rng = np.random.default_rng(100 + rank)
+        heads = (T(rng.normal(0.0, 1.0 / np.sqrt(w.d), (3, w.d))), (0.0, 0.0, 0.0), 0.01, 1.0, 16.0)
+
     def step():
+        if heads is not None:
+            e_, b_, g_ = ttt.ttt_scalar_heads(hidden, *heads, stream=st)
+            return h.prefill(hidden, tokens, W, M, e_, b_, g_, w.b, stream=st)
         return h.prefill(hidden, tokens, W, M, eta, beta, gamma, w.b, stream=st)
 
     for _ in range(args.warmup):
@@ -364,15 +372,32 @@ def run_ours(args, w: I.Workload):
                 "algorithmic_bytes_per_launch": dom["bytes"] / dom["launches"],
                 "peak_source": f"{pk['source']} (bf16 sustained; HBM copy)"}
 
+    # ---- the scalar heads alone (when used): HBM-bound, one read of the hidden rows
+    heads_line = None
+    if heads is not None:
+        reps = 10
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ttt.ttt_scalar_heads(hidden, *heads, stream=st)
+        a_.record(st)
+        for _ in range(reps):
+            ttt.ttt_scalar_heads(hidden, *heads, stream=st)
+        b_.record(st)
+        torch.cuda.synchronize()
+        hms = a_.elapsed_time(b_) / reps
+        hbytes = 4.0 * hidden.numel() + 3 * 4.0 * w.batch * w.T + 12.0 * w.d
+        heads_line = {"us_per_call": 1e3 * hms, "algorithmic_bytes": hbytes,
+                      "achieved_GBs": hbytes / (hms / 1e3) / 1e9, "frac_hbm": hbytes / (hms / 1e3) / 1e9 / pk["hbm"],
+                      "share_of_step": hms / mean_ms}
+
     # ---- end to end through the public API with host buffers
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
     hx = [pin(x["hidden"]), pin(x["tokens"].astype(np.int32)), pin(x["W0"]), pin(x["M0"]), pin(x["eta"]),
           pin(x["beta"]), pin(x["gamma"])]
-    h2d = sum(t.numel() * t.element_size() for t in hx)
+    h2d = sum(t.numel() * t.element_size() for t in (hx[:4] if heads is not None else hx))
     d2h = 2 * hx[2].numel() * 4 + w.batch * w.n_chunks * 4
     del hidden, tokens, W, M, eta, beta, gamma
     torch.cuda.empty_cache()
-    h.prefill_host(*hx, b=w.b, stream=st)    # warm the host path once
+    h.prefill_host(*hx, b=w.b, stream=st, scalar_heads=heads)    # warm the host path once
     e_steps = max(1, min(args.steps, 3))
     if world > 1:
         dist.barrier()
@@ -380,7 +405,7 @@ def run_ours(args, w: I.Workload):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
     for _ in range(e_steps):
-        h.prefill_host(*hx, b=w.b, stream=st)
+        h.prefill_host(*hx, b=w.b, stream=st, scalar_heads=heads)
     e1.record(st)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1) / e_steps, dev)
@@ -401,6 +426,9 @@ def run_ours(args, w: I.Workload):
                                      "sustained": tflops / world / pk["tflops_sustained"], "source": pk["source"]},
                 "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
                 "roofline": roofline, "device_status": status}
+        if heads_line is not None:
+            line["config"]["scalars"] = "input-dependent heads (eta_base 0.01, alpha_base 1, tau 16)"
+            line["scalar_heads"] = heads_line
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
@@ -420,6 +448,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scalar-heads", action="store_true",
+                    help="input-dependent scalars: eta, beta, gamma computed from the hidden rows on the device "
+                         "inside every step (eta_base 0.01, alpha_base 1, tau 16, heads N(0, 1/d))")
     ap.add_argument("--update-rule", default="e2ttt", choices=["e2ttt", "lact"],
                     help="chunk update rule: Proposition 3.1 (default) or LaCT's chunk-wise rule")
     ap.add_argument("--chunks", type=int, default=0,

@@ -205,6 +205,22 @@ ttt_status ttt_scalar_kernels(int32_t rule, int32_t batch, int32_t T, int32_t b,
                               const float* beta, const float* gamma, float* KW, float* KM,
                               float* consts, void* stream);
 
+/* Input-dependent update scalars for every token ([E2-TTT] 依赖于输入的动态参数化):
+ *   eta_t   = eta_base * sigmoid(w_eta . x_t + b_eta)
+ *   beta_t  = sigmoid(w_beta . x_t + b_beta) ^ (1 / tau)
+ *   alpha_t = alpha_base * sigmoid(w_alpha . x_t + b_alpha),  gamma_t = 1 - eta_t alpha_t
+ *   hidden [batch, T, d]   device float32, x_t (the rows entering the updated
+ *                          blocks, as passed to ttt_prefill); 16-byte aligned
+ *   heads  [3, d]          device float32 rows w_eta, w_beta, w_alpha; 16-byte aligned
+ *   eta, beta, gamma [batch, T]  device float32 out, ready for ttt_prefill
+ * The Linear maps carry the biases b_eta, b_beta, b_alpha.  d % 4 == 0 and
+ * tau > 0 (finite) are required (TTT_ERR_SHAPE / TTT_ERR_INVALID_ARG
+ * otherwise).  Float32 dot products in a fixed order (deterministic).  No
+ * handle needed; asynchronous on `stream`. */
+ttt_status ttt_scalar_heads(int32_t batch, int32_t T, int32_t d, const float* hidden, const float* heads,
+                            float b_eta, float b_beta, float b_alpha, float eta_base, float alpha_base,
+                            float tau, float* eta, float* beta, float* gamma, void* stream);
+
 /* The tensor-core GEMM the inner loop is built on, exposed for testing and
  * reuse: D[z] = A[z] B[z]^T for z < batch, i.e.
  *   D[z](m, n) = sum_{k < K} A[z](m, k) * B[z](n, k)

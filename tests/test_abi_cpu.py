@@ -73,6 +73,15 @@ def test_create_rejects_unknown_update_rule(lib):
     assert b"update_rule" in lib.ttt_last_error()
 
 
+def test_scalar_heads_validation(lib):
+    z = ctypes.c_void_p(16)
+    args = lambda d, tau: (1, 4, d, z, z, 0.0, 0.0, 0.0, 0.01, 1.0, tau, z, z, z, None)
+    assert lib.ttt_scalar_heads(*args(6, 16.0)) == 2          # d % 4
+    assert lib.ttt_scalar_heads(*args(8, 0.0)) == 1           # tau <= 0
+    assert lib.ttt_scalar_heads(*args(8, float("inf"))) == 1
+    assert lib.ttt_scalar_heads(0, 0, 8, z, z, 0.0, 0.0, 0.0, 0.01, 1.0, 16.0, z, z, z, None) == 0
+
+
 def test_prefill_rejects_null_handle(lib):
     n = ctypes.c_size_t()
     assert lib.ttt_workspace_size(None, 1, 8, 4, ctypes.byref(n)) == 1

@@ -159,6 +159,49 @@ __global__ void ce_rows_kernel(const float* __restrict__ part, const float* __re
   }
 }
 
+// Input-dependent update scalars ("Rethinking Expressivity and Efficiency in
+// Test-Time Training", 依赖于输入的动态参数化), one warp per token row x_t:
+//   eta_t   = eta_base sigmoid(w_eta . x_t + b_eta)
+//   beta_t  = sigmoid(w_beta . x_t + b_beta)^(1/tau)
+//   gamma_t = 1 - eta_t alpha_base sigmoid(w_alpha . x_t + b_alpha)
+// heads [3, d] = (w_eta, w_beta, w_alpha).  The three dot products are summed
+// in float32 in a fixed order (lane-strided float4, then a shuffle tree), so
+// the result does not depend on scheduling.  d % 4 == 0.
+__global__ void scalar_heads_kernel(const float* __restrict__ x, int64_t rows, int d, const float* __restrict__ heads,
+                                    float b_eta, float b_beta, float b_alpha, float eta_base, float alpha_base,
+                                    float inv_tau, float* __restrict__ eta, float* __restrict__ beta,
+                                    float* __restrict__ gamma) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + r * d);
+  const float4* h0 = reinterpret_cast<const float4*>(heads);
+  const float4* h1 = reinterpret_cast<const float4*>(heads + d);
+  const float4* h2 = reinterpret_cast<const float4*>(heads + 2 * (int64_t)d);
+  float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 v = xr[i], a = h0[i], b = h1[i], c = h2[i];
+    z0 += v.x * a.x + v.y * a.y + v.z * a.z + v.w * a.w;
+    z1 += v.x * b.x + v.y * b.y + v.z * b.z + v.w * b.w;
+    z2 += v.x * c.x + v.y * c.y + v.z * c.z + v.w * c.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    z0 += __shfl_xor_sync(0xffffffffu, z0, o);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, o);
+    z2 += __shfl_xor_sync(0xffffffffu, z2, o);
+  }
+  if (lane == 0) {
+    const float se = 1.f / (1.f + expf(-(z0 + b_eta)));
+    const float sb = 1.f / (1.f + expf(-(z1 + b_beta)));
+    const float sa = 1.f / (1.f + expf(-(z2 + b_alpha)));
+    const float e = eta_base * se;
+    eta[r] = e;
+    beta[r] = powf(sb, inv_tau);
+    gamma[r] = 1.f - e * (alpha_base * sa);
+  }
+}
+
 // Cross-entropy pass B from the logits kept by pass A (fp32):
 // P[r, j] = exp(logit[r, v0 + j] - lse[r]) - [v0 + j == y_r] for j < vs, the
 // operand slab of dz = P E_slab (row pitch Vs).  The same arithmetic as

@@ -735,6 +735,22 @@ ttt_status ttt_scalar_kernels(int32_t rule, int32_t batch, int32_t T, int32_t b,
   return TTT_OK;
 }
 
+ttt_status ttt_scalar_heads(int32_t batch, int32_t T, int32_t d, const float* hidden, const float* heads,
+                            float b_eta, float b_beta, float b_alpha, float eta_base, float alpha_base,
+                            float tau, float* eta, float* beta, float* gamma, void* stream) {
+  if (batch < 0 || T < 0 || d < 4 || d % 4) return fail(TTT_ERR_SHAPE, "batch, T >= 0 and d >= 4, d % 4 == 0 required");
+  if (!(tau > 0.f) || !std::isfinite(tau)) return fail(TTT_ERR_INVALID_ARG, "tau must be positive and finite");
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !heads || !eta || !beta || !gamma) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(heads)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "hidden and heads must be 16-byte aligned");
+  const int64_t rows = (int64_t)batch * T;
+  scalar_heads_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      hidden, rows, d, heads, b_eta, b_beta, b_alpha, eta_base, alpha_base, 1.f / tau, eta, beta, gamma);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
 ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
                                const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
                                const float* gamma, float* chunk_loss, void* stream) {

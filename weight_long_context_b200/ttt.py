@@ -27,7 +27,7 @@ RULE = {"e2ttt": 0, "lact": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
             "ttt_prefill_profiled",
-            "ttt_scalar_kernels", "ttt_gemm_bf16",
+            "ttt_scalar_kernels", "ttt_scalar_heads", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
 
@@ -77,6 +77,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
     lib.ttt_prefill_profiled.restype = I32
     lib.ttt_scalar_kernels.argtypes = [I32, I32, I32, I32, P, P, P, P, P, P, P]
+    F = ctypes.c_float
+    lib.ttt_scalar_heads.argtypes = [I32, I32, I32, P, P, F, F, F, F, F, F, P, P, P, P]
+    lib.ttt_scalar_heads.restype = I32
     lib.ttt_scalar_kernels.restype = I32
     I64 = ctypes.c_int64
     lib.ttt_gemm_bf16.argtypes = [I32, I32, I32, I32, P, I64, I64, I32, P, I64, I64, I32, P, I64, I64, P, SZ, P]
@@ -154,6 +157,24 @@ def ttt_scalar_kernels(eta: torch.Tensor, beta: torch.Tensor, gamma: torch.Tenso
                                              _ptr(KM), _ptr(consts), _stream_ptr(stream)),
            "ttt_scalar_kernels")
     return KW, KM, consts
+
+
+def ttt_scalar_heads(hidden: torch.Tensor, heads: torch.Tensor, bias, eta_base: float, alpha_base: float,
+                     tau: float, stream=None):
+    """Input-dependent (eta, beta, gamma) [B, T] from hidden [B, T, d] and the
+    heads [3, d] (w_eta, w_beta, w_alpha) with biases bias[0..2], as new CUDA tensors."""
+    B, T, d = hidden.shape
+    _dev(hidden, torch.float32, "hidden", hidden.device)
+    _dev(heads, torch.float32, "heads", hidden.device)
+    if tuple(heads.shape) != (3, d):
+        raise ValueError("heads must be [3, d]")
+    eta = torch.empty((B, T), dtype=torch.float32, device=hidden.device)
+    beta = torch.empty_like(eta)
+    gamma = torch.empty_like(eta)
+    _check(load_library().ttt_scalar_heads(B, T, d, _ptr(hidden), _ptr(heads), float(bias[0]), float(bias[1]),
+                                           float(bias[2]), eta_base, alpha_base, tau, _ptr(eta), _ptr(beta),
+                                           _ptr(gamma), _stream_ptr(stream)), "ttt_scalar_heads")
+    return eta, beta, gamma
 
 
 def ttt_gemm_bf16(A: torch.Tensor, B: torch.Tensor, a_kmajor: bool = True, b_kmajor: bool = True,
@@ -265,14 +286,20 @@ class Handle:
                     flops=stats[i].flops, bytes=stats[i].bytes) for i in range(n.value)]
         return loss, out
 
-    def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None):
+    def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None, scalar_heads=None):
         """End-to-end call on HOST tensors: copies the inputs to the device,
         runs the inner loop, copies W, M and the chunk losses back.  Returns
-        (W, M, chunk_loss) as host tensors."""
+        (W, M, chunk_loss) as host tensors.  scalar_heads = (heads [3, d] CUDA
+        tensor, bias[3], eta_base, alpha_base, tau): the scalars come from
+        ttt_scalar_heads on the device (eta, beta, gamma are then ignored)."""
         dev = self.device
         st = stream if stream is not None else torch.cuda.current_stream(dev)
         with torch.cuda.stream(st):
-            d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0, eta, beta, gamma)]
+            if scalar_heads is None:
+                d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0, eta, beta, gamma)]
+            else:
+                d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0)]
+                d_in += list(ttt_scalar_heads(d_in[0], *scalar_heads, stream=st))
             loss = self.prefill(*d_in, b=b, stream=st)
             outs = []
             for t in (d_in[2], d_in[3], loss):
