@@ -180,11 +180,16 @@ def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> flo
     return units_per_rank * world / max_seconds if max_seconds > 0 else 0.0
 
 
+# The sources that define the profiled GEMM kernels (engine, epilogues and the
+# helpers they include): a committed ncu summary is used only while these match.
+KERNEL_SOURCES = ("common.cuh", "gemm_types.cuh", "gemm_tc.cuh", "epilogue.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for dp, _, fs in sorted(os.walk(os.path.join(ROOT, "weight_long_context_b200", "csrc"))):
-        for f in sorted(fs):
-            h.update(open(os.path.join(dp, f), "rb").read())
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "weight_long_context_b200", "csrc", f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "ttt.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
