@@ -189,7 +189,6 @@ def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, "weight_long_context_b200", "csrc", f), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "ttt.h"), "rb").read())
     return h.hexdigest()[:16]
 
 
