@@ -7,5 +7,6 @@ product path never imports it, and it imports nothing from the product.
 from .ttt_oracle import *  # noqa: F401,F403
 from .ttt_oracle import (Model, make_model, prefill, prefill_sequence, scalar_kernels,  # noqa: F401
                          scalar_kernels_ratio_form, chunk_update_closed, chunk_update_explicit,
-                         chunk_update_lact, scalar_heads,
+                         chunk_update_lact, scalar_heads, recon_forward, recon_chunk, prefill_recon,
+                         layer_norm, layer_norm_backward, recon_shapes,
                          token_losses, token_gradients, unpack_blocks, pack_blocks)

@@ -480,6 +480,86 @@ def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
     return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls)
 
 
+# ---------------------------------------------------------------------------
+# E2-TTT's own layer: key/value reconstruction, query outputs
+# ([E2-TTT] 背景知识 (TTT建模范式, 表达能力强的逐Token更新机制), 快速权重网络实例化, Algorithm 1)
+# ---------------------------------------------------------------------------
+
+def recon_shapes(kind: str, d: int, h: int):
+    """Fast-weight matrices of the layer's MLP, [rows, cols] each."""
+    return [(h, d), (d, h)] if kind == GELU else [(h, d), (h, d), (d, h)]
+
+
+def layer_norm(y, eps):
+    """Parameter-free LayerNorm over the last axis; returns (LN(y), 1/std)."""
+    mu = y.mean(axis=-1, keepdims=True)
+    var = ((y - mu) ** 2).mean(axis=-1, keepdims=True)
+    rs = 1.0 / np.sqrt(var + eps)
+    return (y - mu) * rs, rs
+
+
+def layer_norm_backward(g, ln, rs):
+    """dL/dy from dL/dLN(y) for the parameter-free LayerNorm."""
+    return rs * (g - g.mean(axis=-1, keepdims=True) - ln * (g * ln).mean(axis=-1, keepdims=True))
+
+
+def recon_forward(kind: str, mats, X, eps):
+    """f_W(x) = x + LN(MLP_W(x)) ([E2-TTT] 快速权重网络实例化); rows of X."""
+    y, cache = mlp_forward(kind, mats, X)
+    ln, rs = layer_norm(y, eps)
+    return X + ln, (cache, ln, rs)
+
+
+def recon_chunk(kind: str, mats, K, V, eps):
+    """Per-token reconstruction losses L_t = mean_j (f_W(k_t) - v_t)_j^2 (the
+    mean squared error) at the chunk-start weights, and the factor pairs of
+    their gradients (one backward for the chunk)."""
+    f, (cache, ln, rs) = recon_forward(kind, mats, K, eps)
+    r = f - V
+    loss = (r * r).mean(axis=1)
+    gf = 2.0 * r / r.shape[1]
+    gy = layer_norm_backward(gf, ln, rs)
+    _, pairs = mlp_backward(kind, mats, cache, gy)
+    return loss, pairs
+
+
+def prefill_recon(kind: str, d: int, h: int, W0_flat, M0_flat, K, V, Q, eta, beta, gamma, b, eps,
+                  dtype=np.float64, update: str = "closed", reduction: str = "mean",
+                  n_chunks: Optional[int] = None):
+    """The layer over batched sequences (Algorithm 1 chunk after chunk): for each
+    chunk, outputs o_t = f_{W_0}(q_t) and losses at the chunk-start weights, one
+    backward, then the chunk update (Proposition 3.1, or LaCT's rule).
+    K, V, Q [B, T, d]; W0_flat / M0_flat [B * m * h * d].  Returns
+    (W_flat, M_flat, chunk_loss [B, n_chunks], O [B, T, d])."""
+    if update not in UPDATE_RULES:
+        raise ValueError("update must be one of " + ", ".join(UPDATE_RULES))
+    step = {"closed": chunk_update_closed, "explicit": chunk_update_explicit, "lact": chunk_update_lact}[update]
+    gscale = 1.0 / b if reduction == "mean" else 1.0
+    shapes = recon_shapes(kind, d, h)
+    per_seq = sum(r * c for r, c in shapes)
+    Bn, T, _ = np.shape(K)
+    nc = T // b if n_chunks is None else n_chunks
+    W0_flat = np.asarray(W0_flat, dtype=dtype).reshape(Bn, per_seq)
+    M0_flat = np.asarray(M0_flat, dtype=dtype).reshape(Bn, per_seq)
+    Ws, Ms, Ls = [], [], []
+    O = np.zeros((Bn, nc * b, d), dtype=dtype)
+    for s in range(Bn):
+        W = unpack_blocks(W0_flat[s].copy(), 1, shapes)
+        M = unpack_blocks(M0_flat[s].copy(), 1, shapes)
+        losses = np.zeros(nc)
+        for c in range(nc):
+            sl = slice(c * b, (c + 1) * b)
+            Kc, Vc, Qc = (np.asarray(a[s][sl], dtype=dtype) for a in (K, V, Q))
+            O[s, sl] = recon_forward(kind, W[0], Qc, eps)[0]
+            loss, pairs = recon_chunk(kind, W[0], Kc, Vc, eps)
+            losses[c] = float(np.mean(loss))
+            W, M = step(W, M, [pairs], eta[s][sl], beta[s][sl], gamma[s][sl], gscale)
+        Ws.append(pack_blocks(W))
+        Ms.append(pack_blocks(M))
+        Ls.append(losses)
+    return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls), O
+
+
 def token_losses(model: Model, W_flat, X, y, dtype=np.float64):
     """Per-token losses of rows X at fast weights W_flat (one sequence)."""
     mdl = model.astype(dtype)

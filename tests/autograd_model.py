@@ -59,3 +59,18 @@ def per_token_grads(kind, d, h, n_blocks, eps, E, g, static_flat, W_flat, X, y):
         (gt,) = torch.autograd.grad(L[t], W, retain_graph=True)
         rows.append(gt.clone())
     return torch.stack(rows), L.detach()
+
+
+def recon_losses(kind, d, h, eps, W_flat, K, V):
+    """Per-token reconstruction losses of E2-TTT's layer ("Rethinking
+    Expressivity and Efficiency in Test-Time Training", 快速权重网络实例化 and
+    the TTT modelling background): f(k) = k + LayerNorm(MLP(k)) without affine
+    parameters, loss = mean squared error against v (torch tensors, float64)."""
+    (mats,) = split_blocks(W_flat, 1, shapes_of(kind, d, h))
+    f = K + F.layer_norm(_mlp(kind, mats, K), (d,), eps=eps)
+    return F.mse_loss(f, V, reduction="none").mean(dim=1)
+
+
+def recon_outputs(kind, d, h, eps, W_flat, Q):
+    (mats,) = split_blocks(W_flat, 1, shapes_of(kind, d, h))
+    return Q + F.layer_norm(_mlp(kind, mats, Q), (d,), eps=eps)

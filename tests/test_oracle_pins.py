@@ -346,6 +346,87 @@ def test_scalar_heads_linear_in_x_and_bias():
 
 
 # ---------------------------------------------------------------------------
+# 4d. E2-TTT's own layer: reconstruction loss, query outputs, inner LayerNorm
+# ---------------------------------------------------------------------------
+
+def recon_setup(kind="gelu", d=6, h=9, T=8, seed=7, m0=0.05):
+    rng = np.random.default_rng(seed)
+    n = sum(r * c for r, c in AM.shapes_of(kind, d, h))
+    return dict(kind=kind, d=d, h=h, W0=rng.normal(0, 0.4, n), M0=rng.normal(0, m0, n),
+                K=rng.normal(size=(T, d)), V=rng.normal(size=(T, d)), Q=rng.normal(size=(T, d)),
+                eta=0.05 / (1 + np.exp(-rng.normal(size=T))), beta=rng.uniform(0.8, 0.99, T),
+                gamma=rng.uniform(0.99, 1.0, T))
+
+
+def _recon_pairs_as_grads(kind, d, h, W, K, V, eps):
+    """Per-token gradients [T, n] from the oracle's factor pairs."""
+    mats = AM.split_blocks(W, 1, AM.shapes_of(kind, d, h))[0]
+    loss, pairs = O.recon_chunk(kind, mats, K, V, eps)
+    cols = [np.einsum("ti,tj->tij", Lf, Rf).reshape(len(K), -1) for Lf, Rf in pairs]
+    return loss, np.concatenate(cols, axis=1)
+
+
+@pytest.mark.parametrize("kind", ["gelu", "swiglu"])
+def test_recon_losses_and_gradients_match_autograd(kind):
+    s = recon_setup(kind)
+    d, h, eps = s["d"], s["h"], 1e-6
+    loss, G = _recon_pairs_as_grads(kind, d, h, s["W0"], s["K"], s["V"], eps)
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    Wv = T_(s["W0"]).requires_grad_(True)
+    L = AM.recon_losses(kind, d, h, eps, Wv, T_(s["K"]), T_(s["V"]))
+    np.testing.assert_allclose(loss, L.detach().numpy(), rtol=1e-12)
+    for t in range(len(s["K"])):
+        (g,) = torch.autograd.grad(L[t], Wv, retain_graph=True)
+        assert rel(G[t], g.numpy()) < 1e-10
+    Ot = AM.recon_outputs(kind, d, h, eps, T_(s["W0"]), T_(s["Q"])).numpy()
+    mats = AM.split_blocks(s["W0"], 1, AM.shapes_of(kind, d, h))[0]
+    assert rel(O.recon_forward(kind, mats, s["Q"], eps)[0], Ot) < 1e-13
+
+
+def test_recon_gradients_match_finite_differences():
+    s = recon_setup("swiglu", d=5, h=7, T=3, seed=8)
+    d, h, eps = s["d"], s["h"], 1e-6
+    _, G = _recon_pairs_as_grads("swiglu", d, h, s["W0"], s["K"], s["V"], eps)
+    mats_of = lambda W: AM.split_blocks(W, 1, AM.shapes_of("swiglu", d, h))[0]
+    rng = np.random.default_rng(0)
+    for idx in rng.choice(len(s["W0"]), 12, replace=False):
+        e = np.zeros_like(s["W0"])
+        e[idx] = 1e-6
+        lp, _ = O.recon_chunk("swiglu", mats_of(s["W0"] + e), s["K"], s["V"], eps)
+        lm, _ = O.recon_chunk("swiglu", mats_of(s["W0"] - e), s["K"], s["V"], eps)
+        np.testing.assert_allclose(G[:, idx], (lp - lm) / 2e-6, rtol=1e-5, atol=1e-8)
+
+
+def test_recon_zero_output_matrix():
+    """A zero output matrix makes the MLP branch zero and LayerNorm(0) = 0, so
+    the layer is the identity: o_t = q_t and L_t = mean_j (k_t - v_t)_j^2 exactly."""
+    s = recon_setup("gelu", d=6, h=9)
+    W = s["W0"].copy()
+    W[9 * 6:] = 0.0                              # W2 [d, h]
+    Wf, Mf, Ls, Oo = O.prefill_recon("gelu", 6, 9, W, s["M0"], s["K"][None], s["V"][None], s["Q"][None],
+                                     s["eta"][None], s["beta"][None], s["gamma"][None], 8, 1e-6)
+    np.testing.assert_array_equal(Oo[0], s["Q"])
+    assert Ls[0, 0] == pytest.approx(float(((s["K"] - s["V"]) ** 2).mean()), rel=1e-14)
+
+
+@pytest.mark.parametrize("rule", ["closed", "lact"])
+def test_recon_prefill_closed_form_equals_recursion(rule):
+    """Over several chunks the Proposition 3.1 chunk end equals the per-token
+    recursion (and LaCT's rule runs through the same driver)."""
+    s = recon_setup("swiglu", T=12)
+    args = ("swiglu", s["d"], s["h"], s["W0"], s["M0"], s["K"][None], s["V"][None], s["Q"][None],
+            s["eta"][None], s["beta"][None], s["gamma"][None], 4, 1e-6)
+    Wc, Mc, Lc, Oc = O.prefill_recon(*args, update=rule)
+    if rule == "closed":
+        We, Me, Le, Oe = O.prefill_recon(*args, update="explicit")
+        assert rel(Wc, We) < 1e-12 and rel(Mc, Me) < 1e-12
+        np.testing.assert_allclose(Lc, Le, rtol=1e-12)
+        np.testing.assert_allclose(Oc, Oe, rtol=1e-12)
+    else:
+        assert np.all(np.isfinite(Wc)) and Lc.shape == (1, 3)
+
+
+# ---------------------------------------------------------------------------
 # 5. Cross-entropy closed forms
 # ---------------------------------------------------------------------------
 
@@ -507,6 +588,12 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "scalar_heads", heads_tau)
     _must_fail(test_scalar_heads_at_zero_logits)
     monkeypatch.setattr(O, "scalar_heads", orig_heads)
+
+    # (i) LayerNorm backward without its projection term
+    orig_lnb = O.layer_norm_backward
+    monkeypatch.setattr(O, "layer_norm_backward", lambda g, ln, rs: rs * (g - g.mean(axis=-1, keepdims=True)))
+    _must_fail(test_recon_gradients_match_finite_differences)
+    monkeypatch.setattr(O, "layer_norm_backward", orig_lnb)
 
     # (f) the residual dropped from the backward of a block
     orig_mb = O.mlp_backward
