@@ -71,6 +71,7 @@ enum { TTT_MLP_GELU = 0, TTT_MLP_SWIGLU = 1 };
 enum { TTT_PREC_FP32 = 0, TTT_PREC_BF16 = 1 };
 enum { TTT_REDUCE_MEAN = 0, TTT_REDUCE_SUM = 1 };
 enum { TTT_RULE_E2TTT = 0, TTT_RULE_LACT = 1 };
+enum { TTT_HEAD_LM = 0, TTT_HEAD_RECON = 1 };
 
 /* Model shape.  d, hidden, vocab: multiples of 16, at least 16, and
  * d <= 16384, hidden <= 65536, vocab < 2^26.  n_blocks in [1, 64].
@@ -91,7 +92,14 @@ enum { TTT_RULE_E2TTT = 0, TTT_RULE_LACT = 1 };
  * chunk end of M_t = beta_t M_{t-1} + eta_t G_t, W_t = gamma_t W_{t-1} + M_t.
  * TTT_RULE_LACT: LaCT's chunk-wise rule as [E2-TTT] states it (高效的逐块
  * 更新机制): G = sum_t eta_t G_t, M_C = (mean_t beta_t) M_0 + G,
- * W_C = W_0 + M_C (gamma unused). */
+ * W_C = W_0 + M_C (gamma unused).
+ * head: the self-supervised loss that drives the update.  TTT_HEAD_LM: the
+ * frozen RMSNorm + LM head next-token cross-entropy of ttt_prefill.
+ * TTT_HEAD_RECON: [E2-TTT]'s own layer, run by ttt_prefill_recon: key/value
+ * reconstruction through f_W(x) = x + LN(MLP_W(x)) (快速权重网络实例化; LN
+ * without affine parameters, epsilon = rms_eps), loss the mean squared error,
+ * outputs f_{W_0}(q_t); requires n_blocks == 1 and has_static == 0, and
+ * ignores vocab (lm_head and rms_gain may be NULL at creation). */
 typedef struct ttt_config {
   int32_t d;
   int32_t hidden;
@@ -103,6 +111,7 @@ typedef struct ttt_config {
   int32_t loss_reduction; /* TTT_REDUCE_MEAN or TTT_REDUCE_SUM */
   float rms_eps;
   int32_t update_rule; /* TTT_RULE_E2TTT or TTT_RULE_LACT */
+  int32_t head;        /* TTT_HEAD_LM or TTT_HEAD_RECON */
 } ttt_config;
 
 typedef struct ttt_handle ttt_handle;
@@ -185,6 +194,25 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
                                 const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
                                 const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
                                 void* stream, ttt_kernel_stat* stats, int32_t max_stats, int32_t* n_stats);
+
+/* [E2-TTT]'s own layer over `batch` independent sequences of T tokens, chunk
+ * size b, for a handle created with head = TTT_HEAD_RECON (背景知识: TTT建模范式;
+ * 快速权重网络实例化; Algorithm 1).  For every chunk, at the chunk-start weights
+ * W_0: outputs o_t = f_{W_0}(q_t) and losses L_t = mean_j (f_{W_0}(k_t) - v_t)_j^2
+ * with f_W(x) = x + LN(MLP_W(x)); then the chunk update of the handle's rule
+ * from the per-token gradients of one backward (loss reduction as for ttt_prefill).
+ *   K, V, Q    [batch, T, d]  device float32: keys, values, queries
+ *   W, M       [batch * m * hidden * d]  in: W_0, M_0; out: final state (as ttt_prefill)
+ *   eta, beta, gamma [batch, T]  per-token scalars
+ *   O          [batch, T, d]  out: the outputs o_t
+ *   chunk_loss [batch, T/b]   out: mean of the chunk's L_t
+ *   workspace  at least ttt_workspace_size() bytes, 256-byte aligned
+ * K, V, Q, O, W, M 16-byte aligned; T % b == 0.  A handle with the LM head is
+ * TTT_ERR_UNSUPPORTED here (and a reconstruction handle in ttt_prefill). */
+ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* K, const float* V,
+                             const float* Q, float* W, float* M, const float* eta, const float* beta,
+                             const float* gamma, float* O, float* chunk_loss, void* workspace, size_t ws_bytes,
+                             void* stream);
 
 /* The per-token and per-chunk coefficients of a chunk update rule for every
  * chunk, on the device.  rule = TTT_RULE_E2TTT: the scalar kernels of

@@ -82,6 +82,14 @@ def test_scalar_heads_validation(lib):
     assert lib.ttt_scalar_heads(0, 0, 8, z, z, 0.0, 0.0, 0.0, 0.01, 1.0, 16.0, z, z, z, None) == 0
 
 
+def test_recon_head_config_validation(lib):
+    C = ttt.ttt_config
+    assert _create(lib, C(32, 32, 32, 1, 0, 0, 0, 0, 1e-6, 0, 2)) == 1        # unknown head
+    assert _create(lib, C(32, 32, 0, 2, 0, 0, 0, 0, 1e-6, 0, 1)) == 3         # recon: one block only
+    assert _create(lib, C(32, 32, 0, 1, 0, 1, 0, 0, 1e-6, 0, 1)) == 3         # recon: no static MLP
+    assert lib.ttt_prefill_recon(None, 1, 8, 4, *([None] * 10), None, 0, None) == 1   # NULL handle
+
+
 def test_prefill_rejects_null_handle(lib):
     n = ctypes.c_size_t()
     assert lib.ttt_workspace_size(None, 1, 8, 4, ctypes.byref(n)) == 1

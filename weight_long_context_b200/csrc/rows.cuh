@@ -159,6 +159,97 @@ __global__ void ce_rows_kernel(const float* __restrict__ part, const float* __re
   }
 }
 
+// E2-TTT's own layer ("Rethinking Expressivity and Efficiency in Test-Time
+// Training": TTT modelling background, 快速权重网络实例化, Algorithm 1), one warp
+// per chunk row r (token ti):
+//   keys:    f = k + LN(y_k), L_t = mean_j (f - v)_j^2, g_f = 2 (f - v) / d,
+//            g_y = rs (g_f - mean(g_f) - LN(y_k) mean(g_f LN(y_k)))
+//            -> dout_a = g_y (operand of dA = g_y W_down) and the K_W / K_M
+//            scaled, negated copies (operands of the output matrix's update);
+//   queries: o = q + LN(y_q), written to the caller's O at token ti.
+// LN is the parameter-free LayerNorm (epsilon eps); statistics in two passes
+// over the row (mean, then centred sum of squares), float32.
+template <typename T>
+__global__ void recon_rows_kernel(const float* __restrict__ yk, const float* __restrict__ kres,
+                                  const float* __restrict__ Vt, const float* __restrict__ yq,
+                                  const float* __restrict__ qres, TokenMap tm, int64_t n, int d, float eps,
+                                  const float* __restrict__ KW, const float* __restrict__ KM, float kscale,
+                                  float* __restrict__ ltok, T* __restrict__ dout_a, T* __restrict__ doutW,
+                                  T* __restrict__ doutM, float* __restrict__ O) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= n) return;
+  const int64_t ti = tm.index((int)r);
+  const int q4 = d >> 2;
+  const float invd = 1.f / (float)d;
+  auto wsum = [](float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+  };
+  // LayerNorm statistics of one row
+  auto stats = [&](const float4* y, float& mu, float& rs) {
+    float s1 = 0.f;
+    for (int c = lane; c < q4; c += 32) { const float4 a = y[c]; s1 += (a.x + a.y) + (a.z + a.w); }
+    mu = wsum(s1) * invd;
+    float s2 = 0.f;
+    for (int c = lane; c < q4; c += 32) {
+      const float4 a = y[c];
+      const float e0 = a.x - mu, e1 = a.y - mu, e2 = a.z - mu, e3 = a.w - mu;
+      s2 += (e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3);
+    }
+    rs = rsqrtf(wsum(s2) * invd + eps);
+  };
+  // ---- keys: loss and the gradient at the MLP output
+  const float4* yr = reinterpret_cast<const float4*>(yk + r * d);
+  const float4* kr = reinterpret_cast<const float4*>(kres + r * d);
+  const float4* vr = reinterpret_cast<const float4*>(Vt + ti * d);
+  float mu, rs;
+  stats(yr, mu, rs);
+  float sl = 0.f, sg = 0.f, sgl = 0.f;
+  for (int c = lane; c < q4; c += 32) {
+    const float4 y = yr[c], k = kr[c], v = vr[c];
+    const float yy[4] = {y.x, y.y, y.z, y.w}, kk[4] = {k.x, k.y, k.z, k.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float ln = (yy[j] - mu) * rs;
+      const float e = kk[j] + ln - vv[j];
+      const float g = 2.f * e * invd;
+      sl += e * e;
+      sg += g;
+      sgl += g * ln;
+    }
+  }
+  sl = wsum(sl);
+  const float mg = wsum(sg) * invd, mgl = wsum(sgl) * invd;
+  if (lane == 0) ltok[r] = sl * invd;
+  const float kw = -KW[ti] * kscale, km = -KM[ti] * kscale;
+  for (int c = lane; c < q4; c += 32) {
+    const float4 y = yr[c], k = kr[c], v = vr[c];
+    const float yy[4] = {y.x, y.y, y.z, y.w}, kk[4] = {k.x, k.y, k.z, k.w}, vv[4] = {v.x, v.y, v.z, v.w};
+    float gy[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float ln = (yy[j] - mu) * rs;
+      const float g = 2.f * (kk[j] + ln - vv[j]) * invd;
+      gy[j] = rs * (g - mg - ln * mgl);
+    }
+    const int64_t o = r * d + 4 * c;
+    store4<T>(dout_a + o, make_float4(gy[0], gy[1], gy[2], gy[3]));
+    store4<T>(doutW + o, make_float4(kw * gy[0], kw * gy[1], kw * gy[2], kw * gy[3]));
+    store4<T>(doutM + o, make_float4(km * gy[0], km * gy[1], km * gy[2], km * gy[3]));
+  }
+  // ---- queries: the outputs at the chunk-start weights
+  const float4* zr = reinterpret_cast<const float4*>(yq + r * d);
+  const float4* qr = reinterpret_cast<const float4*>(qres + r * d);
+  stats(zr, mu, rs);
+  float4* orow = reinterpret_cast<float4*>(O + ti * d);
+  for (int c = lane; c < q4; c += 32) {
+    const float4 y = zr[c], q = qr[c];
+    orow[c] = make_float4(q.x + (y.x - mu) * rs, q.y + (y.y - mu) * rs, q.z + (y.z - mu) * rs, q.w + (y.w - mu) * rs);
+  }
+}
+
 // Input-dependent update scalars ("Rethinking Expressivity and Efficiency in
 // Test-Time Training", 依赖于输入的动态参数化), one warp per token row x_t:
 //   eta_t   = eta_base sigmoid(w_eta . x_t + b_eta)

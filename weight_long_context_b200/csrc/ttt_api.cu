@@ -67,6 +67,20 @@ struct GraphKey {
 
 }  // namespace ttt
 
+namespace ttt {
+// Pointers and sizes a captured reconstruction prefill graph was built for.
+struct ReconKey {
+  int batch, T, b;
+  const void *K, *V, *Q, *W, *M, *eta, *beta, *gamma, *O, *loss, *ws;
+  size_t ws_bytes;
+  bool operator==(const ReconKey& o) const {
+    return batch == o.batch && T == o.T && b == o.b && K == o.K && V == o.V && Q == o.Q && W == o.W && M == o.M &&
+           eta == o.eta && beta == o.beta && gamma == o.gamma && O == o.O && loss == o.loss && ws == o.ws &&
+           ws_bytes == o.ws_bytes;
+  }
+};
+}  // namespace ttt
+
 struct ttt_handle {
   ttt_config cfg;
   int device = 0;
@@ -81,6 +95,9 @@ struct ttt_handle {
   bool have_key = false;
   bool use_graph = true;
   int64_t launches = 0;     // kernel launches of the last prefill
+  cudaGraphExec_t exec_recon = nullptr;   // the reconstruction head's graph
+  ttt::ReconKey rkey{};
+  bool have_rkey = false;
 };
 
 namespace ttt {
@@ -95,6 +112,8 @@ struct Plan {
   size_t esz;  // operand element size
   size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, logits, P, dz, dout, dout_a,
       doutW[2], doutM[2], dU, sk_partial, sk_counters, total;
+  bool recon;           // reconstruction head: no LM-head buffers; yk, yq, qres below
+  size_t yk, yq, qres;  // fp32 [n, d]: MLP outputs on the keys and queries, the query rows
   size_t sk_partial_bytes, sk_counter_count;
 };
 
@@ -110,7 +129,8 @@ static int head_parts(int precision, int V) {
 static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   Plan p{};
   p.B = B; p.T = T; p.b = b; p.nchunks = b > 0 ? T / b : 0; p.n = B * b;
-  p.d = c.d; p.h = c.hidden; p.V = c.vocab; p.L = c.n_blocks;
+  p.recon = c.head == TTT_HEAD_RECON;
+  p.d = c.d; p.h = c.hidden; p.V = p.recon ? 0 : c.vocab; p.L = c.n_blocks;
   p.swiglu = c.mlp == TTT_MLP_SWIGLU; p.has_static = c.has_static != 0;
   p.m = p.swiglu ? 3 : 2; p.H2 = p.swiglu ? 2 * p.h : p.h;
   p.nM = p.L * (p.has_static ? 2 : 1);
@@ -125,7 +145,7 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   if (vs < 256) vs = 256;
   if (vs >= p.V) vs = p.V;
   p.Vs = (int)vs;
-  p.nslabs = (p.V + p.Vs - 1) / p.Vs;
+  p.nslabs = p.Vs > 0 ? (p.V + p.Vs - 1) / p.Vs : 0;
 
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
@@ -138,7 +158,7 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.actin = take(e * p.nM * n * d);
   p.aw = take(e * p.nM * n * d);
   p.am = take(e * p.nM * n * d);
-  p.act = take(e * p.nM * n * h);
+  p.act = take(e * (p.nM + (p.recon ? 1 : 0)) * n * h);   // reconstruction: key and query activations
   p.fac = take(e * p.nM * n * H2);
   p.z = take(e * n * d);
   p.rstd = take(4 * n);
@@ -155,6 +175,9 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.dout_a = take(e * n * d);
   for (int i = 0; i < 2; ++i) { p.doutW[i] = take(e * n * d); p.doutM[i] = take(e * n * d); }
   p.dU = take(e * n * H2);
+  p.yk = take(p.recon ? 4 * n * d : 0);
+  p.yq = take(p.recon ? 4 * n * d : 0);
+  p.qres = take(p.recon ? 4 * n * d : 0);
   // split-K scratch of the CTA-pair GEMMs (only when 256-row pair tiles exist)
   p.sk_partial_bytes = (c.precision == TTT_PREC_BF16 && n >= 256) ? std::min<size_t>(64ull << 20, 64ull * 1024 * n) : 0;
   p.sk_counter_count = p.sk_partial_bytes ? 65536 : 0;
@@ -204,11 +227,11 @@ static Operand opnd(const void* p, int64_t ld, int64_t bs, int kmajor, int64_t r
 // ---------------------------------------------------------------------------
 enum KernelClass {
   K_SCAN, K_SHADOW, K_GATHER, K_MLP_UP, K_MLP_DOWN, K_RMS_FWD, K_CE_LSE, K_CE_ROWS, K_CE_MEAN,
-  K_CE_GRAD, K_CE_DZ, K_RMS_BWD, K_BWD_DA, K_BWD_DX, K_AGG_UPDATE, K_NCLASS
+  K_CE_GRAD, K_CE_DZ, K_RMS_BWD, K_BWD_DA, K_BWD_DX, K_AGG_UPDATE, K_RECON_ROWS, K_NCLASS
 };
 static const char* kClassName[K_NCLASS] = {
     "scalar_scan", "w_shadow", "gather", "mlp_up", "mlp_down", "rmsnorm_fwd", "ce_logits_lse", "ce_rows",
-    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update"};
+    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update", "recon_rows"};
 
 struct Prof {
   bool timing = false;
@@ -459,6 +482,128 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
 }
 
 // ---------------------------------------------------------------------------
+// E2-TTT's own layer, chunk after chunk ("Rethinking Expressivity and
+// Efficiency in Test-Time Training", Algorithm 1): outputs o_t = f_{W_0}(q_t)
+// and per-token losses at the chunk-start weights, one backward to the
+// activation gradients, the two aggregations of the chunk update.  One dynamic
+// block: f_W(x) = x + LN(MLP_W(x)).
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_recon(ttt_handle* hd, const Plan& p, const float* Kin, const float* Vin, const float* Qin,
+                                 float* W, float* M, const float* eta, const float* beta, const float* gamma,
+                                 float* O, float* chunk_loss, char* ws, cudaStream_t st, Prof& prof) {
+  const int B = p.B, b = p.b, d = p.d, h = p.h, H2 = p.H2;
+  const int64_t n = p.n;
+  float* KW = reinterpret_cast<float*>(ws + p.KW);
+  float* KM = reinterpret_cast<float*>(ws + p.KM);
+  float* consts = reinterpret_cast<float*>(ws + p.consts);
+  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+  float* kres = reinterpret_cast<float*>(ws + p.resid);
+  T* kin = reinterpret_cast<T*>(ws + p.actin);
+  T* aw = reinterpret_cast<T*>(ws + p.aw);
+  T* am = reinterpret_cast<T*>(ws + p.am);
+  T* act_k = reinterpret_cast<T*>(ws + p.act);
+  T* act_q = act_k + n * h;
+  T* fac = reinterpret_cast<T*>(ws + p.fac);
+  T* qin = reinterpret_cast<T*>(ws + p.z);
+  float* ltok = reinterpret_cast<float*>(ws + p.ltok);
+  T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
+  T* doutW = reinterpret_cast<T*>(ws + p.doutW[0]);
+  T* doutM = reinterpret_cast<T*>(ws + p.doutM[0]);
+  T* dU = reinterpret_cast<T*>(ws + p.dU);
+  float* yk = reinterpret_cast<float*>(ws + p.yk);
+  float* yq = reinterpret_cast<float*>(ws + p.yq);
+  float* qres = reinterpret_cast<float*>(ws + p.qres);
+  int* status = hd->status;
+  SplitScratch ss;
+  ss.partial = reinterpret_cast<float*>(ws + p.sk_partial);
+  ss.partial_bytes = p.sk_partial_bytes;
+  ss.counters = reinterpret_cast<int*>(ws + p.sk_counters);
+  ss.counter_count = p.sk_counter_count;
+  if (!p.sk_partial_bytes) ss = SplitScratch();
+  cudaError_t err;
+#define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
+#define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
+  const double e = (double)p.esz;
+  if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
+  LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T,
+         TRY(launch_scalar_scan(hd->cfg.update_rule, eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
+  LAUNCH(K_SHADOW, 0, (4.0 + e) * B * p.m * h * d,
+         (build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B, h, d, p.swiglu ? 1 : 0)));
+  const int64_t seqW = (int64_t)p.m * h * d;   // params per sequence (one block)
+  const bool sw = p.swiglu;
+  const T* w1 = Wsh;
+  const T* w2 = Wsh + (int64_t)H2 * d;
+  for (int c = 0; c < p.nchunks; ++c) {
+    TokenMap tm{b, p.T, c};
+    LAUNCH(K_GATHER, 0, (8.0 + 3 * e) * n * d,
+           (gather_chunk_kernel<T><<<592, 256, 0, st>>>(Kin, p.T, b, c, d, n, kres, kin, aw, am, KW, KM, p.kscale)));
+    LAUNCH(K_GATHER, 0, (8.0 + e) * n * d,
+           (gather_chunk_kernel<T><<<592, 256, 0, st>>>(Qin, p.T, b, c, d, n, qres, qin, nullptr, nullptr, KW, KM,
+                                                        p.kscale)));
+    // forward at the chunk-start weights: keys (with the backward's factors), then queries
+    for (int side = 0; side < 2; ++side) {
+      T* xin = side ? qin : kin;
+      T* aout = side ? act_q : act_k;
+      T* fptr = side ? nullptr : fac;
+      float* y = side ? yq : yk;
+      {
+        GemmShape s{b, H2, d, B};
+        Operand A = opnd(xin, d, (int64_t)b * d, 1, b);
+        Operand Bw = opnd(w1, d, seqW, 1, H2);
+        const double fl = 2.0 * b * H2 * d * B;
+        const double by = e * ((double)n * d + (double)H2 * d * B + (double)n * h + (fptr ? (double)n * H2 : 0.0));
+        if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, b}, st, status, ss))));
+        else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, b}, st, status, ss))));
+      }
+      {
+        GemmShape s{b, d, h, B};
+        Operand A = opnd(aout, h, (int64_t)b * h, 1, b);
+        Operand Bw = opnd(w2, h, seqW, 1, d);
+        LAUNCH(K_MLP_DOWN, 2.0 * b * d * h * B, e * ((double)n * h + (double)d * h * B) + 4.0 * n * d,
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiStoreBatched{y, d, (int64_t)b * d}, st, status, ss))));
+      }
+    }
+    LAUNCH(K_RECON_ROWS, 0, 4.0 * n * d * 6 + 3 * e * n * d,
+           (recon_rows_kernel<T><<<(unsigned)((n + 7) / 8), 256, 0, st>>>(yk, kres, Vin, yq, qres, tm, n, d,
+                                                                          hd->cfg.rms_eps, KW, KM, p.kscale, ltok,
+                                                                          dout_a, doutW, doutM, O)));
+    LAUNCH(K_CE_MEAN, 0, 4.0 * n, (ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status)));
+    {  // dA = g_y W_down -> dU
+      GemmShape s{b, h, d, B};
+      Operand A = opnd(dout_a, d, (int64_t)b * d, 1, b);
+      Operand Bw = opnd(w2, h, seqW, 0, d);
+      const double fl = 2.0 * b * h * d * B;
+      const double by = e * ((double)n * d + (double)d * h * B + 2.0 * n * H2);
+      if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fac, dU, h, b}, st, status, ss))));
+      else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fac, dU, h, b}, st, status, ss))));
+    }
+    {  // rows of W1 (and W2 for SwiGLU): sum_t dU_t (x) (-K_t k_t)
+      GemmShape s{H2, d, b, B};
+      Operand A = opnd(dU, H2, (int64_t)b * H2, 0, b);
+      Operand B1 = opnd(aw, d, (int64_t)b * d, 0, b);
+      Operand B2 = opnd(am, d, (int64_t)b * d, 0, b);
+      EpiUpdate<T> ep{W, M, Wsh, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+      LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B, (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
+             TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
+    }
+    {  // the output matrix: sum_t (-K_t g_y,t) (x) a_t
+      GemmShape s{d, h, b, B};
+      Operand A = opnd(doutW, d, (int64_t)b * d, 0, b);
+      Operand A2 = opnd(doutM, d, (int64_t)b * d, 0, b);
+      Operand Bx = opnd(act_k, h, (int64_t)b * h, 0, b);
+      EpiUpdate<T> ep{W + (int64_t)H2 * d, M + (int64_t)H2 * d, Wsh + (int64_t)H2 * d, seqW, seqW, consts, c,
+                      p.nchunks, h, 0};
+      LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B, (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
+             TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+    }
+  }
+#undef LAUNCH
+#undef TRY
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
 // Validation
 // ---------------------------------------------------------------------------
 static ttt_status check_config(const ttt_config* c) {
@@ -472,11 +617,16 @@ static ttt_status check_config(const ttt_config* c) {
   if (c->update_rule != TTT_RULE_E2TTT && c->update_rule != TTT_RULE_LACT)
     return fail(TTT_ERR_INVALID_ARG, "update_rule must be E2TTT or LACT");
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return fail(TTT_ERR_INVALID_ARG, "rms_eps must be finite and >= 0");
-  if (c->d < 16 || c->hidden < 16 || c->vocab < 16 || c->n_blocks < 1)
+  if (c->head != TTT_HEAD_LM && c->head != TTT_HEAD_RECON) return fail(TTT_ERR_INVALID_ARG, "head must be LM or RECON");
+  const bool recon = c->head == TTT_HEAD_RECON;
+  if (recon && (c->n_blocks != 1 || c->has_static))
+    return fail(TTT_ERR_UNSUPPORTED, "the reconstruction head takes one dynamic block and no static MLP");
+  const int vocab = recon ? 16 : c->vocab;   // unused by the reconstruction head
+  if (c->d < 16 || c->hidden < 16 || vocab < 16 || c->n_blocks < 1)
     return fail(TTT_ERR_SHAPE, "d, hidden, vocab must be >= 16 and n_blocks >= 1");
-  if (c->d > 16384 || c->hidden > 65536 || c->vocab >= (1 << 26) || c->n_blocks > 64)
+  if (c->d > 16384 || c->hidden > 65536 || vocab >= (1 << 26) || c->n_blocks > 64)
     return fail(TTT_ERR_SHAPE, "size above the supported maximum");
-  if (c->d % 16 || c->hidden % 16 || c->vocab % 16)
+  if (c->d % 16 || c->hidden % 16 || vocab % 16)
     return fail(TTT_ERR_UNSUPPORTED, "d, hidden and vocab must be multiples of 16");
   return TTT_OK;
 }
@@ -554,7 +704,9 @@ ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* 
                       const float* static_w, ttt_handle** out) {
   ttt_status s = check_config(cfg);
   if (s != TTT_OK) return s;
-  if (!lm_head || !rms_gain || !out) return fail(TTT_ERR_INVALID_ARG, "lm_head, rms_gain and out must be non-NULL");
+  const bool recon = cfg->head == TTT_HEAD_RECON;
+  if (!out || (!recon && (!lm_head || !rms_gain)))
+    return fail(TTT_ERR_INVALID_ARG, "lm_head, rms_gain and out must be non-NULL");
   if (cfg->has_static && !static_w) return fail(TTT_ERR_INVALID_ARG, "static_w is NULL but has_static = 1");
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
@@ -571,18 +723,20 @@ ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* 
   const int64_t V = cfg->vocab, d = cfg->d, hh = cfg->hidden;
   const int m = cfg->mlp == TTT_MLP_SWIGLU ? 3 : 2;
   const size_t esz = cfg->precision == TTT_PREC_FP32 ? 4 : 2;
-  CTRY(cudaMalloc(&h->E, esz * V * d));
-  CTRY(cudaMalloc(&h->gain, 4 * d));
   CTRY(cudaMalloc(&h->status, 8));
   h->zero_flag = h->status + 1;
   CTRY(cudaMemset(h->status, 0, 8));
   CTRY(cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking));
-  CTRY(cudaMemcpyAsync(h->gain, rms_gain, 4 * d, cudaMemcpyDeviceToDevice, h->cap));
-  if (cfg->precision == TTT_PREC_FP32) {
-    CTRY(cudaMemcpyAsync(h->E, lm_head, 4 * V * d, cudaMemcpyDeviceToDevice, h->cap));
-  } else {
-    cast_kernel<bf16><<<1184, 256, 0, h->cap>>>(lm_head, static_cast<bf16*>(h->E), V * d);
-    CTRY(cudaGetLastError());
+  if (!recon) {   // the frozen LM head and RMSNorm gain
+    CTRY(cudaMalloc(&h->E, esz * V * d));
+    CTRY(cudaMalloc(&h->gain, 4 * d));
+    CTRY(cudaMemcpyAsync(h->gain, rms_gain, 4 * d, cudaMemcpyDeviceToDevice, h->cap));
+    if (cfg->precision == TTT_PREC_FP32) {
+      CTRY(cudaMemcpyAsync(h->E, lm_head, 4 * V * d, cudaMemcpyDeviceToDevice, h->cap));
+    } else {
+      cast_kernel<bf16><<<1184, 256, 0, h->cap>>>(lm_head, static_cast<bf16*>(h->E), V * d);
+      CTRY(cudaGetLastError());
+    }
   }
   if (cfg->has_static) {
     const int64_t count = cfg->n_blocks;
@@ -603,6 +757,7 @@ void ttt_destroy(ttt_handle* h) {
   if (!h) return;
   if (h->cap) cudaStreamSynchronize(h->cap);
   if (h->exec) cudaGraphExecDestroy(h->exec);
+  if (h->exec_recon) cudaGraphExecDestroy(h->exec_recon);
   if (h->E) cudaFree(h->E);
   if (h->gain) cudaFree(h->gain);
   if (h->S) cudaFree(h->S);
@@ -625,6 +780,7 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
                        void* stream) {
   ttt_status s = check_shape(h, batch, T, b);
   if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the reconstruction layer: use ttt_prefill_recon");
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
@@ -673,12 +829,67 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   return TTT_OK;
 }
 
+ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* K, const float* V,
+                             const float* Q, float* W, float* M, const float* eta, const float* beta,
+                             const float* gamma, float* O, float* chunk_loss, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_RECON) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the LM head: use ttt_prefill");
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!K || !V || !Q || !W || !M || !eta || !beta || !gamma || !O || !chunk_loss)
+    return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  Plan p = make_plan(h->cfg, batch, T, b);
+  if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(Q) |
+       reinterpret_cast<uintptr_t>(O) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "K, V, Q, O, W and M must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  Prof prof;
+  auto enqueue = [&](cudaStream_t q) -> cudaError_t {
+    if (h->cfg.precision == TTT_PREC_FP32)
+      return enqueue_recon<float>(h, p, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, ws, q, prof);
+    return enqueue_recon<bf16>(h, p, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, ws, q, prof);
+  };
+  if (!h->use_graph) {
+    cudaError_t e = enqueue(st);
+    if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    h->launches = prof.launches;
+    return TTT_OK;
+  }
+  ReconKey key{batch, T, b, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, workspace, ws_bytes};
+  if (!(h->have_rkey && h->rkey == key && h->exec_recon)) {
+    if (h->exec_recon) { cudaGraphExecDestroy(h->exec_recon); h->exec_recon = nullptr; }
+    h->have_rkey = false;
+    TTT_CUDA_TRY(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+    cudaError_t e = enqueue(h->cap);
+    cudaGraph_t g = nullptr;
+    cudaError_t e2 = cudaStreamEndCapture(h->cap, &g);
+    if (e != cudaSuccess || e2 != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      set_last_error("capture", cudaGetErrorString(e != cudaSuccess ? e : e2), __FILE__, __LINE__);
+      return TTT_ERR_CUDA;
+    }
+    e = cudaGraphInstantiate(&h->exec_recon, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) { h->exec_recon = nullptr; set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    h->rkey = key;
+    h->have_rkey = true;
+    h->launches = prof.launches;
+  }
+  TTT_CUDA_TRY(cudaGraphLaunch(h->exec_recon, st));
+  return TTT_OK;
+}
+
 ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
                                 const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
                                 const float* gamma, float* chunk_loss, void* workspace, size_t ws_bytes,
                                 void* stream, ttt_kernel_stat* stats, int32_t max_stats, int32_t* n_stats) {
   ttt_status s = check_shape(h, batch, T, b);
   if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the reconstruction layer: use ttt_prefill_recon");
   if (!stats || !n_stats || max_stats < 0) return fail(TTT_ERR_INVALID_ARG, "stats / n_stats missing");
   *n_stats = 0;
   if (batch == 0 || T == 0) return TTT_OK;
@@ -756,6 +967,7 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
                                const float* gamma, float* chunk_loss, void* stream) {
   ttt_status s = check_shape(h, batch, T, b);
   if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the reconstruction layer: use ttt_prefill_recon");
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");

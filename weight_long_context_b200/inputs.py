@@ -54,6 +54,7 @@ class Workload:
     rms_eps: float = 1e-6
     reduction: str = "mean"  # chunk objective: mean (default) or sum of token losses
     update_rule: str = "e2ttt"  # chunk update: "e2ttt" (Proposition 3.1) or "lact" (chunk-wise rule)
+    head: str = "lm"  # "lm": next-token cross-entropy; "recon": E2-TTT's key/value reconstruction layer
 
     @property
     def n_mats(self) -> int:
@@ -107,6 +108,27 @@ def zipf_tokens(rng: np.random.Generator, vocab: int, shape, s: float = 1.1) -> 
     u = rng.random(size=shape)
     idx = np.searchsorted(cdf, u, side="right")
     return np.minimum(idx, vocab - 1).astype(np.int32)
+
+
+def make_recon_inputs(w: Workload, seed: int = 0, T: Optional[int] = None, batch: Optional[int] = None,
+                      m0_scale: float = 0.0, w0_per_sequence: bool = False) -> Dict[str, np.ndarray]:
+    """Inputs of E2-TTT's own layer: everything make_inputs draws (its hidden
+    rows serve as the keys K), then values V and queries Q [B,T,d] from a
+    second generator seeded (seed, 1), rows scaled to unit RMS like K."""
+    x = make_inputs(w, seed, T=T, batch=batch, m0_scale=m0_scale, w0_per_sequence=w0_per_sequence)
+    rng = np.random.default_rng([seed, 1])
+    B, T_, d = x["hidden"].shape
+
+    def unit_rows():
+        a = _normal(rng, (B, T_, d))
+        if a.size:
+            rms = np.sqrt(np.mean(a.astype(np.float64) ** 2, axis=-1, keepdims=True))
+            a = (a / rms).astype(np.float32)
+        return a
+    x["K"] = x["hidden"]
+    x["V"] = unit_rows()
+    x["Q"] = unit_rows()
+    return x
 
 
 def make_inputs(w: Workload, seed: int = 0, T: Optional[int] = None,

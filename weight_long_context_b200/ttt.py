@@ -24,9 +24,10 @@ MLP = {"gelu": 0, "swiglu": 1}
 PRECISION = {"fp32": 0, "bf16": 1}
 REDUCTION = {"mean": 0, "sum": 1}
 RULE = {"e2ttt": 0, "lact": 1}
+HEAD = {"lm": 0, "recon": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
-            "ttt_prefill_profiled",
+            "ttt_prefill_profiled", "ttt_prefill_recon",
             "ttt_scalar_kernels", "ttt_scalar_heads", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
@@ -43,7 +44,7 @@ class ttt_config(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("hidden", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("n_blocks", ctypes.c_int32), ("mlp", ctypes.c_int32), ("has_static", ctypes.c_int32),
                 ("precision", ctypes.c_int32), ("loss_reduction", ctypes.c_int32),
-                ("rms_eps", ctypes.c_float), ("update_rule", ctypes.c_int32)]
+                ("rms_eps", ctypes.c_float), ("update_rule", ctypes.c_int32), ("head", ctypes.c_int32)]
 
 
 class ttt_kernel_stat(ctypes.Structure):
@@ -72,6 +73,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill.restype = I32
     lib.ttt_prefill_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P]
+    lib.ttt_prefill_recon.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.ttt_prefill_recon.restype = I32
     lib.ttt_prefill_noalloc.restype = I32
     lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
@@ -221,14 +224,18 @@ class Handle:
     def __init__(self, d: int, hidden: int, vocab: int, n_blocks: int, mlp: str, has_static: bool,
                  precision: str, lm_head: torch.Tensor, rms_gain: torch.Tensor,
                  static_w: Optional[torch.Tensor] = None, rms_eps: float = 1e-6,
-                 reduction: str = "mean", update_rule: str = "e2ttt"):
-        dev = lm_head.device
-        _dev(lm_head, torch.float32, "lm_head", dev)
-        _dev(rms_gain, torch.float32, "rms_gain", dev)
+                 reduction: str = "mean", update_rule: str = "e2ttt", head: str = "lm",
+                 device: Optional[torch.device] = None):
+        dev = lm_head.device if lm_head is not None else device
+        if dev is None:
+            raise ValueError("device is required when lm_head is None")
+        if head == "lm":
+            _dev(lm_head, torch.float32, "lm_head", dev)
+            _dev(rms_gain, torch.float32, "rms_gain", dev)
         if static_w is not None:
             _dev(static_w, torch.float32, "static_w", dev)
         self.cfg = ttt_config(d, hidden, vocab, n_blocks, MLP[mlp], int(bool(has_static)),
-                              PRECISION[precision], REDUCTION[reduction], rms_eps, RULE[update_rule])
+                              PRECISION[precision], REDUCTION[reduction], rms_eps, RULE[update_rule], HEAD[head])
         self.device = dev
         self.n_mats = 2 if mlp == "gelu" else 3
         with torch.cuda.device(dev):
@@ -268,6 +275,49 @@ class Handle:
                                           _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(chunk_loss),
                                           _ptr(ws), ws.numel(), _stream_ptr(stream)), "ttt_prefill")
         return chunk_loss
+
+    def prefill_recon(self, K, V, Q, W, M, eta, beta, gamma, b: int, O: Optional[torch.Tensor] = None,
+                      chunk_loss: Optional[torch.Tensor] = None, stream=None):
+        """E2-TTT's own layer on device tensors (handle created with head="recon"):
+        K, V, Q [B,T,d] f32; W/M [B*m*h*d] f32 updated in place; eta/beta/gamma
+        [B,T].  Returns (chunk_loss [B, T/b], O [B,T,d]) on the device."""
+        dev = self.device
+        B, T, d = K.shape
+        for t, nm in ((K, "K"), (V, "V"), (Q, "Q"), (W, "W"), (M, "M"), (eta, "eta"), (beta, "beta"),
+                      (gamma, "gamma")):
+            _dev(t, torch.float32, nm, dev)
+        if tuple(V.shape) != (B, T, d) or tuple(Q.shape) != (B, T, d):
+            raise ValueError("K, V and Q must have the same shape [B, T, d]")
+        nparams = B * self.n_mats * self.cfg.hidden * self.cfg.d
+        if W.numel() != nparams or M.numel() != nparams:
+            raise ValueError(f"W and M must hold {nparams} floats")
+        nc = T // b if b > 0 else 0
+        if chunk_loss is None:
+            chunk_loss = torch.empty((B, nc), dtype=torch.float32, device=dev)
+        if O is None:
+            O = torch.empty((B, T, d), dtype=torch.float32, device=dev)
+        ws = self.workspace(B, T, b)
+        _check(load_library().ttt_prefill_recon(self._h, B, T, b, _ptr(K), _ptr(V), _ptr(Q), _ptr(W), _ptr(M),
+                                                _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(O), _ptr(chunk_loss),
+                                                _ptr(ws), ws.numel(), _stream_ptr(stream)), "ttt_prefill_recon")
+        return chunk_loss, O
+
+    def prefill_recon_host(self, K, V, Q, W0, M0, eta, beta, gamma, b: int, stream=None):
+        """End-to-end reconstruction call on HOST tensors: copies in, runs, copies
+        W, M, the chunk losses and the outputs back.  Returns host tensors
+        (W, M, chunk_loss, O)."""
+        dev = self.device
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(st):
+            d_in = [t.to(dev, non_blocking=True) for t in (K, V, Q, W0, M0, eta, beta, gamma)]
+            loss, O = self.prefill_recon(*d_in, b=b, stream=st)
+            outs = []
+            for t in (d_in[3], d_in[4], loss, O):
+                o = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                o.copy_(t, non_blocking=True)
+                outs.append(o)
+        st.synchronize()
+        return tuple(outs)
 
     def prefill_profiled(self, hidden, tokens, W, M, eta, beta, gamma, b: int, stream=None):
         """ttt_prefill_profiled: same results as prefill (W, M updated in place),
