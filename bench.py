@@ -59,6 +59,10 @@ def flops_per_token(w: I.Workload) -> float:
     logits recompute of the cross-entropy backward is not counted.
     """
     d, h, V, L, m = w.d, w.hidden, w.vocab, w.n_blocks, w.n_mats
+    if w.head == "recon":
+        # E2-TTT's layer: MLP forward on keys and on queries, backward to the
+        # activation only (one block), both aggregations
+        return float(2 * (2 * m * d * h) + 2 * d * h + 2 * m * d * h * (1 if w.scalars == "sgd" else 2))
     n_static = L if w.has_static else 0
     fwd = (L + n_static) * 2 * m * d * h
     head = 4 * d * V
@@ -214,8 +218,15 @@ def oracle_chunks(w: I.Workload, n_chunks: int, seed: int = 0):
     """Run the oracle on the first n_chunks chunks of one sequence; returns seconds."""
     import oracle  # test infrastructure: the CPU baseline only
     ws = w.with_(T=n_chunks * w.b, batch=1)
-    x = I.make_inputs(ws, seed=seed)
     dtype = np.float64 if w.precision == "fp32" else np.float32
+    if w.head == "recon":
+        x = I.make_recon_inputs(ws, seed=seed)
+        t0 = time.perf_counter()
+        oracle.prefill_recon(w.mlp, w.d, w.hidden, x["W0"], x["M0"], x["K"], x["V"], x["Q"], x["eta"], x["beta"],
+                             x["gamma"], w.b, w.rms_eps, dtype=dtype, reduction=w.reduction,
+                             update="lact" if w.update_rule == "lact" else "closed")
+        return time.perf_counter() - t0
+    x = I.make_inputs(ws, seed=seed)
     model = oracle.make_model(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.rms_eps, x["lm_head"], x["rms_gain"],
                               x["static_w"], dtype=dtype)
     t0 = time.perf_counter()
@@ -276,6 +287,7 @@ def workload_config(w: I.Workload) -> dict:
     return {"workload": w.name, "d": w.d, "hidden": w.hidden, "vocab": w.vocab, "blocks": w.n_blocks,
             "mlp": w.mlp, "static_mlp": w.has_static, "T": w.T, "chunk_b": w.b, "sequences_per_gpu": w.batch,
             "scalars": w.scalars, "loss_reduction": w.reduction, "update_rule": w.update_rule,
+            "head": "next-token cross-entropy" if w.head == "lm" else "key/value reconstruction (E2-TTT layer)",
             "precision": "fp32" if w.precision == "fp32" else "bf16 GEMM operands, fp32 accumulate/state",
             "l2": ("inputs larger than L2 (hidden + fast-weight state %.2f GiB per step)" % ((input_bytes(w) + state_bytes(w)) / 2 ** 30))
                   if big else "L2 flushed between timed steps (write of a 256 MiB buffer)"}
@@ -286,6 +298,8 @@ def workload_config(w: I.Workload) -> dict:
 # ---------------------------------------------------------------------------
 
 def run_ours(args, w: I.Workload):
+    if w.head == "recon":
+        return run_ours_recon(args, w)
     import torch
     from weight_long_context_b200 import ttt
 
@@ -444,12 +458,121 @@ def run_ours(args, w: I.Workload):
     return 0
 
 
+def run_ours_recon(args, w: I.Workload):
+    """E2-TTT's own layer (ttt_prefill_recon): the same timing rules; the
+    roofline is taken over the whole step (this head has no per-kernel replay)."""
+    import torch
+    from weight_long_context_b200 import ttt
+
+    rank, world, local = dist_env()
+    if world > 1:
+        init_dist("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    st = torch.cuda.current_stream(dev)
+    x = I.make_recon_inputs(w, seed=rank)
+    T = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    h = ttt.Handle(w.d, w.hidden, w.vocab, 1, w.mlp, False, w.precision, None, None, None, w.rms_eps, w.reduction,
+                   w.update_rule, head="recon", device=dev)
+    K, V, Q, W, M = T(x["K"]), T(x["V"]), T(x["Q"]), T(x["W0"]), T(x["M0"])
+    eta, beta, gamma = T(x["eta"]), T(x["beta"]), T(x["gamma"])
+    O = torch.empty_like(K)
+    flush = None
+    if 3 * K.numel() * 4 + state_bytes(w) <= 2 * L2_BYTES:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        return h.prefill_recon(K, V, Q, W, M, eta, beta, gamma, w.b, O=O, stream=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert h.device_status() == 0, "device status after warm-up"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        ev[i][0].record(st)
+        step()
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    status = h.device_status()
+    mean_ms = reduce_max(statistics.mean(step_ms), dev)
+    tokens_per_step = w.batch * w.T
+    value = whole_job_rate(tokens_per_step, world, mean_ms / 1e3)
+    pk = peaks()
+    # kernels per step in ttt_prefill_recon's launch sequence: the scalar scan and
+    # the operand shadow, then per chunk two gathers, four forward GEMMs, the
+    # row kernel, the chunk mean, the backward GEMM and the two aggregations
+    launches = 2 + 11 * w.n_chunks
+
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    hx = [pin(x[k]) for k in ("K", "V", "Q", "W0", "M0", "eta", "beta", "gamma")]
+    h2d = sum(t.numel() * t.element_size() for t in hx)
+    d2h = 2 * hx[3].numel() * 4 + w.batch * w.n_chunks * 4 + hx[0].numel() * 4
+    del K, V, Q, W, M, eta, beta, gamma, O
+    torch.cuda.empty_cache()
+    h.prefill_recon_host(*hx, b=w.b, stream=st)
+    e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e_steps):
+        h.prefill_recon_host(*hx, b=w.b, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e_steps, dev)
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        fl = flops_per_token(w)
+        tflops = value * fl / 1e12
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16" if w.precision == "bf16" else "f32", "data": "synthetic",
+                "config": workload_config(w), "algorithmic_tflops": tflops,
+                "pct_of_bf16_peak": {"burst": tflops / world / pk["tflops"],
+                                     "sustained": tflops / world / pk["tflops_sustained"], "source": pk["source"]},
+                "clocks": clk,
+                "e2e": {"value": whole_job_rate(tokens_per_step, world, e2e_ms / 1e3), "unit": UNIT,
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                        "steps": e_steps},
+                "gpu_launches": launches * args.steps,
+                "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": pk["tflops_sustained"],
+                             "unit": "TFLOP/s", "frac": tflops / world / pk["tflops_sustained"], "traffic": None,
+                             "kernel": "whole step (this head has no per-kernel replay)",
+                             "peak_source": f"{pk['source']} (bf16 sustained)"},
+                "device_status": status}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER + ["e2ttt_layer_128k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scalar-heads", action="store_true",

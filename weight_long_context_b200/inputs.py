@@ -89,6 +89,10 @@ WORKLOADS: Dict[str, Workload] = {
     # 16 independent sequences, GELU d=1024, h=4096, V=16384, T=8192, b=256
     "batched_16": Workload("batched_16", 1024, 4096, 16384, 1, GELU, False, "bf16",
                            8192, 256, 16, "e2ttt"),
+    # E2-TTT's own layer (key/value reconstruction) at the 128K stack's layer
+    # dimensions: one SwiGLU fast-weight MLP d=2048, h=5632, T=131072, b=1024
+    "e2ttt_layer_128k": Workload("e2ttt_layer_128k", 2048, 5632, 16, 1, SWIGLU, False, "bf16",
+                                 131072, 1024, 1, "e2ttt", head="recon"),
 }
 WORKLOAD_ORDER = ["tiny_sgd", "e2ttt_block", "sgd_3b", "stack_128k", "batched_16"]
 
