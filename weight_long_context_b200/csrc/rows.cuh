@@ -73,10 +73,7 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ h, const float* __r
   const float4* gr = reinterpret_cast<const float4*>(g);
   for (int c = lane; c < (d >> 2); c += 32) {
     float4 x = hr[c], gg = gr[c];
-    zr[4 * c + 0] = from_f<T>(x.x * r * gg.x);
-    zr[4 * c + 1] = from_f<T>(x.y * r * gg.y);
-    zr[4 * c + 2] = from_f<T>(x.z * r * gg.z);
-    zr[4 * c + 3] = from_f<T>(x.w * r * gg.w);
+    store4<T>(zr + 4 * c, make_float4(x.x * r * gg.x, x.y * r * gg.y, x.z * r * gg.z, x.w * r * gg.w));
   }
 }
 
@@ -118,11 +115,11 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dz, const float* __
     float o4[4] = {r * a.x * gg.x - x.x * coef, r * a.y * gg.y - x.y * coef,
                    r * a.z * gg.z - x.z * coef, r * a.w * gg.w - x.w * coef};
     reinterpret_cast<float4*>(dout + row * d)[c] = make_float4(o4[0], o4[1], o4[2], o4[3]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int64_t idx = row * d + 4 * c + j;
-      dout_a[idx] = from_f<T>(o4[j]);
-      if (doutW) { doutW[idx] = from_f<T>(kw * o4[j]); doutM[idx] = from_f<T>(km * o4[j]); }
+    const int64_t idx = row * d + 4 * c;
+    store4<T>(dout_a + idx, make_float4(o4[0], o4[1], o4[2], o4[3]));
+    if (doutW) {
+      store4<T>(doutW + idx, make_float4(kw * o4[0], kw * o4[1], kw * o4[2], kw * o4[3]));
+      store4<T>(doutM + idx, make_float4(km * o4[0], km * o4[1], km * o4[2], km * o4[3]));
     }
   }
 }

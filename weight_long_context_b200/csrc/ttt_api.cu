@@ -137,9 +137,11 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.esz = c.precision == TTT_PREC_FP32 ? 4 : 2;
   p.kscale = (c.loss_reduction == TTT_REDUCE_MEAN && b > 0) ? 1.0f / (float)b : 1.0f;
   p.ntn = head_parts(c.precision, p.V);
-  // vocabulary slab: the [n, Vs] slab of dl/dlogits is the only per-vocabulary
-  // buffer; capped at 32 MiB so it stays resident in L2.
-  const size_t cap = 32ull << 20;
+  // vocabulary slab: the [n, Vs] slab of dl/dlogits.  Recomputing the logits
+  // (fp32 path): capped at 32 MiB so it stays resident in L2.  With the logits
+  // kept (bf16 path) pass B is elementwise and one dz GEMM over the whole
+  // vocabulary beats two smaller ones: capped at 128 MiB.
+  const size_t cap = (c.precision == TTT_PREC_BF16 ? 128ull : 32ull) << 20;
   int64_t vs = (int64_t)(cap / ((size_t)p.n * p.esz));
   vs = vs / 256 * 256;
   if (vs < 256) vs = 256;
