@@ -33,7 +33,7 @@ Pages cited by title:
   with suffix products btilde_t = prod_{i>t} beta_i, gtilde_t = prod_{i>t}
   gamma_i and R_t = sum_{i>=t} gtilde_i / btilde_i.
 
-Readings where the pages leave a step open (each listed in the design doc):
+Readings where the pages leave a step open:
   * tokens[t] is the label of hidden row t (the caller pre-shifts);
   * the chunk objective is the MEAN next-token loss over the chunk (the default
     reduction of the first inner-loop sketch on [TTT-E2E]); the per-token loss
