@@ -32,6 +32,9 @@ Pages cited by title:
   W_C = gtilde_0 W_0 + btilde_0 R_1 M_0 + sum_t eta_t btilde_t R_t G_t,
   with suffix products btilde_t = prod_{i>t} beta_i, gtilde_t = prod_{i>t}
   gamma_i and R_t = sum_{i>=t} gtilde_i / btilde_i.
+* After the inner loop the whole sequence is scored again at the final
+  weights W_T, forward only ([TTT-E2E] 持续学习框架, 预测 step; the sketch's
+  最终预测 part), per token and per group of b positions ([Review] 图6).
 
 Readings where the pages leave a step open:
   * tokens[t] is the label of hidden row t (the caller pre-shifts);
@@ -478,6 +481,49 @@ def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
         Ms.append(pack_blocks(M))
         Ls.append(L)
     return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls)
+
+
+# ---------------------------------------------------------------------------
+# Final prediction with the updated weights
+# ([TTT-E2E] 持续学习框架 (预测 step) and the sketch's 最终预测 part;
+#  per-position breakdown as in [Review] 图6)
+# ---------------------------------------------------------------------------
+
+def group_means(loss: np.ndarray, b: int) -> np.ndarray:
+    """Mean of each run of b consecutive positions of one sequence."""
+    return loss.reshape(-1, b).mean(axis=1)
+
+
+def final_prediction(model: Model, W_flat, hidden, tokens, b, dtype=np.float64):
+    """Forward-only pass of whole sequences at fixed fast weights.
+
+    After the inner loop the weights W_T hold the context; the sequence is
+    run again through the blocks, the frozen RMSNorm and the LM head at W_T,
+    with no update, and scored by the next-token loss.  Every row is
+    independent here (the weights do not change), so the whole sequence is
+    one forward.  Reading: the losses are reported per token and as the mean
+    of each group of b positions (the loss-by-position curve); the sketch's
+    single final loss is the mean of all of them.
+
+    hidden [B,T,d], tokens [B,T] (labels, as in ``prefill``),
+    W_flat [B * n_blocks * m * h * d].  Returns (token_loss [B,T],
+    group_loss [B, T // b]) in ``dtype``.
+    """
+    mdl = model.astype(dtype)
+    B, T = np.asarray(tokens).shape
+    if T % b != 0:
+        raise ValueError("T must be a multiple of b")
+    shapes = mdl.mat_shapes()
+    per_seq = mdl.n_blocks * sum(r * c for r, c in shapes)
+    Wf = np.asarray(W_flat, dtype=dtype).reshape(B, per_seq)
+    tok = np.zeros((B, T), dtype=dtype)
+    grp = np.zeros((B, T // b), dtype=dtype)
+    for s in range(B):
+        W = unpack_blocks(Wf[s].copy(), mdl.n_blocks, shapes)
+        loss, _ = chunk_forward(mdl, W, np.asarray(hidden[s], dtype=dtype), np.asarray(tokens[s]))
+        tok[s] = loss
+        grp[s] = group_means(loss, b)
+    return tok, grp
 
 
 # ---------------------------------------------------------------------------

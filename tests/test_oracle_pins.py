@@ -508,6 +508,53 @@ def test_chunk_loss_is_mean_at_chunk_start_weights():
 
 
 # ---------------------------------------------------------------------------
+# 6b. Final prediction at the updated weights ([TTT-E2E] 持续学习框架, the
+#     预测 step, and the sketch's 最终预测 part)
+# ---------------------------------------------------------------------------
+
+def test_final_prediction_matches_autograd_restatement():
+    """Two sequences, each at its own W_T from the inner loop: every token's
+    loss equals the independent torch restatement over the whole sequence."""
+    s = tiny_setup(kind="gelu", d=4, h=6, V=7, L=2, static=True, T=12)
+    s2 = tiny_setup(kind="gelu", d=4, h=6, V=7, L=2, static=True, T=12, seed=5)
+    WA, _, _ = run_prefill(s, 4)
+    WB, _, _ = run_prefill(dict(s, X=s2["X"], y=s2["y"], W0=s2["W0"]), 3)
+    X = np.stack([s["X"], s2["X"]])
+    y = np.stack([s["y"], s2["y"]])
+    tok, grp = O.final_prediction(s["model"], np.concatenate([WA, WB]), X, y, 4)
+    assert tok.shape == (2, 12) and grp.shape == (2, 3)
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    for i, W in enumerate((WA, WB)):
+        l = AM.losses("gelu", 4, 6, 2, 1e-6, T_(s["E"]), T_(s["g"]), T_(s["static_w"]), T_(W),
+                      T_(X[i]), torch.tensor(y[i])).numpy()
+        np.testing.assert_allclose(tok[i], l, rtol=1e-12)
+
+
+def test_final_prediction_groups_are_chunk_start_losses():
+    """At the chunk-start weights W_c, group c of a forward-only pass is the
+    loss the inner loop reports for chunk c ([E2-TTT] O^[r] = f_{W^[r-1]}(Q^[r]))."""
+    s = tiny_setup(kind="swiglu", d=4, h=5, V=7, L=2, static=True, T=12)
+    _, _, Ls = run_prefill(s, 4)
+    for c in range(3):
+        if c == 0:
+            Wc = s["W0"]
+        else:
+            sc = dict(s, X=s["X"][:4 * c], y=s["y"][:4 * c], eta=s["eta"][:4 * c],
+                      beta=s["beta"][:4 * c], gamma=s["gamma"][:4 * c])
+            Wc, _, _ = run_prefill(sc, 4)
+        _, grp = O.final_prediction(s["model"], Wc, s["X"][None], s["y"][None], 4)
+        assert grp[0, c] == pytest.approx(Ls[c], rel=1e-13)
+
+
+def test_final_prediction_zero_head_is_log_v():
+    s = tiny_setup(kind="swiglu", d=4, h=5, V=11, L=1, static=False, T=8)
+    s["model"].lm_head[:] = 0.0
+    tok, grp = O.final_prediction(s["model"], s["W0"], s["X"][None], s["y"][None], 2)
+    np.testing.assert_allclose(tok, np.log(11.0), rtol=1e-14)
+    np.testing.assert_allclose(grp, np.log(11.0), rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
 # 7. Planted mistakes: a plausible bug anywhere must fail one of the pins
 # ---------------------------------------------------------------------------
 
@@ -594,6 +641,12 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "layer_norm_backward", lambda g, ln, rs: rs * (g - g.mean(axis=-1, keepdims=True)))
     _must_fail(test_recon_gradients_match_finite_differences)
     monkeypatch.setattr(O, "layer_norm_backward", orig_lnb)
+
+    # (j) final prediction: groups of strided positions instead of consecutive ones
+    orig_gm = O.group_means
+    monkeypatch.setattr(O, "group_means", lambda loss, b: loss.reshape(b, -1).mean(axis=0))
+    _must_fail(test_final_prediction_groups_are_chunk_start_losses)
+    monkeypatch.setattr(O, "group_means", orig_gm)
 
     # (f) the residual dropped from the backward of a block
     orig_mb = O.mlp_backward
