@@ -71,6 +71,13 @@ def flops_per_token(w: I.Workload) -> float:
     return float(fwd + head + bwd + agg)
 
 
+def predict_flops_per_token(w: I.Workload) -> float:
+    """Algorithmic FLOPs per token of the forward-only final prediction: every
+    MLP forward 2 m d h and the logits 2 d V."""
+    n_static = w.n_blocks if w.has_static else 0
+    return float((w.n_blocks + n_static) * 2 * w.n_mats * w.d * w.hidden + 2 * w.d * w.vocab)
+
+
 def state_bytes(w: I.Workload) -> int:
     return w.batch * w.n_blocks * w.block_params * 4 * 2
 
@@ -256,6 +263,24 @@ def cpu_baseline(w: I.Workload, budget_s: float = 12.0) -> dict:
     return {"value": k * w.b / tk, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
             "sample": f"first {k} chunk(s) ({k * w.b} tokens) of one sequence of {w.name}, numpy {prec} "
                       f"BLAS, {tk:.1f} s"}
+
+
+def cpu_baseline_predict(w: I.Workload, rows: int = 512) -> dict:
+    """Oracle tokens/s of the final prediction on a bounded sample: the first
+    `rows` tokens of one sequence."""
+    import oracle  # test infrastructure: the CPU baseline only
+    ws = w.with_(T=rows, b=rows, batch=1)
+    x = I.make_inputs(ws, seed=0)
+    dtype = np.float64 if w.precision == "fp32" else np.float32
+    model = oracle.make_model(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.rms_eps, x["lm_head"], x["rms_gain"],
+                              x["static_w"], dtype=dtype)
+    t0 = time.perf_counter()
+    oracle.final_prediction(model, x["W0"], x["hidden"], x["tokens"], rows, dtype=dtype)
+    dt = time.perf_counter() - t0
+    prec = "float64" if w.precision == "fp32" else "float32"
+    return {"value": rows / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"final prediction of the first {rows} tokens of one sequence of {w.name}, numpy {prec} "
+                      f"BLAS, {dt:.1f} s"}
 
 
 def run_reference(args, w: I.Workload):
@@ -567,6 +592,120 @@ def run_ours_recon(args, w: I.Workload):
     return 0
 
 
+def run_ours_predict(args, w: I.Workload):
+    """Forward-only final prediction at fixed fast weights (ttt_predict) over
+    the whole sequence, args.predict_rows rows per sequence per pass; the same
+    timing rules as the inner loop, the roofline over the whole step."""
+    import torch
+    from weight_long_context_b200 import ttt
+
+    rank, world, local = dist_env()
+    if world > 1:
+        init_dist("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    st = torch.cuda.current_stream(dev)
+    rows = args.predict_rows
+    if w.T % rows:
+        raise SystemExit(f"--predict-rows must divide T = {w.T}")
+    x = I.make_inputs(w, seed=rank)
+    T = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
+    h = ttt.Handle(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.has_static, w.precision, T(x["lm_head"]),
+                   T(x["rms_gain"]), T(x["static_w"]) if x["static_w"] is not None else None, w.rms_eps,
+                   w.reduction, w.update_rule)
+    hidden, tokens, W = T(x["hidden"]), T(x["tokens"], torch.int32), T(x["W0"])
+    grp = torch.empty((w.batch, w.T // rows), dtype=torch.float32, device=dev)
+    flush = None
+    if input_bytes(w) + state_bytes(w) <= 2 * L2_BYTES:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        return h.predict(hidden, tokens, W, rows, group_loss=grp, stream=st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert h.device_status() == 0, "device status after warm-up"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    if rank == 0:
+        clocks.start()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        ev[i][0].record(st)
+        step()
+        ev[i][1].record(st)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    status = h.device_status()
+    mean_ms = reduce_max(statistics.mean(step_ms), dev)
+    tokens_per_step = w.batch * w.T
+    value = whole_job_rate(tokens_per_step, world, mean_ms / 1e3)
+    pk = peaks()
+    # kernels per step in ttt_predict's launch sequence: the operand shadow of
+    # W, then per pass the gather, two GEMMs per MLP, the RMSNorm, the logits
+    # GEMM, the cross-entropy row reduction and the group mean
+    n_mlp = w.n_blocks * (2 if w.has_static else 1)
+    launches = 1 + (w.T // rows) * (5 + 2 * n_mlp)
+
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    hx = [pin(x["hidden"]), pin(x["tokens"].astype(np.int32)), pin(x["W0"])]
+    h2d = sum(t.numel() * t.element_size() for t in hx)
+    d2h = grp.numel() * 4
+    del hidden, tokens, W
+    torch.cuda.empty_cache()
+    h.predict_host(*hx, b=rows, stream=st)
+    e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e_steps):
+        h.predict_host(*hx, b=rows, stream=st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / e_steps, dev)
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        tflops = value * predict_flops_per_token(w) / 1e12
+        cfg = workload_config(w)
+        cfg.update(workload=w.name + " final prediction", rows_per_pass=rows,
+                   pass_kind="forward only at fixed fast weights (no backward, no update)")
+        line = {"metric": "final-prediction tokens/sec at 1 B200 (forward only at W_T)", "value": value,
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.precision == "bf16" else "f32", "data": "synthetic", "config": cfg,
+                "algorithmic_tflops": tflops, "clocks": clk,
+                "e2e": {"value": whole_job_rate(tokens_per_step, world, e2e_ms / 1e3), "unit": UNIT,
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                        "steps": e_steps},
+                "gpu_launches": launches * args.steps,
+                "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": pk["tflops_sustained"],
+                             "unit": "TFLOP/s", "frac": tflops / world / pk["tflops_sustained"], "traffic": None,
+                             "kernel": "whole step (forward GEMMs and the logits GEMM dominate)",
+                             "peak_source": f"{pk['source']} (bf16 sustained)"},
+                "device_status": status}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_predict(w)
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,6 +722,11 @@ def main(argv=None):
     ap.add_argument("--chunks", type=int, default=0,
                     help="profiling captures only: run the first N chunks of each sequence instead of the full T "
                          "(every launch keeps its full-size shape; the line's config names the reduced T)")
+    ap.add_argument("--final-prediction", action="store_true",
+                    help="time the forward-only final prediction at fixed fast weights (ttt_predict) instead of "
+                         "the inner loop")
+    ap.add_argument("--predict-rows", type=int, default=8192,
+                    help="rows per sequence in one pass of the final prediction")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -593,6 +737,10 @@ def main(argv=None):
         w = w.with_(update_rule=args.update_rule)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.final_prediction:
+        if w.head != "lm":
+            ap.error("--final-prediction needs a next-token workload")
+        return run_ours_predict(args, w)
     return run_ours(args, w)
 
 

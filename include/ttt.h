@@ -214,6 +214,29 @@ ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
                              const float* gamma, float* O, float* chunk_loss, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Final prediction at fixed fast weights ([TTT-E2E] 持续学习框架, the 预测
+ * step: after the inner loop the weights W_T hold the context, and the
+ * sequence is scored again with them; the page's inner-loop sketch ends with
+ * this forward-only pass).  The forward of ttt_prefill (blocks, frozen
+ * RMSNorm, LM head, next-token loss) at W, with no backward and no update:
+ *   hidden [batch, T, d]  device float32, 16-byte aligned
+ *   tokens [batch, T]     device int32 labels in [0, vocab), as in ttt_prefill
+ *   W      [batch, n_blocks, m, h, d]  device float32 fast weights (read
+ *                         only), ttt_prefill's layout; 16-byte aligned
+ *   group_loss [batch, T/b]  device float32 out: the mean loss of each run of
+ *                         b consecutive positions (the loss-by-position curve;
+ *                         the mean of all of them is the final loss)
+ *   token_loss [batch, T]    device float32 out, or NULL: every token's loss
+ *   workspace  at least ttt_workspace_size(h, batch, T, b) bytes, 256-byte aligned
+ * b is only the number of rows per sequence in one pass (any divisor of T;
+ * a larger b gives larger GEMMs and needs a larger workspace).  Token range
+ * errors and non-finite group losses are recorded in the device status word,
+ * as in ttt_prefill.  Captured into a CUDA graph per distinct call, like
+ * ttt_prefill.  A reconstruction-head handle is TTT_ERR_UNSUPPORTED. */
+ttt_status ttt_predict(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                       const int32_t* tokens, const float* W, float* group_loss, float* token_loss,
+                       void* workspace, size_t ws_bytes, void* stream);
+
 /* The per-token and per-chunk coefficients of a chunk update rule for every
  * chunk, on the device.  rule = TTT_RULE_E2TTT: the scalar kernels of
  * Proposition 3.1 ([E2-TTT] 定义高效后缀乘积与比例和, 命题3.1; computed in the

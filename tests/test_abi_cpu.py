@@ -93,3 +93,8 @@ def test_recon_head_config_validation(lib):
 def test_prefill_rejects_null_handle(lib):
     n = ctypes.c_size_t()
     assert lib.ttt_workspace_size(None, 1, 8, 4, ctypes.byref(n)) == 1
+
+
+def test_predict_rejects_null_handle(lib):
+    assert lib.ttt_predict(None, 1, 8, 4, *([None] * 5), None, 0, None) == 1
+    assert b"NULL" in lib.ttt_last_error()

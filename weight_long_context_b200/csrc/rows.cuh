@@ -126,11 +126,13 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dz, const float* __
 
 // ---------------------------------------------------------------------------
 // Cross-entropy reduction, one warp per row: combine the row's online-softmax
-// partials (max, sum exp) into lse and form l_t = lse - logit[y_t].
+// partials (max, sum exp) into lse and form l_t = lse - logit[y_t]; with
+// tok_out also store l_t at the token's [B, T] position.
 // ---------------------------------------------------------------------------
 __global__ void ce_rows_kernel(const float* __restrict__ part, const float* __restrict__ tgt, int ntn,
                                const int* __restrict__ tokens, TokenMap tm, int V, int64_t n,
-                               float* __restrict__ lse, float* __restrict__ ltok, int* status) {
+                               float* __restrict__ lse, float* __restrict__ ltok, int* status,
+                               float* __restrict__ tok_out = nullptr) {
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= n) return;
@@ -147,12 +149,10 @@ __global__ void ce_rows_kernel(const float* __restrict__ part, const float* __re
     float l = m + logf(sum);
     lse[r] = l;
     int y = tokens[tm.index((int)r)];
-    if (y < 0 || y >= V) {
-      record_error(status, TTT_ERR_TOKEN_RANGE);
-      ltok[r] = 0.f;
-    } else {
-      ltok[r] = l - tgt[r];
-    }
+    const float lt = (y < 0 || y >= V) ? 0.f : l - tgt[r];
+    if (y < 0 || y >= V) record_error(status, TTT_ERR_TOKEN_RANGE);
+    ltok[r] = lt;
+    if (tok_out) tok_out[tm.index((int)r)] = lt;
   }
 }
 

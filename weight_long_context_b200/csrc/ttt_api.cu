@@ -11,13 +11,17 @@
 //   RMSNorm backward -> per MLP, top down: B1 (dA, dU), B2 (dX) when a
 //   dynamic MLP lies below, and for dynamic MLPs the dual-accumulator
 //   aggregation whose epilogue writes W, M and the operand shadow in place.
-// The whole sequence of launches is captured once into a CUDA graph on a
-// private stream and replayed on the caller's stream.
+// The final prediction (ttt_predict) runs the same forward and CE pass A at
+// fixed weights, with no backward.  The whole sequence of launches of a call
+// is captured once into a CUDA graph on a private stream and replayed on the
+// caller's stream.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cmath>
+#include <iterator>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -54,31 +58,28 @@ using bf16 = __nv_bfloat16;
 // ---------------------------------------------------------------------------
 // Handle
 // ---------------------------------------------------------------------------
-struct GraphKey {
-  int batch, T, b;
-  const void *hidden, *tokens, *W, *M, *eta, *beta, *gamma, *loss, *ws;
-  size_t ws_bytes;
-  bool operator==(const GraphKey& o) const {
-    return batch == o.batch && T == o.T && b == o.b && hidden == o.hidden && tokens == o.tokens &&
-           W == o.W && M == o.M && eta == o.eta && beta == o.beta && gamma == o.gamma &&
-           loss == o.loss && ws == o.ws && ws_bytes == o.ws_bytes;
+// Pointers and sizes a captured graph was built for: a graph is replayed only
+// for exactly the call it was captured from.
+struct CallKey {
+  int batch = 0, T = 0, b = 0;
+  const void* ptr[16] = {};
+  size_t ws_bytes = 0;
+  bool operator==(const CallKey& o) const {
+    if (batch != o.batch || T != o.T || b != o.b || ws_bytes != o.ws_bytes) return false;
+    for (int i = 0; i < 16; ++i)
+      if (ptr[i] != o.ptr[i]) return false;
+    return true;
   }
 };
 
-}  // namespace ttt
-
-namespace ttt {
-// Pointers and sizes a captured reconstruction prefill graph was built for.
-struct ReconKey {
-  int batch, T, b;
-  const void *K, *V, *Q, *W, *M, *eta, *beta, *gamma, *O, *loss, *ws;
-  size_t ws_bytes;
-  bool operator==(const ReconKey& o) const {
-    return batch == o.batch && T == o.T && b == o.b && K == o.K && V == o.V && Q == o.Q && W == o.W && M == o.M &&
-           eta == o.eta && beta == o.beta && gamma == o.gamma && O == o.O && loss == o.loss && ws == o.ws &&
-           ws_bytes == o.ws_bytes;
-  }
+// One cached graph per kind of call.
+struct GraphSlot {
+  cudaGraphExec_t exec = nullptr;
+  CallKey key;
+  bool have = false;
 };
+enum { SLOT_PREFILL, SLOT_RECON, SLOT_PREDICT, N_SLOTS };
+
 }  // namespace ttt
 
 struct ttt_handle {
@@ -90,14 +91,8 @@ struct ttt_handle {
   int* status = nullptr;    // device status word
   int* zero_flag = nullptr; // a device int that stays 0 (bounded-wait self-test)
   cudaStream_t cap = nullptr;
-  cudaGraphExec_t exec = nullptr;
-  ttt::GraphKey key;
-  bool have_key = false;
+  ttt::GraphSlot graph[ttt::N_SLOTS];
   bool use_graph = true;
-  int64_t launches = 0;     // kernel launches of the last prefill
-  cudaGraphExec_t exec_recon = nullptr;   // the reconstruction head's graph
-  ttt::ReconKey rkey{};
-  bool have_rkey = false;
 };
 
 namespace ttt {
@@ -142,7 +137,7 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   // kept (bf16 path) pass B is elementwise and one dz GEMM over the whole
   // vocabulary beats two smaller ones: capped at 128 MiB.
   const size_t cap = (c.precision == TTT_PREC_BF16 ? 128ull : 32ull) << 20;
-  int64_t vs = (int64_t)(cap / ((size_t)p.n * p.esz));
+  int64_t vs = p.n > 0 ? (int64_t)(cap / ((size_t)p.n * p.esz)) : 0;   // batch 0: no rows
   vs = vs / 256 * 256;
   if (vs < 256) vs = 256;
   if (vs >= p.V) vs = p.V;
@@ -262,6 +257,86 @@ struct Prof {
   }
 };
 
+// Launch helpers of the enqueue functions below: each has `err`, `prof` and
+// `st` in scope.
+#define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
+#define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
+
+// ---------------------------------------------------------------------------
+// Forward of chunk c's rows at the operand shadow Wsh: gather, then per block
+// [static MLP], dynamic MLP, each with its residual.  With `train` the
+// launches also keep what the backward reads: the activation factors and the
+// K-scaled copies of each dynamic MLP's input.
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_forward(ttt_handle* hd, const Plan& p, const float* hidden, const T* Wsh, int c,
+                                   bool train, const float* KW, const float* KM, char* ws,
+                                   const SplitScratch& ss, cudaStream_t st, Prof& prof) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, L = p.L;
+  float* resid = reinterpret_cast<float*>(ws + p.resid);
+  T* actin = reinterpret_cast<T*>(ws + p.actin);
+  T* aw = reinterpret_cast<T*>(ws + p.aw);
+  T* am = reinterpret_cast<T*>(ws + p.am);
+  T* act = reinterpret_cast<T*>(ws + p.act);
+  T* fac = reinterpret_cast<T*>(ws + p.fac);
+  const T* S = static_cast<const T*>(hd->S);
+  int* status = hd->status;
+  cudaError_t err;
+  const double e = (double)p.esz;
+  const TokenMap tm{b, p.T, c};
+  const int64_t blk = (int64_t)p.m * h * d;          // params per block
+  const int64_t seqW = (int64_t)L * blk;             // params per sequence
+  const bool sw = p.swiglu;
+  // Forward order: per block [static], dynamic.  Lowest MLP the backward reaches:
+  const int per_blk = p.has_static ? 2 : 1;
+  const int i_min = per_blk - 1;
+  auto is_dyn = [&](int i) { return (i % per_blk) == per_blk - 1; };
+  auto blk_of = [&](int i) { return i / per_blk; };
+  {
+    const bool first_dyn = train && is_dyn(0);
+    LAUNCH(K_GATHER, 0, (8.0 + e * (first_dyn ? 3 : 1)) * n * d,
+           (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin,
+                                                        first_dyn ? aw : nullptr, first_dyn ? am : nullptr,
+                                                        KW, KM, p.kscale)));
+  }
+  for (int i = 0; i < p.nM; ++i) {
+    const bool dyn = is_dyn(i);
+    const int l = blk_of(i);
+    const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+    const T* w2 = w1 + (int64_t)H2 * d;
+    const int64_t wstride = dyn ? seqW : 0;
+    const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+    T* ain = actin + (int64_t)i * n * d;
+    T* aout = act + (int64_t)i * n * h;
+    T* fi = fac + (int64_t)i * n * H2;
+    {
+      GemmShape s{Mz, H2, d, Bz};
+      Operand A = opnd(ain, d, (int64_t)Mz * d, 1, Mz);
+      Operand Bw = opnd(w1, d, wstride, 1, H2);
+      T* fptr = (train && i >= i_min) ? fi : nullptr;
+      const double fl = 2.0 * Mz * H2 * d * Bz;
+      const double by = e * ((double)n * d + (double)H2 * d * Bz + (double)n * h + (fptr ? (double)n * H2 : 0.0));
+      if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status, ss))));
+      else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status, ss))));
+    }
+    {
+      GemmShape s{Mz, d, h, Bz};
+      Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
+      Operand Bw = opnd(w2, h, wstride, 1, d);
+      T* next = (i + 1 < p.nM) ? actin + (int64_t)(i + 1) * n * d : nullptr;
+      const bool next_dyn = train && i + 1 < p.nM && is_dyn(i + 1);
+      T* nw = next_dyn ? aw + (int64_t)(i + 1) * n * d : nullptr;
+      T* nmm = next_dyn ? am + (int64_t)(i + 1) * n * d : nullptr;
+      LAUNCH(K_MLP_DOWN, 2.0 * Mz * d * h * Bz,
+             e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0) + (nw ? 2.0 * n * d : 0.0)) +
+                 8.0 * n * d,
+             TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, nw, nmm, KW, KM, p.kscale, tm, d, Mz}, st,
+                              status, ss))));
+    }
+  }
+  return cudaSuccess;
+}
+
 // ---------------------------------------------------------------------------
 // Enqueue one prefill (all chunks) on `st`.
 // ---------------------------------------------------------------------------
@@ -305,8 +380,6 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   ss.counter_count = p.sk_counter_count;
   if (!p.sk_partial_bytes) ss = SplitScratch();
   cudaError_t err;
-#define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
-#define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
   const double e = (double)p.esz;
 
   // K1 for all chunks (depends only on the scalars).
@@ -329,50 +402,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
 
   for (int c = 0; c < p.nchunks; ++c) {
     TokenMap tm{b, p.T, c};
-    {
-      const bool first_dyn = is_dyn(0);
-      LAUNCH(K_GATHER, 0, (8.0 + e * (first_dyn ? 3 : 1)) * n * d,
-             (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin,
-                                                          first_dyn ? aw : nullptr, first_dyn ? am : nullptr,
-                                                          KW, KM, p.kscale)));
-    }
-
-    // ---- forward through the blocks ----
-    for (int i = 0; i < p.nM; ++i) {
-      const bool dyn = is_dyn(i);
-      const int l = blk_of(i);
-      const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
-      const T* w2 = w1 + (int64_t)H2 * d;
-      const int64_t wstride = dyn ? seqW : 0;
-      const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
-      T* ain = actin + (int64_t)i * n * d;
-      T* aout = act + (int64_t)i * n * h;
-      T* fi = fac + (int64_t)i * n * H2;
-      {
-        GemmShape s{Mz, H2, d, Bz};
-        Operand A = opnd(ain, d, (int64_t)Mz * d, 1, Mz);
-        Operand Bw = opnd(w1, d, wstride, 1, H2);
-        T* fptr = (i >= i_min) ? fi : nullptr;
-        const double fl = 2.0 * Mz * H2 * d * Bz;
-        const double by = e * ((double)n * d + (double)H2 * d * Bz + (double)n * h + (fptr ? (double)n * H2 : 0.0));
-        if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status, ss))));
-        else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status, ss))));
-      }
-      {
-        GemmShape s{Mz, d, h, Bz};
-        Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
-        Operand Bw = opnd(w2, h, wstride, 1, d);
-        T* next = (i + 1 < p.nM) ? actin + (int64_t)(i + 1) * n * d : nullptr;
-        const bool next_dyn = i + 1 < p.nM && is_dyn(i + 1);
-        T* nw = next_dyn ? aw + (int64_t)(i + 1) * n * d : nullptr;
-        T* nmm = next_dyn ? am + (int64_t)(i + 1) * n * d : nullptr;
-        LAUNCH(K_MLP_DOWN, 2.0 * Mz * d * h * Bz,
-               e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0) + (nw ? 2.0 * n * d : 0.0)) +
-                   8.0 * n * d,
-               TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, nw, nmm, KW, KM, p.kscale, tm, d, Mz}, st,
-                                status, ss))));
-      }
-    }
+    TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, true, KW, KM, ws, ss, st, prof));
 
     // ---- head: RMSNorm, CE pass A, reduce ----
     LAUNCH(K_RMS_FWD, 0, (4.0 + e) * n * d,
@@ -478,8 +508,6 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       }
     }
   }
-#undef LAUNCH
-#undef TRY
   return cudaSuccess;
 }
 
@@ -524,8 +552,6 @@ static cudaError_t enqueue_recon(ttt_handle* hd, const Plan& p, const float* Kin
   ss.counter_count = p.sk_counter_count;
   if (!p.sk_partial_bytes) ss = SplitScratch();
   cudaError_t err;
-#define TRY(x) do { err = (x); if (err != cudaSuccess) return err; } while (0)
-#define LAUNCH(cls, flops, bytes, expr) do { prof.begin(cls, st); expr; TRY(cudaGetLastError()); prof.end(flops, bytes, st); } while (0)
   const double e = (double)p.esz;
   if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
   LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T,
@@ -600,9 +626,99 @@ static cudaError_t enqueue_recon(ttt_handle* hd, const Plan& p, const float* Kin
              TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
     }
   }
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Final prediction ("TTT-E2E：端到端测试时训练的长上下文语言建模", 持续学习框架,
+// the 预测 step, and the final-prediction part of its inner-loop sketch): the
+// prefill's forward and CE pass A at fixed weights W, b rows per sequence at a
+// time, scored by the next-token loss.  No backward, no update.
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_predict(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
+                                   const float* W, float* group_loss, float* token_loss, char* ws,
+                                   cudaStream_t st, Prof& prof) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, V = p.V, L = p.L;
+  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+  float* resid = reinterpret_cast<float*>(ws + p.resid);
+  T* z = reinterpret_cast<T*>(ws + p.z);
+  float* rstd = reinterpret_cast<float*>(ws + p.rstd);
+  float* part = reinterpret_cast<float*>(ws + p.part);
+  float* tgt = reinterpret_cast<float*>(ws + p.tgt);
+  float* lse = reinterpret_cast<float*>(ws + p.lse);
+  float* ltok = reinterpret_cast<float*>(ws + p.ltok);
+  const T* E = static_cast<const T*>(hd->E);
+  int* status = hd->status;
+  SplitScratch ss;
+  if (p.sk_partial_bytes) {
+    ss.partial = reinterpret_cast<float*>(ws + p.sk_partial);
+    ss.partial_bytes = p.sk_partial_bytes;
+    ss.counters = reinterpret_cast<int*>(ws + p.sk_counters);
+    ss.counter_count = p.sk_counter_count;
+  }
+  cudaError_t err;
+  const double e = (double)p.esz;
+  if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
+  LAUNCH(K_SHADOW, 0, (4.0 + e) * B * L * p.m * h * d,
+         (build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0)));
+  for (int c = 0; c < p.nchunks; ++c) {
+    const TokenMap tm{b, p.T, c};
+    TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, false, nullptr, nullptr, ws, ss, st, prof));
+    LAUNCH(K_RMS_FWD, 0, (4.0 + e) * n * d,
+           (rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd)));
+    {
+      GemmShape s{n, V, d, 1};
+      Operand A = opnd(z, d, 0, 1, n);
+      Operand Be = opnd(E, d, 0, 1, V);
+      LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, nullptr, V}, st, status, ss))));
+    }
+    LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + (token_loss ? 20.0 : 16.0) * n,
+           (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status,
+                                                        token_loss)));
+    LAUNCH(K_CE_MEAN, 0, 4.0 * n, (ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, group_loss, c, p.nchunks, status)));
+  }
+  return cudaSuccess;
+}
 #undef LAUNCH
 #undef TRY
-  return cudaSuccess;
+
+// Replays the graph captured for exactly this call, capturing it first when
+// the slot holds another call's graph or none; with graphs off (TTT_GRAPH=0)
+// the launches go straight to the caller's stream.
+template <class Enqueue>
+static ttt_status run_graph(ttt_handle* h, int slot, const CallKey& key, Enqueue enqueue, cudaStream_t st) {
+  if (!h->use_graph) {
+    cudaError_t e = enqueue(st);
+    if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
+    return TTT_OK;
+  }
+  GraphSlot& g = h->graph[slot];
+  if (!(g.have && g.key == key && g.exec)) {
+    if (g.exec) { cudaGraphExecDestroy(g.exec); g.exec = nullptr; }
+    g.have = false;
+    TTT_CUDA_TRY(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+    cudaError_t e = enqueue(h->cap);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e2 = cudaStreamEndCapture(h->cap, &graph);
+    if (e != cudaSuccess || e2 != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      set_last_error("capture", cudaGetErrorString(e != cudaSuccess ? e : e2), __FILE__, __LINE__);
+      return TTT_ERR_CUDA;
+    }
+    e = cudaGraphInstantiate(&g.exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+      g.exec = nullptr;
+      set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__);
+      return TTT_ERR_CUDA;
+    }
+    g.key = key;
+    g.have = true;
+  }
+  TTT_CUDA_TRY(cudaGraphLaunch(g.exec, st));
+  return TTT_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -758,8 +874,8 @@ ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* 
 void ttt_destroy(ttt_handle* h) {
   if (!h) return;
   if (h->cap) cudaStreamSynchronize(h->cap);
-  if (h->exec) cudaGraphExecDestroy(h->exec);
-  if (h->exec_recon) cudaGraphExecDestroy(h->exec_recon);
+  for (auto& g : h->graph)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
   if (h->E) cudaFree(h->E);
   if (h->gain) cudaFree(h->gain);
   if (h->S) cudaFree(h->S);
@@ -801,34 +917,11 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
     return enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
   };
 
-  if (!h->use_graph) {
-    cudaError_t e = enqueue(st);
-    if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
-    h->launches = prof.launches;
-    return TTT_OK;
-  }
-  GraphKey key{batch, T, b, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, workspace, ws_bytes};
-  if (!(h->have_key && h->key == key && h->exec)) {
-    if (h->exec) { cudaGraphExecDestroy(h->exec); h->exec = nullptr; }
-    h->have_key = false;
-    TTT_CUDA_TRY(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = enqueue(h->cap);
-    cudaGraph_t g = nullptr;
-    cudaError_t e2 = cudaStreamEndCapture(h->cap, &g);
-    if (e != cudaSuccess || e2 != cudaSuccess) {
-      if (g) cudaGraphDestroy(g);
-      set_last_error("capture", cudaGetErrorString(e != cudaSuccess ? e : e2), __FILE__, __LINE__);
-      return TTT_ERR_CUDA;
-    }
-    e = cudaGraphInstantiate(&h->exec, g, 0);
-    cudaGraphDestroy(g);
-    if (e != cudaSuccess) { h->exec = nullptr; set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
-    h->key = key;
-    h->have_key = true;
-    h->launches = prof.launches;
-  }
-  TTT_CUDA_TRY(cudaGraphLaunch(h->exec, st));
-  return TTT_OK;
+  CallKey key;
+  key.batch = batch; key.T = T; key.b = b; key.ws_bytes = ws_bytes;
+  const void* ptrs[] = {hidden, tokens, W, M, eta, beta, gamma, chunk_loss, workspace};
+  std::copy(std::begin(ptrs), std::end(ptrs), key.ptr);
+  return run_graph(h, SLOT_PREFILL, key, enqueue, st);
 }
 
 ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* K, const float* V,
@@ -855,34 +948,39 @@ ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
       return enqueue_recon<float>(h, p, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, ws, q, prof);
     return enqueue_recon<bf16>(h, p, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, ws, q, prof);
   };
-  if (!h->use_graph) {
-    cudaError_t e = enqueue(st);
-    if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
-    h->launches = prof.launches;
-    return TTT_OK;
-  }
-  ReconKey key{batch, T, b, K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, workspace, ws_bytes};
-  if (!(h->have_rkey && h->rkey == key && h->exec_recon)) {
-    if (h->exec_recon) { cudaGraphExecDestroy(h->exec_recon); h->exec_recon = nullptr; }
-    h->have_rkey = false;
-    TTT_CUDA_TRY(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
-    cudaError_t e = enqueue(h->cap);
-    cudaGraph_t g = nullptr;
-    cudaError_t e2 = cudaStreamEndCapture(h->cap, &g);
-    if (e != cudaSuccess || e2 != cudaSuccess) {
-      if (g) cudaGraphDestroy(g);
-      set_last_error("capture", cudaGetErrorString(e != cudaSuccess ? e : e2), __FILE__, __LINE__);
-      return TTT_ERR_CUDA;
-    }
-    e = cudaGraphInstantiate(&h->exec_recon, g, 0);
-    cudaGraphDestroy(g);
-    if (e != cudaSuccess) { h->exec_recon = nullptr; set_last_error("cudaGraphInstantiate", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
-    h->rkey = key;
-    h->have_rkey = true;
-    h->launches = prof.launches;
-  }
-  TTT_CUDA_TRY(cudaGraphLaunch(h->exec_recon, st));
-  return TTT_OK;
+  CallKey key;
+  key.batch = batch; key.T = T; key.b = b; key.ws_bytes = ws_bytes;
+  const void* ptrs[] = {K, V, Q, W, M, eta, beta, gamma, O, chunk_loss, workspace};
+  std::copy(std::begin(ptrs), std::end(ptrs), key.ptr);
+  return run_graph(h, SLOT_RECON, key, enqueue, st);
+}
+
+ttt_status ttt_predict(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
+                       const int32_t* tokens, const float* W, float* group_loss, float* token_loss,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the reconstruction layer: it has no next-token prediction");
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !tokens || !W || !group_loss) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  Plan p = make_plan(h->cfg, batch, T, b);
+  if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "hidden and W must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  Prof prof;
+  auto enqueue = [&](cudaStream_t q) -> cudaError_t {
+    if (h->cfg.precision == TTT_PREC_FP32)
+      return enqueue_predict<float>(h, p, hidden, tokens, W, group_loss, token_loss, ws, q, prof);
+    return enqueue_predict<bf16>(h, p, hidden, tokens, W, group_loss, token_loss, ws, q, prof);
+  };
+  CallKey key;
+  key.batch = batch; key.T = T; key.b = b; key.ws_bytes = ws_bytes;
+  const void* ptrs[] = {hidden, tokens, W, group_loss, token_loss, workspace};
+  std::copy(std::begin(ptrs), std::end(ptrs), key.ptr);
+  return run_graph(h, SLOT_PREDICT, key, enqueue, st);
 }
 
 ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
@@ -931,7 +1029,6 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
     ++k;
   }
   *n_stats = k;
-  h->launches = prof.launches;
   return TTT_OK;
 }
 

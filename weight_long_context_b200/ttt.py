@@ -27,7 +27,7 @@ RULE = {"e2ttt": 0, "lact": 1}
 HEAD = {"lm": 0, "recon": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
-            "ttt_prefill_profiled", "ttt_prefill_recon",
+            "ttt_prefill_profiled", "ttt_prefill_recon", "ttt_predict",
             "ttt_scalar_kernels", "ttt_scalar_heads", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P]
     lib.ttt_prefill_recon.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill_recon.restype = I32
+    lib.ttt_predict.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, SZ, P]
+    lib.ttt_predict.restype = I32
     lib.ttt_prefill_noalloc.restype = I32
     lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
@@ -275,6 +277,46 @@ class Handle:
                                           _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(chunk_loss),
                                           _ptr(ws), ws.numel(), _stream_ptr(stream)), "ttt_prefill")
         return chunk_loss
+
+    def predict(self, hidden, tokens, W, b: int, token_loss: bool = False,
+                group_loss: Optional[torch.Tensor] = None, stream=None):
+        """Final prediction at fixed fast weights W (no update) on device tensors:
+        hidden [B,T,d] f32, tokens [B,T] i32, W [B*n_blocks*m*h*d] f32.  b rows
+        per sequence per pass (any divisor of T).  Returns (group_loss [B, T/b],
+        token_loss [B, T] or None) on the device."""
+        dev = self.device
+        B, T, d = hidden.shape
+        _dev(hidden, torch.float32, "hidden", dev)
+        _dev(W, torch.float32, "W", dev)
+        _dev(tokens, torch.int32, "tokens", dev)
+        nparams = B * self.cfg.n_blocks * self.n_mats * self.cfg.hidden * self.cfg.d
+        if W.numel() != nparams:
+            raise ValueError(f"W must hold {nparams} floats")
+        if tuple(tokens.shape) != (B, T):
+            raise ValueError("tokens must be [B, T]")
+        nc = T // b if b > 0 else 0
+        if group_loss is None:
+            group_loss = torch.empty((B, nc), dtype=torch.float32, device=dev)
+        tl = torch.empty((B, T), dtype=torch.float32, device=dev) if token_loss else None
+        ws = self.workspace(B, T, b)
+        _check(load_library().ttt_predict(self._h, B, T, b, _ptr(hidden), _ptr(tokens), _ptr(W),
+                                          _ptr(group_loss), _ptr(tl), _ptr(ws), ws.numel(), _stream_ptr(stream)),
+               "ttt_predict")
+        return group_loss, tl
+
+    def predict_host(self, hidden, tokens, W, b: int, stream=None):
+        """End-to-end final prediction on HOST tensors: copies hidden, tokens and
+        W in, runs, copies the group losses back.  Returns group_loss [B, T/b]
+        (host)."""
+        dev = self.device
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(st):
+            d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W)]
+            grp, _ = self.predict(*d_in, b=b, stream=st)
+            out = torch.empty(grp.shape, dtype=grp.dtype, pin_memory=True)
+            out.copy_(grp, non_blocking=True)
+        st.synchronize()
+        return out
 
     def prefill_recon(self, K, V, Q, W, M, eta, beta, gamma, b: int, O: Optional[torch.Tensor] = None,
                       chunk_loss: Optional[torch.Tensor] = None, stream=None):
