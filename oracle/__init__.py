@@ -5,6 +5,7 @@ __graft_entry__ and by the benchmark's cpu_baseline / reference leg.  The
 product path never imports it, and it imports nothing from the product.
 """
 from .ttt_oracle import *  # noqa: F401,F403
+from . import swa_oracle  # noqa: F401
 from .ttt_oracle import (Model, make_model, prefill, prefill_sequence, scalar_kernels,  # noqa: F401
                          scalar_kernels_ratio_form, chunk_update_closed, chunk_update_explicit,
                          chunk_update_lact, scalar_heads, recon_forward, recon_chunk, prefill_recon,

@@ -74,3 +74,57 @@ def recon_losses(kind, d, h, eps, W_flat, K, V):
 def recon_outputs(kind, d, h, eps, W_flat, Q):
     (mats,) = split_blocks(W_flat, 1, shapes_of(kind, d, h))
     return Q + F.layer_norm(_mlp(kind, mats, Q), (d,), eps=eps)
+
+
+# ---------------------------------------------------------------------------
+# Blocks with frozen sliding-window attention in front of the MLPs
+# ("TTT-E2E：端到端测试时训练的长上下文语言建模", the sketch's TTTE2EBlock,
+# TTTSelfAttention and RotaryEmbedding; causal window, no biases).  Written with
+# library routines where one exists: F.layer_norm, F.scaled_dot_product_attention
+# with a boolean mask, and the rotary embedding as a complex multiplication.
+# ---------------------------------------------------------------------------
+
+def rope_complex(x, pos, base=10000.0):
+    """Rotary embedding as (x_first_half + i x_second_half) * exp(i pos theta_j)."""
+    dh = x.shape[-1]
+    half = dh // 2
+    theta = torch.pow(torch.tensor(base, dtype=torch.float64),
+                      -2.0 * torch.arange(half, dtype=torch.float64) / dh)
+    ang = pos.to(torch.float64)[:, None] * theta[None, :]
+    z = torch.complex(x[..., :half], x[..., half:]) * torch.polar(torch.ones_like(ang), ang)
+    return torch.cat([z.real, z.imag], dim=-1)
+
+
+def swa_losses(kind, d, h, n_blocks, eps, E, g, static_flat, W_flat, X, y, pos0, swa, kv):
+    """Per-token losses of one chunk (rows X at positions pos0..) and the
+    chunk's rotated keys and values per block (detached).
+
+    swa: dict with n_heads, window, ln_eps and per-block lists Wq, Wk, Wv, Wo,
+    ln_gain, ln_bias; kv: per block (K [H, m, dh], V [H, m, dh], positions [m])."""
+    n = X.shape[0]
+    H = swa["n_heads"]
+    dh = d // H
+    shapes = shapes_of(kind, d, h)
+    Wb = split_blocks(W_flat, n_blocks, shapes)
+    Sb = split_blocks(static_flat, n_blocks, shapes) if static_flat is not None else None
+    pos = torch.arange(pos0, pos0 + n)
+    hcur = X
+    new_kv = []
+    for l in range(n_blocks):
+        a = F.layer_norm(hcur, (d,), swa["ln_gain"][l], swa["ln_bias"][l], swa["ln_eps"])
+        split = lambda m: (a @ m.T).reshape(n, H, dh).transpose(0, 1)
+        q = rope_complex(split(swa["Wq"][l]), pos)
+        k = rope_complex(split(swa["Wk"][l]), pos)
+        v = split(swa["Wv"][l])
+        Kp, Vp, pp = kv[l]
+        Ka, Va, kp = torch.cat([Kp, k], 1), torch.cat([Vp, v], 1), torch.cat([pp, pos])
+        delta = pos[:, None] - kp[None, :]
+        mask = (delta >= 0) & (delta < swa["window"])
+        o = F.scaled_dot_product_attention(q, Ka, Va, attn_mask=mask)
+        hcur = hcur + o.transpose(0, 1).reshape(n, d) @ swa["Wo"][l].T
+        new_kv.append((k.detach(), v.detach(), pos))
+        if Sb is not None:
+            hcur = hcur + _mlp(kind, Sb[l], hcur)
+        hcur = hcur + _mlp(kind, Wb[l], hcur)
+    z = hcur * torch.rsqrt(hcur.pow(2).mean(dim=1, keepdim=True) + eps) * g
+    return F.cross_entropy(z @ E.T, y, reduction="none"), new_kv
