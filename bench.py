@@ -68,7 +68,35 @@ def flops_per_token(w: I.Workload) -> float:
     head = 4 * d * V
     bwd = L * 2 * d * h + (L - 1) * 2 * (m - 1) * d * h + (max(n_static - 1, 0)) * 2 * m * d * h
     agg = L * 2 * m * d * h * (1 if w.scalars == "sgd" else 2)
-    return float(fwd + head + bwd + agg)
+    return float(fwd + head + bwd + agg) + attention_flops_per_token(w)
+
+
+def attention_flops_per_token(w: I.Workload) -> float:
+    """Algorithmic FLOPs per token added by frozen sliding-window attention.
+
+    Forward, every block: the q|k|v and o projections 8 d^2 and the scores and
+    P V over the keys a query sees, 4 d k_bar (k_bar = mean over positions of
+    min(window, t + 1)).  Backward, every block above the lowest, once per
+    weighted stream (two): the projections 8 d^2, dP and dQ 4 d k_bar, dK and
+    dV over the query's own chunk 4 d b_bar (b_bar = mean of min(window, i + 1)
+    over in-chunk positions i); plus the second stream through the MLPs of the
+    blocks below the top one (B1 2 d h, B2 2 (m - 1) d h where a gradient
+    continues below).
+    """
+    if not w.attn_heads:
+        return 0.0
+    d, h, L, m = w.d, w.hidden, w.n_blocks, w.n_mats
+    t = np.arange(w.T)
+    kbar = float(np.minimum(w.attn_window, t + 1).mean())
+    bbar = float(np.minimum(w.attn_window, np.arange(w.b) + 1).mean())
+    fwd = L * (8 * d * d + 4 * d * kbar)
+    bwd = (L - 1) * 2 * (8 * d * d + 4 * d * kbar + 4 * d * bbar)
+    mlp2 = 0.0
+    for l in range(L - 1):
+        mlp2 += 2 * d * h + (2 * (m - 1) * d * h if l > 0 else 0)
+        if w.has_static and l > 0:
+            mlp2 += 2 * d * h + 2 * (m - 1) * d * h
+    return float(fwd + bwd + mlp2)
 
 
 def predict_flops_per_token(w: I.Workload) -> float:
@@ -236,6 +264,14 @@ def oracle_chunks(w: I.Workload, n_chunks: int, seed: int = 0):
     x = I.make_inputs(ws, seed=seed)
     model = oracle.make_model(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.rms_eps, x["lm_head"], x["rms_gain"],
                               x["static_w"], dtype=dtype)
+    if w.attn_heads:
+        a = I.make_swa_inputs(ws, seed=seed)
+        sw = oracle.swa_oracle.make_swa(w.d, w.n_blocks, w.attn_heads, w.attn_window, a["attn_w"], a["ln_gain"],
+                                        a["ln_bias"])
+        t0 = time.perf_counter()
+        oracle.swa_oracle.prefill(model, sw, x["W0"], x["M0"], x["hidden"], x["tokens"], x["eta"], x["beta"],
+                                  x["gamma"], w.b, dtype=dtype, rule=w.update_rule, reduction=w.reduction)
+        return time.perf_counter() - t0
     t0 = time.perf_counter()
     oracle.prefill(model, x["W0"], x["M0"], x["hidden"], x["tokens"], x["eta"], x["beta"], x["gamma"], w.b,
                    dtype=dtype, reduction=w.reduction, update="lact" if w.update_rule == "lact" else "closed")
@@ -314,6 +350,9 @@ def workload_config(w: I.Workload) -> dict:
             "scalars": w.scalars, "loss_reduction": w.reduction, "update_rule": w.update_rule,
             "head": "next-token cross-entropy" if w.head == "lm" else "key/value reconstruction (E2-TTT layer)",
             "precision": "fp32" if w.precision == "fp32" else "bf16 GEMM operands, fp32 accumulate/state",
+            **({"attention": {"heads": w.attn_heads, "window": w.attn_window,
+                              "kind": "frozen causal sliding-window, rotary, LayerNorm in front"}}
+               if w.attn_heads else {}),
             "l2": ("inputs larger than L2 (hidden + fast-weight state %.2f GiB per step)" % ((input_bytes(w) + state_bytes(w)) / 2 ** 30))
                   if big else "L2 flushed between timed steps (write of a 256 MiB buffer)"}
 
@@ -340,6 +379,9 @@ def run_ours(args, w: I.Workload):
     h = ttt.Handle(w.d, w.hidden, w.vocab, w.n_blocks, w.mlp, w.has_static, w.precision, T(x["lm_head"]),
                    T(x["rms_gain"]), T(x["static_w"]) if x["static_w"] is not None else None, w.rms_eps,
                    w.reduction, w.update_rule)
+    if w.attn_heads:
+        a = I.make_swa_inputs(w, seed=rank)
+        h.set_attention(w.attn_heads, w.attn_window, T(a["attn_w"]), T(a["ln_gain"]), T(a["ln_bias"]))
     hidden, tokens = T(x["hidden"]), T(x["tokens"], torch.int32)
     W, M = T(x["W0"]), T(x["M0"])
     eta, beta, gamma = T(x["eta"]), T(x["beta"]), T(x["gamma"])
@@ -711,7 +753,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOAD_ORDER + ["e2ttt_layer_128k"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=I.WORKLOAD_ORDER + ["e2ttt_layer_128k", "stack_128k_swa"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scalar-heads", action="store_true",

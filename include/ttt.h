@@ -214,6 +214,33 @@ ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
                              const float* gamma, float* O, float* chunk_loss, void* workspace, size_t ws_bytes,
                              void* stream);
 
+/* Frozen sliding-window attention in front of every updated block ([TTT-E2E]
+ * the sketch's TTTE2EBlock and TTTSelfAttention; 滑动窗口注意力, window k = 8K
+ * and chunk b = 1K with k >= b in 关键设计参数).  After this call ttt_prefill
+ * runs each block as h <- h + Attn(LN(h)), then the static and dynamic MLPs:
+ *   LN(h) = (h - mean) / sqrt(var + ln_eps) * ln_gain + ln_bias
+ *   q, k, v = LN(h) Wq^T, Wk^T, Wv^T split into n_heads heads of d / n_heads;
+ *   q and k rotated by the rotary embedding (rotate-half form, angle
+ *   pos * 10000^(-2i/d_head) at the token's position in the sequence);
+ *   softmax(q.k / sqrt(d_head)) over the keys at positions j with
+ *   0 <= pos - j < window (causal; earlier chunks' keys and values inside the
+ *   window included, as computed when their chunk ran); output o Wo^T.
+ * With attention a token's loss depends on earlier tokens' rows, so the
+ * update below the top block's attention is formed from the gradients of the
+ * K_W- and K_M-weighted chunk losses (sum_t K_t G_t = grad of sum_t K_t l_t).
+ *   attn_w  [n_blocks, 4, d, d]  device float32: Wq, Wk, Wv, Wo of each block
+ *                                (copied, in the handle's operand precision)
+ *   ln_gain, ln_bias [n_blocks, d]  device float32, 16-byte aligned (copied)
+ * n_heads = 0 removes the attention.  d % n_heads == 0 and d / n_heads a
+ * multiple of 16 (TTT_ERR_SHAPE), window >= 1 and ln_eps > 0
+ * (TTT_ERR_INVALID_ARG); the handle's head must be TTT_HEAD_LM
+ * (TTT_ERR_UNSUPPORTED).  With attention, ttt_prefill needs b % 8 == 0 and a
+ * workspace that holds the keys and values of the whole sequence
+ * (ttt_workspace_size reports it); ttt_predict is TTT_ERR_UNSUPPORTED.
+ * Synchronous. */
+ttt_status ttt_set_attention(ttt_handle* h, int32_t n_heads, int32_t window, const float* attn_w,
+                             const float* ln_gain, const float* ln_bias, float ln_eps);
+
 /* Final prediction at fixed fast weights ([TTT-E2E] 持续学习框架, the 预测
  * step: after the inner loop the weights W_T hold the context, and the
  * sequence is scored again with them; the page's inner-loop sketch ends with

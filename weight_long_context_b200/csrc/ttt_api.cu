@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "epilogue.cuh"
+#include "attention.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "rows.cuh"
@@ -93,6 +94,15 @@ struct ttt_handle {
   cudaStream_t cap = nullptr;
   ttt::GraphSlot graph[ttt::N_SLOTS];
   bool use_graph = true;
+  // Frozen sliding-window attention in front of every updated block
+  // (ttt_set_attention); attn_heads == 0: none.
+  int attn_heads = 0;
+  int attn_window = 0;
+  float attn_ln_eps = 1e-5f;
+  void* Wqkv = nullptr;       // [n_blocks][3d][d] operand copy (rows q | k | v)
+  void* Wo = nullptr;         // [n_blocks][d][d] operand copy
+  float* ln_gain = nullptr;   // [n_blocks][d]
+  float* ln_bias = nullptr;   // [n_blocks][d]
 };
 
 namespace ttt {
@@ -110,6 +120,10 @@ struct Plan {
   bool recon;           // reconstruction head: no LM-head buffers; yk, yq, qres below
   size_t yk, yq, qres;  // fp32 [n, d]: MLP outputs on the keys and queries, the query rows
   size_t sk_partial_bytes, sk_counter_count;
+  // frozen sliding-window attention (attn_heads > 0)
+  int H, dh, window, ldS;
+  size_t rope_tab, xhat, lnr, qkv, qh, kh, vh, S, Pa, Of, Oc, dOh, dSa, dq, dk, dv, dqkv, da, sdout[2], sdoutT[2][2],
+      sdU[2];
 };
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -121,7 +135,8 @@ static int head_parts(int precision, int V) {
   return (V + tc::HEAD_BN - 1) / tc::HEAD_BN * tc::EPI_PARTS;
 }
 
-static Plan make_plan(const ttt_config& c, int B, int T, int b) {
+static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
+  const ttt_config& c = hd->cfg;
   Plan p{};
   p.B = B; p.T = T; p.b = b; p.nchunks = b > 0 ? T / b : 0; p.n = B * b;
   p.recon = c.head == TTT_HEAD_RECON;
@@ -180,6 +195,42 @@ static Plan make_plan(const ttt_config& c, int B, int T, int b) {
   p.sk_counter_count = p.sk_partial_bytes ? 65536 : 0;
   p.sk_partial = take(p.sk_partial_bytes);
   p.sk_counters = take(4 * p.sk_counter_count);
+  // Attention: a query of chunk c sees keys from j0 = c*b - window + 1 rounded
+  // down to a multiple of 8 (16-byte aligned operand rows) up to the chunk's
+  // end, so at most b + window + 6 keys; the key/value history spans the
+  // whole sequence.
+  p.H = hd->attn_heads;
+  if (p.H > 0) {
+    p.window = hd->attn_window;
+    p.dh = p.d / p.H;
+    int64_t ks = std::min<int64_t>((int64_t)T, (int64_t)b + p.window + 6);
+    p.ldS = (int)align_up((size_t)ks, 8);
+    const size_t H = p.H, L = p.L, ldS = p.ldS;
+    p.rope_tab = take(8ull * T * (p.dh / 2));
+    p.xhat = take(4 * L * n * d);
+    p.lnr = take(4 * L * n);
+    p.qkv = take(4 * n * 3 * d);
+    p.qh = take(e * L * n * d);
+    p.kh = take(e * L * B * T * d);
+    p.vh = take(e * L * B * T * d);
+    p.S = take(4 * H * b * ldS);
+    p.Pa = take(e * L * B * H * b * ldS);
+    p.Of = take(4 * L * n * d);
+    p.Oc = take(e * n * d);
+    p.dOh = take(e * n * d);
+    p.dSa = take(e * H * b * ldS);
+    p.dq = take(4 * n * d);
+    p.dk = take(4 * n * d);
+    p.dv = take(4 * n * d);
+    p.dqkv = take(e * n * 3 * d);
+    p.da = take(4 * n * d);
+    for (int i = 0; i < 2; ++i) {
+      p.sdout[i] = take(4 * n * d);
+      p.sdoutT[i][0] = take(e * n * d);
+      p.sdoutT[i][1] = take(e * n * d);
+      p.sdU[i] = take(e * n * H2);
+    }
+  }
   p.total = off;
   return p;
 }
@@ -224,11 +275,13 @@ static Operand opnd(const void* p, int64_t ld, int64_t bs, int kmajor, int64_t r
 // ---------------------------------------------------------------------------
 enum KernelClass {
   K_SCAN, K_SHADOW, K_GATHER, K_MLP_UP, K_MLP_DOWN, K_RMS_FWD, K_CE_LSE, K_CE_ROWS, K_CE_MEAN,
-  K_CE_GRAD, K_CE_DZ, K_RMS_BWD, K_BWD_DA, K_BWD_DX, K_AGG_UPDATE, K_RECON_ROWS, K_NCLASS
+  K_CE_GRAD, K_CE_DZ, K_RMS_BWD, K_BWD_DA, K_BWD_DX, K_AGG_UPDATE, K_RECON_ROWS, K_ATTN_PROJ, K_ATTN_SCORE,
+  K_ATTN_ROWS, K_NCLASS
 };
 static const char* kClassName[K_NCLASS] = {
     "scalar_scan", "w_shadow", "gather", "mlp_up", "mlp_down", "rmsnorm_fwd", "ce_logits_lse", "ce_rows",
-    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update", "recon_rows"};
+    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update", "recon_rows",
+    "attn_proj", "attn_scores", "attn_rows"};
 
 struct Prof {
   bool timing = false;
@@ -338,24 +391,18 @@ static cudaError_t enqueue_forward(ttt_handle* hd, const Plan& p, const float* h
 }
 
 // ---------------------------------------------------------------------------
-// Enqueue one prefill (all chunks) on `st`.
+// Head of chunk c: RMSNorm, CE pass A (logit tiles -> online-softmax
+// partials), the per-token and chunk losses, CE pass B and dz per vocabulary
+// slab, RMSNorm backward.  Leaves the residual-stream gradient in dout (fp32),
+// its operand copy in dout_a and the K-scaled copies for the top MLP in
+// doutW / doutM [(nM - 1) & 1].
 // ---------------------------------------------------------------------------
 template <typename T>
-static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
-                                   float* W, float* M, const float* eta, const float* beta,
-                                   const float* gamma, float* chunk_loss, char* ws, cudaStream_t st,
-                                   Prof& prof) {
-  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, V = p.V, L = p.L;
-  float* KW = reinterpret_cast<float*>(ws + p.KW);
-  float* KM = reinterpret_cast<float*>(ws + p.KM);
-  float* consts = reinterpret_cast<float*>(ws + p.consts);
-  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens, float* chunk_loss, int c,
+                                const float* KW, const float* KM, char* ws, const SplitScratch& ss,
+                                cudaStream_t st, Prof& prof) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, V = p.V;
   float* resid = reinterpret_cast<float*>(ws + p.resid);
-  T* actin = reinterpret_cast<T*>(ws + p.actin);
-  T* aw = reinterpret_cast<T*>(ws + p.aw);
-  T* am = reinterpret_cast<T*>(ws + p.am);
-  T* act = reinterpret_cast<T*>(ws + p.act);
-  T* fac = reinterpret_cast<T*>(ws + p.fac);
   T* z = reinterpret_cast<T*>(ws + p.z);
   float* rstd = reinterpret_cast<float*>(ws + p.rstd);
   float* part = reinterpret_cast<float*>(ws + p.part);
@@ -369,8 +416,78 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
   T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
   T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
-  T* dU = reinterpret_cast<T*>(ws + p.dU);
   const T* E = static_cast<const T*>(hd->E);
+  int* status = hd->status;
+  cudaError_t err;
+  const double e = (double)p.esz;
+  const TokenMap tm{b, p.T, c};
+  LAUNCH(K_RMS_FWD, 0, (4.0 + e) * n * d,
+         (rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd)));
+  {
+    GemmShape s{n, V, d, 1};
+    Operand A = opnd(z, d, 0, 1, n);
+    Operand Be = opnd(E, d, 0, 1, V);
+    LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
+           TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, logits, V}, st, status, ss))));
+  }
+  LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
+         (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
+  LAUNCH(K_CE_MEAN, 0, 4.0 * n, (ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status)));
+  // ---- CE pass B and dz, one vocabulary slab at a time ----
+  for (int sl = 0; sl < p.nslabs; ++sl) {
+    const int v0 = sl * p.Vs;
+    const int vs = V - v0 < p.Vs ? V - v0 : p.Vs;
+    if (logits) {   // softmax - onehot from the kept logits
+      const int64_t work = (int64_t)n * ((vs + 7) / 8);
+      LAUNCH(K_CE_GRAD, 0, (4.0 + e) * n * vs,
+             (ce_dlogits_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(logits, V, lse, tokens, tm, P,
+                                                                                  p.Vs, v0, vs, n)));
+    } else {        // fp32 path: recompute the slab's logits
+      GemmShape s{n, vs, d, 1};
+      Operand A = opnd(z, d, 0, 1, n);
+      Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
+      LAUNCH(K_CE_GRAD, 2.0 * n * vs * d, e * ((double)n * d + (double)vs * d + (double)n * vs),
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status, ss))));
+    }
+    {
+      GemmShape s{n, d, vs, 1};
+      Operand A = opnd(P, p.Vs, 0, 1, n);
+      Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 0, vs);
+      LAUNCH(K_CE_DZ, 2.0 * n * d * vs, e * ((double)n * vs + (double)vs * d) + (sl > 0 ? 8.0 : 4.0) * n * d,
+             TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status, ss))));
+    }
+  }
+  {
+    const int top = p.nM - 1;  // always dynamic
+    LAUNCH(K_RMS_BWD, 0, (12.0 + 3.0 * e) * n * d,
+           (rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
+                                                               doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm)));
+  }
+  return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Enqueue one prefill (all chunks) on `st`.
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
+                                   float* W, float* M, const float* eta, const float* beta,
+                                   const float* gamma, float* chunk_loss, char* ws, cudaStream_t st,
+                                   Prof& prof) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, L = p.L;
+  float* KW = reinterpret_cast<float*>(ws + p.KW);
+  float* KM = reinterpret_cast<float*>(ws + p.KM);
+  float* consts = reinterpret_cast<float*>(ws + p.consts);
+  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+  T* aw = reinterpret_cast<T*>(ws + p.aw);
+  T* am = reinterpret_cast<T*>(ws + p.am);
+  T* act = reinterpret_cast<T*>(ws + p.act);
+  T* fac = reinterpret_cast<T*>(ws + p.fac);
+  float* dout = reinterpret_cast<float*>(ws + p.dout);
+  T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
+  T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
+  T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
+  T* dU = reinterpret_cast<T*>(ws + p.dU);
   const T* S = static_cast<const T*>(hd->S);
   int* status = hd->status;
   SplitScratch ss;
@@ -404,49 +521,7 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
     TokenMap tm{b, p.T, c};
     TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, true, KW, KM, ws, ss, st, prof));
 
-    // ---- head: RMSNorm, CE pass A, reduce ----
-    LAUNCH(K_RMS_FWD, 0, (4.0 + e) * n * d,
-           (rmsnorm_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->gain, hd->cfg.rms_eps, n, d, z, rstd)));
-    {
-      GemmShape s{n, V, d, 1};
-      Operand A = opnd(z, d, 0, 1, n);
-      Operand Be = opnd(E, d, 0, 1, V);
-      LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, logits, V}, st, status, ss))));
-    }
-    LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
-           (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
-    LAUNCH(K_CE_MEAN, 0, 4.0 * n, (ce_mean_kernel<<<B, 256, 0, st>>>(ltok, b, chunk_loss, c, p.nchunks, status)));
-    // ---- CE pass B and dz, one vocabulary slab at a time ----
-    for (int sl = 0; sl < p.nslabs; ++sl) {
-      const int v0 = sl * p.Vs;
-      const int vs = V - v0 < p.Vs ? V - v0 : p.Vs;
-      if (logits) {   // softmax - onehot from the kept logits
-        const int64_t work = (int64_t)n * ((vs + 7) / 8);
-        LAUNCH(K_CE_GRAD, 0, (4.0 + e) * n * vs,
-               (ce_dlogits_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(logits, V, lse, tokens, tm, P,
-                                                                                    p.Vs, v0, vs, n)));
-      } else {        // fp32 path: recompute the slab's logits
-        GemmShape s{n, vs, d, 1};
-        Operand A = opnd(z, d, 0, 1, n);
-        Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
-        LAUNCH(K_CE_GRAD, 2.0 * n * vs * d, e * ((double)n * d + (double)vs * d + (double)n * vs),
-               TRY((gemm<T, 1>(s, A, A, Be, EpiCEGrad<T>{P, lse, tokens, tm, p.Vs, v0}, st, status, ss))));
-      }
-      {
-        GemmShape s{n, d, vs, 1};
-        Operand A = opnd(P, p.Vs, 0, 1, n);
-        Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 0, vs);
-        LAUNCH(K_CE_DZ, 2.0 * n * d * vs, e * ((double)n * vs + (double)vs * d) + (sl > 0 ? 8.0 : 4.0) * n * d,
-               TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status, ss))));
-      }
-    }
-    {
-      const int top = p.nM - 1;  // always dynamic
-      LAUNCH(K_RMS_BWD, 0, (12.0 + 3.0 * e) * n * d,
-             (rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
-                                                                 doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm)));
-    }
+    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof));
 
     // ---- backward, top down ----
     for (int i = p.nM - 1; i >= i_min; --i) {
@@ -509,6 +584,415 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
     }
   }
   return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// The inner loop with frozen sliding-window attention in front of every
+// updated block ("TTT-E2E：端到端测试时训练的长上下文语言建模": the sketch's
+// TTTE2EBlock; 滑动窗口注意力): per block h <- h + Attn(LN(h)), then the static
+// and dynamic MLPs.  A chunk's queries see the keys and values of earlier
+// chunks inside the window (kept for the whole sequence, written when their
+// chunk ran) and of their own chunk.
+//
+// The backward above the top block's attention is row-local, as without
+// attention (the top block's MLPs aggregate with K-scaled operand copies).
+// Below it attention mixes the chunk's rows, so sum_t K_t G_t is taken as the
+// gradient of the K-weighted chunk loss: two cotangent streams (K_W- and
+// K_M-weighted) run through the attention and MLP backward, and the lower
+// blocks' aggregations pair each stream's activation gradients with the
+// unscaled inputs (two A operands sharing B).
+// ---------------------------------------------------------------------------
+template <typename T>
+static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens,
+                                       float* W, float* M, const float* eta, const float* beta,
+                                       const float* gamma, float* chunk_loss, char* ws, cudaStream_t st,
+                                       Prof& prof) {
+  const int B = p.B, b = p.b, n = p.n, d = p.d, h = p.h, H2 = p.H2, L = p.L;
+  const int H = p.H, dh = p.dh, ldS = p.ldS;
+  float* KW = reinterpret_cast<float*>(ws + p.KW);
+  float* KM = reinterpret_cast<float*>(ws + p.KM);
+  float* consts = reinterpret_cast<float*>(ws + p.consts);
+  T* Wsh = reinterpret_cast<T*>(ws + p.Wsh);
+  float* resid = reinterpret_cast<float*>(ws + p.resid);
+  T* actin = reinterpret_cast<T*>(ws + p.actin);
+  T* aw = reinterpret_cast<T*>(ws + p.aw);
+  T* am = reinterpret_cast<T*>(ws + p.am);
+  T* act = reinterpret_cast<T*>(ws + p.act);
+  T* fac = reinterpret_cast<T*>(ws + p.fac);
+  T* zT = reinterpret_cast<T*>(ws + p.z);            // LayerNorm output (the head reuses it later)
+  float* dout = reinterpret_cast<float*>(ws + p.dout);
+  T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
+  T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
+  T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
+  T* dU = reinterpret_cast<T*>(ws + p.dU);
+  const float2* rtab = reinterpret_cast<const float2*>(ws + p.rope_tab);
+  float* xhat = reinterpret_cast<float*>(ws + p.xhat);
+  float* lnr = reinterpret_cast<float*>(ws + p.lnr);
+  float* qkv = reinterpret_cast<float*>(ws + p.qkv);
+  T* qh = reinterpret_cast<T*>(ws + p.qh);
+  T* kh = reinterpret_cast<T*>(ws + p.kh);
+  T* vh = reinterpret_cast<T*>(ws + p.vh);
+  float* Sc = reinterpret_cast<float*>(ws + p.S);
+  T* Pa = reinterpret_cast<T*>(ws + p.Pa);
+  float* Of = reinterpret_cast<float*>(ws + p.Of);
+  T* Oc = reinterpret_cast<T*>(ws + p.Oc);
+  T* dOh = reinterpret_cast<T*>(ws + p.dOh);
+  T* dSa = reinterpret_cast<T*>(ws + p.dSa);
+  float* dq = reinterpret_cast<float*>(ws + p.dq);
+  float* dk = reinterpret_cast<float*>(ws + p.dk);
+  float* dv = reinterpret_cast<float*>(ws + p.dv);
+  T* dqkv = reinterpret_cast<T*>(ws + p.dqkv);
+  float* da = reinterpret_cast<float*>(ws + p.da);
+  float* sdout[2] = {reinterpret_cast<float*>(ws + p.sdout[0]), reinterpret_cast<float*>(ws + p.sdout[1])};
+  T* sdoutT[2][2] = {{reinterpret_cast<T*>(ws + p.sdoutT[0][0]), reinterpret_cast<T*>(ws + p.sdoutT[0][1])},
+                     {reinterpret_cast<T*>(ws + p.sdoutT[1][0]), reinterpret_cast<T*>(ws + p.sdoutT[1][1])}};
+  T* sdU[2] = {reinterpret_cast<T*>(ws + p.sdU[0]), reinterpret_cast<T*>(ws + p.sdU[1])};
+  const T* S = static_cast<const T*>(hd->S);
+  const T* Wqkv = static_cast<const T*>(hd->Wqkv);
+  const T* Wo = static_cast<const T*>(hd->Wo);
+  int* status = hd->status;
+  SplitScratch ss;
+  if (p.sk_partial_bytes) {
+    ss.partial = reinterpret_cast<float*>(ws + p.sk_partial);
+    ss.partial_bytes = p.sk_partial_bytes;
+    ss.counters = reinterpret_cast<int*>(ws + p.sk_counters);
+    ss.counter_count = p.sk_counter_count;
+  }
+  cudaError_t err;
+  const double e = (double)p.esz;
+  const float scale = 1.0f / sqrtf((float)dh);
+  const int64_t Tn = p.T;
+
+  if (p.sk_counter_count) TRY(cudaMemsetAsync(ws + p.sk_counters, 0, 4 * p.sk_counter_count, st));
+  LAUNCH(K_SCAN, 0, 5.0 * 4 * B * p.T,
+         TRY(launch_scalar_scan(hd->cfg.update_rule, eta, beta, gamma, B, p.T, b, KW, KM, consts, st)));
+  LAUNCH(K_SHADOW, 0, (4.0 + e) * B * L * p.m * h * d,
+         (build_shadow_kernel<T><<<1184, 256, 0, st>>>(W, Wsh, (int64_t)B * L, h, d, p.swiglu ? 1 : 0)));
+  LAUNCH(K_ATTN_ROWS, 0, 8.0 * Tn * (dh / 2),
+         (rope_table_kernel<<<1184, 256, 0, st>>>(Tn, dh / 2, 10000.0, reinterpret_cast<float2*>(ws + p.rope_tab))));
+
+  const int64_t blk = (int64_t)p.m * h * d;
+  const int64_t seqW = (int64_t)L * blk;
+  const bool sw = p.swiglu;
+  const int per_blk = p.has_static ? 2 : 1;
+  const int i_min = per_blk - 1;
+  const int i_top = (L - 1) * per_blk;   // first MLP of the top block
+  auto is_dyn = [&](int i) { return (i % per_blk) == per_blk - 1; };
+  auto blk_of = [&](int i) { return i / per_blk; };
+  const int64_t hist = (int64_t)B * H * Tn * dh;   // history elements per block
+  const int64_t pblk = (int64_t)B * H * b * ldS;  // probabilities per block
+
+  for (int c = 0; c < p.nchunks; ++c) {
+    const TokenMap tm{b, p.T, c};
+    const int64_t q0 = (int64_t)c * b;
+    int64_t j0 = q0 - p.window + 1;
+    j0 = j0 < 0 ? 0 : j0 / 8 * 8;
+    const int nk = (int)(q0 + b - j0);
+    LAUNCH(K_GATHER, 0, (8.0 + e) * n * d,
+           (gather_chunk_kernel<T><<<592, 256, 0, st>>>(hidden, p.T, b, c, d, n, resid, actin, nullptr, nullptr, KW,
+                                                        KM, p.kscale)));
+    // ---- forward ----
+    for (int l = 0; l < L; ++l) {
+      const int i0 = l * per_blk;      // the block's first MLP
+      T* qb = qh + (int64_t)l * n * d;
+      T* kb = kh + l * hist;
+      T* vb = vh + l * hist;
+      float* ob = Of + (int64_t)l * n * d;
+      LAUNCH(K_ATTN_ROWS, 0, (12.0 + e) * n * d,
+             (ln_affine_fwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(resid, hd->ln_gain + (int64_t)l * d,
+                                                                   hd->ln_bias + (int64_t)l * d, hd->attn_ln_eps, n, d, zT,
+                                                                   xhat + (int64_t)l * n * d, lnr + (int64_t)l * n)));
+      {
+        GemmShape s{n, 3 * d, d, 1};
+        LAUNCH(K_ATTN_PROJ, 2.0 * n * 3 * d * d, e * ((double)n * d + 3.0 * d * d) + 12.0 * n * d,
+               TRY((gemm<T, 1>(s, opnd(zT, d, 0, 1, n), opnd(zT, d, 0, 1, n),
+                               opnd(Wqkv + (int64_t)l * 3 * d * d, d, 0, 1, 3 * d), EpiStoreF32{qkv, 3 * d, 0}, st,
+                               status, ss))));
+      }
+      LAUNCH(K_ATTN_ROWS, 0, (12.0 + 3.0 * e) * n * d,
+             (rope_split_kernel<T><<<592, 256, 0, st>>>(qkv, rtab, n, b, d, H, Tn, c, qb, kb, vb)));
+      for (int s = 0; s < B; ++s) {
+        T* qs = qb + (int64_t)s * H * b * dh;
+        T* ks = kb + (int64_t)s * H * Tn * dh + j0 * dh;
+        T* vs = vb + (int64_t)s * H * Tn * dh + j0 * dh;
+        T* ps = Pa + l * pblk + (int64_t)s * H * b * ldS;
+        {
+          GemmShape g{b, nk, dh, H};
+          LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 4.0 * H * b * nk,
+                 TRY((gemm<T, 1>(g, opnd(qs, dh, (int64_t)b * dh, 1, b), opnd(qs, dh, (int64_t)b * dh, 1, b),
+                                 opnd(ks, dh, Tn * dh, 1, nk), EpiStoreBatched{Sc, ldS, (int64_t)b * ldS}, st,
+                                 status, ss))));
+        }
+        LAUNCH(K_ATTN_ROWS, 0, (4.0 + e) * H * b * nk,
+               (attn_softmax_kernel<T><<<(H * b + 7) / 8, 256, 0, st>>>(Sc, ps, H * b, b, nk, ldS, q0, j0,
+                                                                        p.window, scale)));
+        {
+          GemmShape g{b, dh, nk, H};
+          LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b * nk + (double)nk * dh) * H + 4.0 * b * d,
+                 TRY((gemm<T, 1>(g, opnd(ps, ldS, (int64_t)b * ldS, 1, b), opnd(ps, ldS, (int64_t)b * ldS, 1, b),
+                                 opnd(vs, dh, Tn * dh, 0, nk), EpiStoreBatched{ob + (int64_t)s * b * d, d, dh}, st,
+                                 status, ss))));
+        }
+      }
+      LAUNCH(K_ATTN_ROWS, 0, (4.0 + e) * n * d,
+             (cast_kernel<T><<<592, 256, 0, st>>>(ob, Oc, (int64_t)n * d)));
+      {
+        // the output projection adds into the residual stream and writes the
+        // block's first MLP input (with its K-scaled copies when that MLP is
+        // dynamic and row-local, i.e. in the top block)
+        const bool rowloc = l == L - 1 && is_dyn(i0);
+        T* next = actin + (int64_t)i0 * n * d;
+        GemmShape s{n, d, d, 1};
+        LAUNCH(K_ATTN_PROJ, 2.0 * n * d * d, e * ((double)n * d * (rowloc ? 4 : 2) + (double)d * d) + 8.0 * n * d,
+               TRY((gemm<T, 1>(s, opnd(Oc, d, 0, 1, n), opnd(Oc, d, 0, 1, n),
+                               opnd(Wo + (int64_t)l * d * d, d, 0, 1, d),
+                               EpiResid<T>{resid, next, rowloc ? aw + (int64_t)i0 * n * d : nullptr,
+                                           rowloc ? am + (int64_t)i0 * n * d : nullptr, KW, KM, p.kscale, tm, d, n},
+                               st, status, ss))));
+      }
+      for (int i = i0; i < i0 + per_blk; ++i) {
+        const bool dyn = is_dyn(i);
+        const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+        const T* w2 = w1 + (int64_t)H2 * d;
+        const int64_t wstride = dyn ? seqW : 0;
+        const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+        T* ain = actin + (int64_t)i * n * d;
+        T* aout = act + (int64_t)i * n * h;
+        T* fptr = i >= i_min ? fac + (int64_t)i * n * H2 : nullptr;
+        {
+          GemmShape s{Mz, H2, d, Bz};
+          Operand A = opnd(ain, d, (int64_t)Mz * d, 1, Mz);
+          Operand Bw = opnd(w1, d, wstride, 1, H2);
+          const double fl = 2.0 * Mz * H2 * d * Bz;
+          const double by = e * ((double)n * d + (double)H2 * d * Bz + (double)n * h + (fptr ? (double)n * H2 : 0.0));
+          if (sw) LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, true>{aout, fptr, h, Mz}, st, status, ss))));
+          else LAUNCH(K_MLP_UP, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiF1<T, false>{aout, fptr, h, Mz}, st, status, ss))));
+        }
+        {
+          // the block's last MLP feeds the next block's LayerNorm (or the head)
+          // through the fp32 residual stream alone
+          const bool last = i == i0 + per_blk - 1;
+          T* next = last ? nullptr : actin + (int64_t)(i + 1) * n * d;
+          const bool next_rl = !last && l == L - 1 && is_dyn(i + 1);
+          T* nw = next_rl ? aw + (int64_t)(i + 1) * n * d : nullptr;
+          T* nmm = next_rl ? am + (int64_t)(i + 1) * n * d : nullptr;
+          GemmShape s{Mz, d, h, Bz};
+          Operand A = opnd(aout, h, (int64_t)Mz * h, 1, Mz);
+          Operand Bw = opnd(w2, h, wstride, 1, d);
+          LAUNCH(K_MLP_DOWN, 2.0 * Mz * d * h * Bz,
+                 e * ((double)n * h + (double)d * h * Bz + (next ? (double)n * d : 0.0) + (nw ? 2.0 * n * d : 0.0)) +
+                     8.0 * n * d,
+                 TRY((gemm<T, 1>(s, A, A, Bw, EpiResid<T>{resid, next, nw, nmm, KW, KM, p.kscale, tm, d, Mz}, st,
+                                  status, ss))));
+        }
+      }
+    }
+
+    // ---- head ----
+    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof));
+
+    // ---- backward of the top block's MLPs (row-local) ----
+    for (int i = p.nM - 1; i >= std::max(i_top, i_min); --i) {
+      const bool dyn = is_dyn(i);
+      const int l = blk_of(i);
+      const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+      const T* w2 = w1 + (int64_t)H2 * d;
+      const int64_t wstride = dyn ? seqW : 0;
+      const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+      const bool need_dx = i > i_min;
+      T* fi = fac + (int64_t)i * n * H2;
+      {
+        GemmShape s{Mz, h, d, Bz};
+        Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
+        Operand Bw = opnd(w2, h, wstride, 0, d);
+        const double fl = 2.0 * Mz * h * d * Bz;
+        const double by = e * ((double)n * d + (double)d * h * Bz + 2.0 * n * H2);
+        if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, dU, h, Mz}, st, status, ss))));
+        else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, dU, h, Mz}, st, status, ss))));
+      }
+      if (need_dx) {
+        GemmShape s{Mz, d, H2, Bz};
+        Operand A = opnd(dU, H2, (int64_t)Mz * H2, 1, Mz);
+        Operand Bw = opnd(w1, d, wstride, 0, H2);
+        const bool below_rl = i - 1 >= i_top && is_dyn(i - 1);
+        T* ow = below_rl ? doutW[(i - 1) & 1] : nullptr;
+        T* om = below_rl ? doutM[(i - 1) & 1] : nullptr;
+        LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
+               e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
+               TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status, ss))));
+      }
+      if (dyn) {
+        T* aout = act + (int64_t)i * n * h;
+        float* Wl = W + l * blk;
+        float* Ml = M + l * blk;
+        T* Sl = Wsh + l * blk;
+        {
+          GemmShape s{H2, d, b, B};
+          Operand A = opnd(dU, H2, (int64_t)b * H2, 0, b);
+          Operand B1 = opnd(aw + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+          Operand B2 = opnd(am + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+          EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+          LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B, (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
+                 TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
+        }
+        {
+          GemmShape s{d, h, b, B};
+          Operand A = opnd(doutW[i & 1], d, (int64_t)b * d, 0, b);
+          Operand A2 = opnd(doutM[i & 1], d, (int64_t)b * d, 0, b);
+          Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
+          EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
+                          consts, c, p.nchunks, h, 0};
+          LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B, (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
+                 TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+        }
+      }
+    }
+    if (L == 1) continue;   // block 0's attention reads the frozen hidden rows
+
+    // ---- the two weighted streams, through attention and the lower blocks ----
+    int cur = 0;   // sdoutT[st][cur]: operand copy of stream st's cotangent
+    LAUNCH(K_ATTN_ROWS, 0, (4.0 + 8.0 + 2.0 * e) * n * d,
+           (stream_split_kernel<T><<<592, 256, 0, st>>>(dout, KW, KM, p.kscale, tm, n, d, sdout[0], sdout[1],
+                                                        sdoutT[0][0], sdoutT[1][0])));
+    for (int l = L - 1; l >= 1; --l) {
+      T* qb = qh + (int64_t)l * n * d;
+      T* kb = kh + l * hist;
+      T* vb = vh + l * hist;
+      float* ob = Of + (int64_t)l * n * d;
+      const int64_t off = q0 - j0;   // the chunk's own keys start at this column
+      for (int sidx = 0; sidx < 2; ++sidx) {
+        {
+          GemmShape s{n, d, d, 1};
+          LAUNCH(K_ATTN_PROJ, 2.0 * n * d * d, e * (2.0 * n * d + (double)d * d),
+                 TRY((gemm<T, 1>(s, opnd(sdoutT[sidx][cur], d, 0, 1, n), opnd(sdoutT[sidx][cur], d, 0, 1, n),
+                                 opnd(Wo + (int64_t)l * d * d, d, 0, 0, d), EpiStoreHeads<T>{dOh, b, H, dh}, st,
+                                 status, ss))));
+        }
+        for (int s = 0; s < B; ++s) {
+          T* qs = qb + (int64_t)s * H * b * dh;
+          T* ks = kb + (int64_t)s * H * Tn * dh + j0 * dh;
+          T* vs = vb + (int64_t)s * H * Tn * dh + j0 * dh;
+          T* ps = Pa + l * pblk + (int64_t)s * H * b * ldS;
+          T* dos = dOh + (int64_t)s * H * b * dh;
+          {
+            GemmShape g{b, nk, dh, H};
+            LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 4.0 * H * b * nk,
+                   TRY((gemm<T, 1>(g, opnd(dos, dh, (int64_t)b * dh, 1, b), opnd(dos, dh, (int64_t)b * dh, 1, b),
+                                   opnd(vs, dh, Tn * dh, 1, nk), EpiStoreBatched{Sc, ldS, (int64_t)b * ldS}, st,
+                                   status, ss))));
+          }
+          LAUNCH(K_ATTN_ROWS, 0, (4.0 + 2.0 * e) * H * b * nk,
+                 (attn_dsoftmax_kernel<T><<<(H * b + 7) / 8, 256, 0, st>>>(Sc, ps, dos, ob + (int64_t)s * b * d, dSa,
+                                                                           H * b, b, ldS, d, dh, scale)));
+          {
+            GemmShape g{b, dh, nk, H};
+            LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b * nk + (double)nk * dh) * H + 4.0 * b * d,
+                   TRY((gemm<T, 1>(g, opnd(dSa, ldS, (int64_t)b * ldS, 1, b), opnd(dSa, ldS, (int64_t)b * ldS, 1, b),
+                                   opnd(ks, dh, Tn * dh, 0, nk), EpiStoreBatched{dq + (int64_t)s * b * d, d, dh}, st,
+                                   status, ss))));
+          }
+          {
+            GemmShape g{b, dh, b, H};
+            LAUNCH(K_ATTN_SCORE, 2.0 * b * b * dh * H, e * ((double)b * b + (double)b * dh) * H + 4.0 * b * d,
+                   TRY((gemm<T, 1>(g, opnd(dSa + off, ldS, (int64_t)b * ldS, 0, b),
+                                   opnd(dSa + off, ldS, (int64_t)b * ldS, 0, b), opnd(qs, dh, (int64_t)b * dh, 0, b),
+                                   EpiStoreBatched{dk + (int64_t)s * b * d, d, dh}, st, status, ss))));
+            LAUNCH(K_ATTN_SCORE, 2.0 * b * b * dh * H, e * ((double)b * b + (double)b * dh) * H + 4.0 * b * d,
+                   TRY((gemm<T, 1>(g, opnd(ps + off, ldS, (int64_t)b * ldS, 0, b),
+                                   opnd(ps + off, ldS, (int64_t)b * ldS, 0, b), opnd(dos, dh, (int64_t)b * dh, 0, b),
+                                   EpiStoreBatched{dv + (int64_t)s * b * d, d, dh}, st, status, ss))));
+          }
+          LAUNCH(K_ATTN_ROWS, 0, (12.0 + 3.0 * e) * b * d,
+                 (rope_bwd_pack_kernel<T><<<592, 256, 0, st>>>(dq + (int64_t)s * b * d, dk + (int64_t)s * b * d,
+                                                               dv + (int64_t)s * b * d, rtab, b, d, H, c,
+                                                               dqkv + (int64_t)s * b * 3 * d)));
+        }
+        {
+          GemmShape s{n, d, 3 * d, 1};
+          LAUNCH(K_ATTN_PROJ, 2.0 * n * d * 3 * d, e * ((double)n * 3 * d + 3.0 * d * d) + 4.0 * n * d,
+                 TRY((gemm<T, 1>(s, opnd(dqkv, 3 * d, 0, 1, n), opnd(dqkv, 3 * d, 0, 1, n),
+                                 opnd(Wqkv + (int64_t)l * 3 * d * d, d, 0, 0, 3 * d), EpiStoreF32{da, d, 0}, st,
+                                 status, ss))));
+        }
+        LAUNCH(K_ATTN_ROWS, 0, (20.0 + e) * n * d,
+               (ln_affine_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(da, xhat + (int64_t)l * n * d,
+                                                                     lnr + (int64_t)l * n, hd->ln_gain + (int64_t)l * d,
+                                                                     n, d, sdout[sidx], sdoutT[sidx][cur ^ 1])));
+      }
+      cur ^= 1;
+      // block l-1's MLPs, top down, both streams
+      for (int i = l * per_blk - 1; i >= std::max((l - 1) * per_blk, i_min); --i) {
+        const bool dyn = is_dyn(i);
+        const int lb = blk_of(i);
+        const T* w1 = dyn ? Wsh + lb * blk : S + lb * blk;
+        const T* w2 = w1 + (int64_t)H2 * d;
+        const int64_t wstride = dyn ? seqW : 0;
+        const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+        const bool need_dx = i > i_min;
+        T* fi = fac + (int64_t)i * n * H2;
+        for (int sidx = 0; sidx < 2; ++sidx) {
+          GemmShape s{Mz, h, d, Bz};
+          Operand A = opnd(sdoutT[sidx][cur], d, (int64_t)Mz * d, 1, Mz);
+          Operand Bw = opnd(w2, h, wstride, 0, d);
+          const double fl = 2.0 * Mz * h * d * Bz;
+          const double by = e * ((double)n * d + (double)d * h * Bz + 2.0 * n * H2);
+          if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, sdU[sidx], h, Mz}, st, status, ss))));
+          else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, sdU[sidx], h, Mz}, st, status, ss))));
+        }
+        if (need_dx) {
+          for (int sidx = 0; sidx < 2; ++sidx) {
+            GemmShape s{Mz, d, H2, Bz};
+            Operand A = opnd(sdU[sidx], H2, (int64_t)Mz * H2, 1, Mz);
+            Operand Bw = opnd(w1, d, wstride, 0, H2);
+            LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz, e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d) + 8.0 * n * d,
+                   TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{sdout[sidx], sdoutT[sidx][cur ^ 1], nullptr, nullptr, KW, KM,
+                                                          p.kscale, tm, d, Mz}, st, status, ss))));
+          }
+        }
+        if (dyn) {
+          T* aout = act + (int64_t)i * n * h;
+          float* Wl = W + lb * blk;
+          float* Ml = M + lb * blk;
+          T* Sl = Wsh + lb * blk;
+          {
+            // rows of W1 (and W2): sum_t dU^W_t (x) x_t and sum_t dU^M_t (x) x_t
+            GemmShape s{H2, d, b, B};
+            Operand A = opnd(sdU[0], H2, (int64_t)b * H2, 0, b);
+            Operand A2 = opnd(sdU[1], H2, (int64_t)b * H2, 0, b);
+            Operand Bx = opnd(actin + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+            EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+            LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B, (16.0 + e) * H2 * d * B + e * (2.0 * n * H2 + (double)n * d),
+                   TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+          }
+          {
+            GemmShape s{d, h, b, B};
+            Operand A = opnd(sdoutT[0][cur], d, (int64_t)b * d, 0, b);
+            Operand A2 = opnd(sdoutT[1][cur], d, (int64_t)b * d, 0, b);
+            Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
+            EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
+                            consts, c, p.nchunks, h, 0};
+            LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B, (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
+                   TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+          }
+        }
+        if (need_dx) cur ^= 1;
+      }
+    }
+  }
+  return cudaSuccess;
+}
+
+// The LM-head inner loop: with or without frozen attention in the blocks,
+// in the handle's operand precision.
+static cudaError_t enqueue_lm(ttt_handle* hd, const Plan& p, const float* hidden, const int* tokens, float* W,
+                              float* M, const float* eta, const float* beta, const float* gamma, float* chunk_loss,
+                              char* ws, cudaStream_t st, Prof& prof) {
+  const bool fp32 = hd->cfg.precision == TTT_PREC_FP32;
+  if (p.H > 0)
+    return fp32 ? enqueue_prefill_swa<float>(hd, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
+                : enqueue_prefill_swa<bf16>(hd, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
+  return fp32 ? enqueue_prefill<float>(hd, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
+              : enqueue_prefill<bf16>(hd, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
 }
 
 // ---------------------------------------------------------------------------
@@ -756,6 +1240,7 @@ static ttt_status check_shape(const ttt_handle* h, int batch, int T, int b) {
   if (T % b != 0) return fail(TTT_ERR_SHAPE, "T must be a multiple of b");
   if ((int64_t)batch * b > (1 << 24)) return fail(TTT_ERR_SHAPE, "batch * b above 2^24 tokens per step");
   if ((int64_t)batch * T > ((int64_t)1 << 31) - 1) return fail(TTT_ERR_SHAPE, "batch * T above 2^31 - 1");
+  if (h->attn_heads > 0 && b % 8) return fail(TTT_ERR_SHAPE, "with attention the chunk size b must be a multiple of 8");
   return TTT_OK;
 }
 
@@ -879,16 +1364,69 @@ void ttt_destroy(ttt_handle* h) {
   if (h->E) cudaFree(h->E);
   if (h->gain) cudaFree(h->gain);
   if (h->S) cudaFree(h->S);
+  if (h->Wqkv) cudaFree(h->Wqkv);
+  if (h->Wo) cudaFree(h->Wo);
+  if (h->ln_gain) cudaFree(h->ln_gain);
+  if (h->ln_bias) cudaFree(h->ln_bias);
   if (h->status) cudaFree(h->status);
   if (h->cap) cudaStreamDestroy(h->cap);
   delete h;
+}
+
+ttt_status ttt_set_attention(ttt_handle* h, int32_t n_heads, int32_t window, const float* attn_w,
+                             const float* ln_gain, const float* ln_bias, float ln_eps) {
+  if (!h) return fail(TTT_ERR_INVALID_ARG, "handle is NULL");
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "attention blocks need the LM head");
+  if (n_heads < 0) return fail(TTT_ERR_INVALID_ARG, "n_heads must be >= 0");
+  auto release = [&]() {
+    cudaFree(h->Wqkv); cudaFree(h->Wo); cudaFree(h->ln_gain); cudaFree(h->ln_bias);
+    h->Wqkv = h->Wo = nullptr;
+    h->ln_gain = h->ln_bias = nullptr;
+    h->attn_heads = 0;
+    for (auto& g : h->graph) g.have = false;   // captured graphs hold the old layout
+  };
+  if (n_heads == 0) { release(); return TTT_OK; }
+  const int d = h->cfg.d;
+  if (d % n_heads) return fail(TTT_ERR_SHAPE, "d must be a multiple of n_heads");
+  const int dh = d / n_heads;
+  if (dh % 16) return fail(TTT_ERR_SHAPE, "the head size d / n_heads must be a multiple of 16");
+  if (window < 1) return fail(TTT_ERR_INVALID_ARG, "window must be >= 1");
+  if (!(ln_eps > 0.f) || !std::isfinite(ln_eps)) return fail(TTT_ERR_INVALID_ARG, "ln_eps must be positive and finite");
+  if (!attn_w || !ln_gain || !ln_bias) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(ln_gain) | reinterpret_cast<uintptr_t>(ln_bias)) % 16)
+    return fail(TTT_ERR_INVALID_ARG, "ln_gain and ln_bias must be 16-byte aligned");
+  release();
+  const int64_t L = h->cfg.n_blocks, dd = (int64_t)d * d;
+  const size_t esz = h->cfg.precision == TTT_PREC_FP32 ? 4 : 2;
+  TTT_CUDA_TRY(cudaMalloc(&h->Wqkv, esz * L * 3 * dd));
+  TTT_CUDA_TRY(cudaMalloc(&h->Wo, esz * L * dd));
+  TTT_CUDA_TRY(cudaMalloc(&h->ln_gain, 4 * L * d));
+  TTT_CUDA_TRY(cudaMalloc(&h->ln_bias, 4 * L * d));
+  TTT_CUDA_TRY(cudaMemcpyAsync(h->ln_gain, ln_gain, 4 * L * d, cudaMemcpyDeviceToDevice, h->cap));
+  TTT_CUDA_TRY(cudaMemcpyAsync(h->ln_bias, ln_bias, 4 * L * d, cudaMemcpyDeviceToDevice, h->cap));
+  for (int64_t l = 0; l < L; ++l) {   // attn_w[l] = Wq, Wk, Wv, Wo: the first three are the fused q|k|v rows
+    const float* src = attn_w + l * 4 * dd;
+    if (h->cfg.precision == TTT_PREC_FP32) {
+      TTT_CUDA_TRY(cudaMemcpyAsync(static_cast<float*>(h->Wqkv) + l * 3 * dd, src, 4 * 3 * dd, cudaMemcpyDeviceToDevice, h->cap));
+      TTT_CUDA_TRY(cudaMemcpyAsync(static_cast<float*>(h->Wo) + l * dd, src + 3 * dd, 4 * dd, cudaMemcpyDeviceToDevice, h->cap));
+    } else {
+      cast_kernel<bf16><<<1184, 256, 0, h->cap>>>(src, static_cast<bf16*>(h->Wqkv) + l * 3 * dd, 3 * dd);
+      cast_kernel<bf16><<<1184, 256, 0, h->cap>>>(src + 3 * dd, static_cast<bf16*>(h->Wo) + l * dd, dd);
+      TTT_CUDA_TRY(cudaGetLastError());
+    }
+  }
+  TTT_CUDA_TRY(cudaStreamSynchronize(h->cap));
+  h->attn_heads = n_heads;
+  h->attn_window = window;
+  h->attn_ln_eps = ln_eps;
+  return TTT_OK;
 }
 
 ttt_status ttt_workspace_size(const ttt_handle* h, int32_t batch, int32_t T, int32_t b, size_t* bytes) {
   ttt_status s = check_shape(h, batch, T, b);
   if (s != TTT_OK) return s;
   if (!bytes) return fail(TTT_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = make_plan(h->cfg, batch, T, b).total;
+  *bytes = make_plan(h, batch, T, b).total;
   return TTT_OK;
 }
 
@@ -902,7 +1440,7 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  Plan p = make_plan(h->cfg, batch, T, b);
+  Plan p = make_plan(h, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
@@ -912,9 +1450,7 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
 
   Prof prof;
   auto enqueue = [&](cudaStream_t q) -> cudaError_t {
-    if (h->cfg.precision == TTT_PREC_FP32)
-      return enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
-    return enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
+    return enqueue_lm(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, q, prof);
   };
 
   CallKey key;
@@ -934,7 +1470,7 @@ ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
   if (batch == 0 || T == 0) return TTT_OK;
   if (!K || !V || !Q || !W || !M || !eta || !beta || !gamma || !O || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  Plan p = make_plan(h->cfg, batch, T, b);
+  Plan p = make_plan(h, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(Q) |
@@ -961,9 +1497,10 @@ ttt_status ttt_predict(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   ttt_status s = check_shape(h, batch, T, b);
   if (s != TTT_OK) return s;
   if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the handle's head is the reconstruction layer: it has no next-token prediction");
+  if (h->attn_heads > 0) return fail(TTT_ERR_UNSUPPORTED, "the final prediction does not run attention blocks");
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !group_loss) return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  Plan p = make_plan(h->cfg, batch, T, b);
+  Plan p = make_plan(h, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W)) % 16)
@@ -995,7 +1532,7 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
   if (batch == 0 || T == 0) return TTT_OK;
   if (!hidden || !tokens || !W || !M || !eta || !beta || !gamma || !chunk_loss)
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
-  Plan p = make_plan(h->cfg, batch, T, b);
+  Plan p = make_plan(h, batch, T, b);
   if (!workspace || ws_bytes < p.total) return fail(TTT_ERR_WORKSPACE, "workspace missing or too small");
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
@@ -1005,9 +1542,7 @@ ttt_status ttt_prefill_profiled(ttt_handle* h, int32_t batch, int32_t T, int32_t
   Prof prof;
   prof.timing = true;
   prof.recs.reserve(1 << 16);
-  cudaError_t e = h->cfg.precision == TTT_PREC_FP32
-                      ? enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
-                      : enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
+  cudaError_t e = enqueue_lm(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
   if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
   TTT_CUDA_TRY(cudaStreamSynchronize(st));
   ttt_kernel_stat agg[K_NCLASS];
@@ -1072,7 +1607,7 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
     return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
   if ((reinterpret_cast<uintptr_t>(hidden) | reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(M)) % 16)
     return fail(TTT_ERR_INVALID_ARG, "hidden, W and M must be 16-byte aligned");
-  Plan p = make_plan(h->cfg, batch, T, b);
+  Plan p = make_plan(h, batch, T, b);
   if (p.total > kNoAllocScratchBytes) {
     static thread_local char msg[160];
     snprintf(msg, sizeof(msg), "ttt_prefill_noalloc needs %zu bytes of scratch; its static scratch holds %zu bytes",
@@ -1091,9 +1626,7 @@ ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t 
   Prof prof;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(scratch);
-  cudaError_t e = h->cfg.precision == TTT_PREC_FP32
-                      ? enqueue_prefill<float>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof)
-                      : enqueue_prefill<bf16>(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
+  cudaError_t e = enqueue_lm(h, p, hidden, tokens, W, M, eta, beta, gamma, chunk_loss, ws, st, prof);
   if (e != cudaSuccess) { set_last_error("enqueue", cudaGetErrorString(e), __FILE__, __LINE__); return TTT_ERR_CUDA; }
   return TTT_OK;
 }

@@ -55,6 +55,8 @@ class Workload:
     reduction: str = "mean"  # chunk objective: mean (default) or sum of token losses
     update_rule: str = "e2ttt"  # chunk update: "e2ttt" (Proposition 3.1) or "lact" (chunk-wise rule)
     head: str = "lm"  # "lm": next-token cross-entropy; "recon": E2-TTT's key/value reconstruction layer
+    attn_heads: int = 0   # > 0: frozen sliding-window attention in front of every updated block
+    attn_window: int = 0
 
     @property
     def n_mats(self) -> int:
@@ -93,6 +95,10 @@ WORKLOADS: Dict[str, Workload] = {
     # dimensions: one SwiGLU fast-weight MLP d=2048, h=5632, T=131072, b=1024
     "e2ttt_layer_128k": Workload("e2ttt_layer_128k", 2048, 5632, 16, 1, SWIGLU, False, "bf16",
                                  131072, 1024, 1, "e2ttt", head="recon"),
+    # the 128K stack with frozen sliding-window attention in every block:
+    # 32 heads of 64, window 8192 (the pages' k = 8K with b = 1K)
+    "stack_128k_swa": Workload("stack_128k_swa", 2048, 5632, 32000, 4, SWIGLU, True, "bf16",
+                               131072, 1024, 1, "e2ttt", attn_heads=32, attn_window=8192),
 }
 WORKLOAD_ORDER = ["tiny_sgd", "e2ttt_block", "sgd_3b", "stack_128k", "batched_16"]
 
@@ -112,6 +118,19 @@ def zipf_tokens(rng: np.random.Generator, vocab: int, shape, s: float = 1.1) -> 
     u = rng.random(size=shape)
     idx = np.searchsorted(cdf, u, side="right")
     return np.minimum(idx, vocab - 1).astype(np.int32)
+
+
+def make_swa_inputs(w: Workload, seed: int = 0, scale: float = 0.02) -> Dict[str, np.ndarray]:
+    """Frozen attention parameters of every updated block, drawn from their own
+    generator (seed, 2): attn_w [n_blocks, 4, d, d] (Wq, Wk, Wv, Wo) ~
+    N(0, scale^2), LayerNorm gain ~ U(0.8, 1.2) and bias ~ N(0, 0.1^2)
+    [n_blocks, d]."""
+    rng = np.random.default_rng([seed, 2])
+    L, d = w.n_blocks, w.d
+    attn_w = _normal(rng, (L, 4, d, d), scale)
+    ln_gain = rng.uniform(0.8, 1.2, (L, d)).astype(np.float32)
+    ln_bias = _normal(rng, (L, d), 0.1)
+    return {"attn_w": attn_w, "ln_gain": ln_gain, "ln_bias": ln_bias}
 
 
 def make_recon_inputs(w: Workload, seed: int = 0, T: Optional[int] = None, batch: Optional[int] = None,

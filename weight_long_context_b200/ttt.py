@@ -27,7 +27,7 @@ RULE = {"e2ttt": 0, "lact": 1}
 HEAD = {"lm": 0, "recon": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
-            "ttt_prefill_profiled", "ttt_prefill_recon", "ttt_predict",
+            "ttt_prefill_profiled", "ttt_prefill_recon", "ttt_predict", "ttt_set_attention",
             "ttt_scalar_kernels", "ttt_scalar_heads", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
             "ttt_last_error"]
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill_recon.restype = I32
     lib.ttt_predict.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, SZ, P]
     lib.ttt_predict.restype = I32
+    lib.ttt_set_attention.argtypes = [P, I32, I32, P, P, P, ctypes.c_float]
+    lib.ttt_set_attention.restype = I32
     lib.ttt_prefill_noalloc.restype = I32
     lib.ttt_prefill_profiled.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P,
                                          ctypes.POINTER(ttt_kernel_stat), I32, ctypes.POINTER(I32)]
@@ -242,6 +244,21 @@ class Handle:
         self.n_mats = 2 if mlp == "gelu" else 3
         with torch.cuda.device(dev):
             self._h = ttt_create(self.cfg, lm_head, rms_gain, static_w)
+        self._ws = None
+
+    def set_attention(self, n_heads: int, window: int, attn_w, ln_gain, ln_bias, ln_eps: float = 1e-5):
+        """Frozen sliding-window attention in front of every updated block:
+        attn_w [n_blocks, 4, d, d] (Wq, Wk, Wv, Wo), ln_gain / ln_bias
+        [n_blocks, d], float32 CUDA tensors (copied).  n_heads = 0 removes it."""
+        if n_heads:
+            for t, nm in ((attn_w, "attn_w"), (ln_gain, "ln_gain"), (ln_bias, "ln_bias")):
+                _dev(t, torch.float32, nm, self.device)
+            L, d = self.cfg.n_blocks, self.cfg.d
+            if attn_w.numel() != L * 4 * d * d or ln_gain.numel() != L * d or ln_bias.numel() != L * d:
+                raise ValueError("attn_w must be [n_blocks, 4, d, d], ln_gain and ln_bias [n_blocks, d]")
+        with torch.cuda.device(self.device):
+            _check(load_library().ttt_set_attention(self._h, n_heads, window, _ptr(attn_w), _ptr(ln_gain),
+                                                    _ptr(ln_bias), ln_eps), "ttt_set_attention")
         self._ws = None
 
     # workspace cached per handle, grown on demand
