@@ -68,3 +68,29 @@ def test_multirank_max_and_whole_job_rate():
     # every rank sees the max over ranks; whole-job rate = units of all ranks / that time
     assert all(mx == 15.0 for _, mx, _ in res)
     assert all(rate == pytest.approx(2 * 1000.0 / 0.015) for _, _, rate in res)
+
+
+def test_predict_flops_per_token():
+    """Forward only: 8 MLPs (4 static + 4 dynamic) of 2 m d h and the logits 2 d V."""
+    w = I.WORKLOADS["stack_128k"]
+    assert bench.predict_flops_per_token(w) == 8 * 2 * 3 * w.d * w.hidden + 2 * w.d * w.vocab
+    assert bench.predict_flops_per_token(w) == pytest.approx(684.72e6, rel=1e-4)
+
+
+def test_attention_flops_per_token():
+    """No attention adds nothing; with window >= T every query sees t + 1 keys
+    (mean (T + 1) / 2), and the lower blocks' MLP backward runs a second time."""
+    w = I.WORKLOADS["stack_128k"]
+    assert bench.attention_flops_per_token(w) == 0.0
+    small = w.with_(T=64, b=16, attn_heads=2, attn_window=1 << 20, n_blocks=2, has_static=False)
+    d, h, m = small.d, small.hidden, small.n_mats
+    kbar, bbar = (64 + 1) / 2, (16 + 1) / 2
+    expect = (2 * (8 * d * d + 4 * d * kbar) + 1 * 2 * (8 * d * d + 4 * d * kbar + 4 * d * bbar)
+              + 2 * d * h)                 # block 0's dynamic MLP: B1 only (nothing dynamic below it)
+    assert bench.attention_flops_per_token(small) == pytest.approx(expect, rel=1e-12)
+    # a window of one key: each query sees only itself
+    one = small.with_(attn_window=1)
+    expect1 = 2 * (8 * d * d + 4 * d) + 2 * (8 * d * d + 4 * d + 4 * d) + 2 * d * h
+    assert bench.attention_flops_per_token(one) == pytest.approx(expect1, rel=1e-12)
+    assert bench.flops_per_token(I.WORKLOADS["stack_128k_swa"]) == pytest.approx(
+        bench.flops_per_token(w) + bench.attention_flops_per_token(I.WORKLOADS["stack_128k_swa"]))
