@@ -264,9 +264,12 @@ def rule_coefficients(rule: str, eta, beta, gamma):
 
 
 def prefill_sequence(model: Model, sw: Swa, W0, M0, hidden, tokens, eta, beta, gamma, b,
-                     rule: str = "e2ttt", reduction: str = "mean", n_chunks: Optional[int] = None):
+                     rule: str = "e2ttt", reduction: str = "mean", n_chunks: Optional[int] = None,
+                     pos0: int = 0, kv_in=None, return_kv: bool = False):
     """Chunk-serial inner loop of one sequence with attention in the blocks.
-    Returns (W, M, chunk_loss [n_chunks])."""
+    Returns (W, M, chunk_loss [n_chunks]), and the key/value history too with
+    return_kv.  To resume a sequence, pass the rows from position pos0 on, the
+    state reached there and its history as kv_in."""
     gscale = 1.0 / b if reduction == "mean" else 1.0
     T, d = hidden.shape
     if T % b:
@@ -274,11 +277,11 @@ def prefill_sequence(model: Model, sw: Swa, W0, M0, hidden, tokens, eta, beta, g
     nc = T // b if n_chunks is None else n_chunks
     W = [[m.copy() for m in blk] for blk in W0]
     M = [[m.copy() for m in blk] for blk in M0]
-    kv = [empty_kv(sw, d, hidden.dtype) for _ in range(model.n_blocks)]
+    kv = list(kv_in) if kv_in is not None else [empty_kv(sw, d, hidden.dtype) for _ in range(model.n_blocks)]
     losses = np.zeros(nc)
     for c in range(nc):
         s = slice(c * b, (c + 1) * b)
-        loss, fwd, new_kv = chunk_forward(model, sw, W, hidden[s], tokens[s], c * b, kv)
+        loss, fwd, new_kv = chunk_forward(model, sw, W, hidden[s], tokens[s], pos0 + c * b, kv)
         losses[c] = float(np.mean(loss))
         KW, KM, g0, b0, cM = rule_coefficients(rule, eta[s], beta[s], gamma[s])
         gW = weighted_backward(model, sw, W, tokens[s], fwd, KW)
@@ -293,6 +296,8 @@ def prefill_sequence(model: Model, sw: Swa, W0, M0, hidden, tokens, eta, beta, g
             K0, V0, p0 = kv[l]
             kv[l] = (np.concatenate([K0, kr], axis=1), np.concatenate([V0, v], axis=1),
                      np.concatenate([p0, p]))
+    if return_kv:
+        return W, M, losses, kv
     return W, M, losses
 
 

@@ -172,6 +172,60 @@ def test_window_one_is_the_value_path():
     np.testing.assert_allclose(out, a @ sw.Wv[0].T @ sw.Wo[0].T, rtol=1e-12, atol=1e-12)
 
 
+def test_window_covering_the_sequence_is_causal_attention():
+    """Window >= T: a chunk's rows over the earlier chunks' history give the
+    rows of plain causal attention over the whole sequence (torch SDPA with
+    is_causal on equal query and key lengths)."""
+    s = setup(d=8, H=2, window=10 ** 6)
+    sw = s["swa"]
+    rng = np.random.default_rng(11)
+    h = rng.normal(size=(12, 8))
+    pos = np.arange(12)
+    out_all, _, (kr, v, _) = S.attention_forward(sw, 0, h, pos, S.empty_kv(sw, 8))
+    _, _, hist = S.attention_forward(sw, 0, h[:8], pos[:8], S.empty_kv(sw, 8))
+    out_tail, _, _ = S.attention_forward(sw, 0, h[8:], pos[8:], hist)
+    np.testing.assert_allclose(out_tail, out_all[8:], rtol=1e-12, atol=1e-12)
+    a = F.layer_norm(torch.tensor(h), (8,), torch.tensor(sw.ln_gain[0]), torch.tensor(sw.ln_bias[0]), 1e-5)
+    split = lambda m: (a @ torch.tensor(m).T).reshape(12, 2, 4).transpose(0, 1)
+    q = AM.rope_complex(split(sw.Wq[0]), torch.tensor(pos))
+    k = AM.rope_complex(split(sw.Wk[0]), torch.tensor(pos))
+    o = F.scaled_dot_product_attention(q, k, split(sw.Wv[0]), is_causal=True)
+    ref = o.transpose(0, 1).reshape(12, 8) @ torch.tensor(sw.Wo[0]).T
+    np.testing.assert_allclose(out_all, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_common_position_shift_leaves_attention_unchanged():
+    """The rotary embedding makes scores depend on position differences only:
+    shifting the queries' and the history's positions together changes nothing."""
+    s = setup(d=8, H=2, window=6)
+    sw = s["swa"]
+    rng = np.random.default_rng(12)
+    h0, h1 = rng.normal(size=(5, 8)), rng.normal(size=(4, 8))
+    outs = []
+    for shift in (0, 1000):
+        _, _, hist = S.attention_forward(sw, 1, h0, np.arange(5) + shift, S.empty_kv(sw, 8))
+        out, _, _ = S.attention_forward(sw, 1, h1, np.arange(5, 9) + shift, hist)
+        outs.append(out)
+    np.testing.assert_allclose(outs[1], outs[0], rtol=1e-9, atol=1e-11)
+
+
+def test_resume_with_the_history():
+    """Only (W, M) and the key/value history cross chunk boundaries: two runs
+    that hand both over equal one run, bit for bit."""
+    s = setup(kind="swiglu", T=12, window=7)
+    mdl, sw = s["model"], s["swa"]
+    shapes = mdl.mat_shapes()
+    W0 = O.unpack_blocks(s["W0"].copy(), mdl.n_blocks, shapes)
+    M0 = O.unpack_blocks(s["M0"].copy(), mdl.n_blocks, shapes)
+    args = lambda sl: (s["X"][sl], s["y"][sl], s["eta"][sl], s["beta"][sl], s["gamma"][sl])
+    W, M, L = S.prefill_sequence(mdl, sw, W0, M0, *args(slice(0, 12)), 4)
+    Wa, Ma, La, kv = S.prefill_sequence(mdl, sw, W0, M0, *args(slice(0, 4)), 4, return_kv=True)
+    Wb, Mb, Lb = S.prefill_sequence(mdl, sw, Wa, Ma, *args(slice(4, 12)), 4, pos0=4, kv_in=kv)
+    assert all(np.array_equal(x, y) for bx, by in zip(Wb, W) for x, y in zip(bx, by))
+    assert all(np.array_equal(x, y) for bx, by in zip(Mb, M) for x, y in zip(bx, by))
+    np.testing.assert_array_equal(np.concatenate([La, Lb]), L)
+
+
 # ---------------------------------------------------------------------------
 # The inner loop against its definition
 # ---------------------------------------------------------------------------
