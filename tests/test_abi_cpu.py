@@ -98,3 +98,8 @@ def test_prefill_rejects_null_handle(lib):
 def test_predict_rejects_null_handle(lib):
     assert lib.ttt_predict(None, 1, 8, 4, *([None] * 5), None, 0, None) == 1
     assert b"NULL" in lib.ttt_last_error()
+
+
+def test_set_attention_rejects_null_handle(lib):
+    assert lib.ttt_set_attention(None, 4, 8, None, None, None, 1e-5) == 1
+    assert b"NULL" in lib.ttt_last_error()
