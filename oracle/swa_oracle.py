@@ -322,3 +322,32 @@ def prefill(model: Model, sw: Swa, W0_flat, M0_flat, hidden, tokens, eta, beta, 
         Ms.append(pack_blocks(M))
         Ls.append(L)
     return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls)
+
+
+def final_prediction(model: Model, sw: Swa, W_flat, hidden, tokens, b, dtype=np.float64):
+    """Forward-only pass of whole sequences at fixed fast weights with the
+    attention blocks ([TTT-E2E] 持续学习框架, the 预测 step, and the sketch's
+    最终预测 part): the rows are processed b at a time, and every key and value
+    in the window is computed at the same weights W, so the result does not
+    depend on b.  Returns (token_loss [B,T], group_loss [B, T // b]) as
+    ttt_oracle.final_prediction does."""
+    mdl = model.astype(dtype)
+    s_w = sw.astype(dtype)
+    B, T = np.asarray(tokens).shape
+    if T % b:
+        raise ValueError("T must be a multiple of b")
+    shapes = mdl.mat_shapes()
+    per_seq = mdl.n_blocks * sum(r * c for r, c in shapes)
+    Wf = np.asarray(W_flat, dtype=dtype).reshape(B, per_seq)
+    tok = np.zeros((B, T), dtype=dtype)
+    for s_ in range(B):
+        W = unpack_blocks(Wf[s_].copy(), mdl.n_blocks, shapes)
+        X = np.asarray(hidden[s_], dtype=dtype)
+        kv = [empty_kv(s_w, mdl.d, dtype) for _ in range(mdl.n_blocks)]
+        for c in range(T // b):
+            sl = slice(c * b, (c + 1) * b)
+            loss, _, new_kv = chunk_forward(mdl, s_w, W, X[sl], np.asarray(tokens[s_])[sl], c * b, kv)
+            tok[s_, sl] = loss
+            kv = [(np.concatenate([kv[l][0], new_kv[l][0]], axis=1), np.concatenate([kv[l][1], new_kv[l][1]], axis=1),
+                   np.concatenate([kv[l][2], new_kv[l][2]])) for l in range(mdl.n_blocks)]
+    return tok, tok.reshape(B, -1, b).mean(axis=2)

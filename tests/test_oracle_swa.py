@@ -296,6 +296,45 @@ def _row_local_update(s, b):
 
 
 # ---------------------------------------------------------------------------
+# Final prediction with the attention blocks
+# ---------------------------------------------------------------------------
+
+def test_final_prediction_is_one_pass_over_the_sequence():
+    """At fixed weights every key and value comes from the same W, so the
+    grouped pass equals one pass of the independent restatement over the whole
+    sequence (torch), for any group size."""
+    s = setup(kind="swiglu", T=12, window=5)
+    W = s["W0"]
+    T_ = lambda a: torch.tensor(a, dtype=torch.float64)
+    H, dh = s["H"], s["d"] // s["H"]
+    kv0 = [(torch.zeros(H, 0, dh, dtype=torch.float64), torch.zeros(H, 0, dh, dtype=torch.float64),
+            torch.zeros(0, dtype=torch.long)) for _ in range(s["L"])]
+    ref, _ = AM.swa_losses(s["kind"], s["d"], s["h"], s["L"], 1e-6, T_(s["E"]), T_(s["g"]), T_(s["static_w"]),
+                           T_(W), T_(s["X"]), torch.tensor(s["y"]), 0, torch_swa(s), kv0)
+    for b in (3, 4, 12):
+        tok, grp = S.final_prediction(s["model"], s["swa"], W, s["X"][None], s["y"][None], b)
+        np.testing.assert_allclose(tok[0], ref.numpy(), rtol=1e-11)
+        np.testing.assert_allclose(grp[0], ref.numpy().reshape(-1, b).mean(axis=1), rtol=1e-11)
+
+
+def test_final_prediction_zero_output_projection_is_the_plain_prediction():
+    s = setup(kind="gelu", T=8, window=3)
+    s["attn_w"][:, 3] = 0.0
+    sw = S.make_swa(s["d"], s["L"], s["H"], s["window"], s["attn_w"], s["ln_gain"], s["ln_bias"])
+    tok, grp = S.final_prediction(s["model"], sw, s["W0"], s["X"][None], s["y"][None], 4)
+    tok_p, grp_p = O.final_prediction(s["model"], s["W0"], s["X"][None], s["y"][None], 4)
+    np.testing.assert_allclose(tok, tok_p, rtol=1e-12)
+    np.testing.assert_allclose(grp, grp_p, rtol=1e-12)
+
+
+def test_final_prediction_first_group_is_the_first_chunk_loss():
+    s = setup(kind="swiglu", T=8, window=6)
+    _, _, Ls = run_oracle(s, 4)
+    _, grp = S.final_prediction(s["model"], s["swa"], s["W0"], s["X"][None], s["y"][None], 4)
+    assert grp[0, 0] == pytest.approx(Ls[0], rel=1e-13)
+
+
+# ---------------------------------------------------------------------------
 # Planted mistakes
 # ---------------------------------------------------------------------------
 
