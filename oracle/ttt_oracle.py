@@ -64,7 +64,7 @@ from dataclasses import dataclass
 from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
-from scipy.special import erf
+from scipy.special import erf, expit
 
 GELU = "gelu"
 SWIGLU = "swiglu"
@@ -85,7 +85,8 @@ def gelu_grad(x):
 
 
 def sigmoid(x):
-    return 1.0 / (1.0 + np.exp(-x))
+    # the logistic function from the library: no overflow of exp(-x) for large negative x
+    return expit(x)
 
 
 def silu(x):
