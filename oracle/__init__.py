@@ -11,4 +11,4 @@ from .ttt_oracle import (Model, make_model, prefill, prefill_sequence, scalar_ke
                          chunk_update_lact, scalar_heads, recon_forward, recon_chunk, prefill_recon,
                          layer_norm, layer_norm_backward, recon_shapes,
                          token_losses, token_gradients, unpack_blocks, pack_blocks,
-                         final_prediction, group_means)
+                         final_prediction, group_means, state_without_gradients)

@@ -484,6 +484,42 @@ def prefill(model: Model, W0_flat, M0_flat, hidden, tokens, eta, beta, gamma, b,
     return np.concatenate(Ws), np.concatenate(Ms), np.stack(Ls)
 
 
+def state_without_gradients(W0_flat, M0_flat, eta, beta, gamma, b, n_chunks: Optional[int] = None,
+                            update: str = "closed"):
+    """The chunk-end states the inner loop would reach if every G_t were 0.
+
+    Proposition 3.1 ([E2-TTT] 命题3.1) with the gradient sums dropped, chunk by
+    chunk: W <- gtilde_0 W + btilde_0 R_1 M, M <- btilde_0 M; under LaCT's
+    rule ([E2-TTT] 高效的逐块更新机制) M <- mean(beta) M, W <- W + M.  It is
+    elementwise, so W0_flat / M0_flat may be any subset of the flat state of
+    each sequence: arrays [B, n] (or [n] for one sequence), eta/beta/gamma
+    [B, T].  Subtracting it from a final state leaves the part the gradients
+    contributed (the update GEMMs' work), which the parity tests check on its
+    own because the decayed initial state can dominate W.  float64.
+    """
+    W = np.array(W0_flat, dtype=np.float64, copy=True)
+    M = np.array(M0_flat, dtype=np.float64, copy=True)
+    one = W.ndim == 1
+    if one:
+        W, M = W[None], M[None]
+    eta = np.asarray(eta, dtype=np.float64).reshape(W.shape[0], -1)
+    beta = np.asarray(beta, dtype=np.float64).reshape(W.shape[0], -1)
+    gamma = np.asarray(gamma, dtype=np.float64).reshape(W.shape[0], -1)
+    nc = eta.shape[1] // b if n_chunks is None else n_chunks
+    for s in range(W.shape[0]):
+        for c in range(nc):
+            sl = slice(c * b, (c + 1) * b)
+            if update == "lact":
+                bbar = float(np.mean(beta[s, sl]))
+                M[s] = bbar * M[s]
+                W[s] = W[s] + M[s]
+            else:
+                _, _, g0, b0, cM = scalar_kernels(eta[s, sl], beta[s, sl], gamma[s, sl])
+                W[s] = g0 * W[s] + cM * M[s]
+                M[s] = b0 * M[s]
+    return (W[0], M[0]) if one else (W, M)
+
+
 # ---------------------------------------------------------------------------
 # Final prediction with the updated weights
 # ([TTT-E2E] 持续学习框架 (预测 step) and the sketch's 最终预测 part;

@@ -657,3 +657,58 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(O, "mlp_backward", no_resid)
     _must_fail(test_gradients_and_losses_match_autograd, "gelu", True, 3)
     monkeypatch.undo()
+
+
+# ---------------------------------------------------------------------------
+# The state without gradients (what the parity tests subtract to isolate the
+# gradient-driven part of the final state)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rule", ["closed", "lact"])
+def test_state_without_gradients_is_the_zero_head_run(rule):
+    """A zero LM head gives zero gradients everywhere ([TTT-E2E] 核心方法: the
+    loss reaches the weights only through the head), so the full inner loop
+    must end exactly where the gradient-free recursion of Proposition 3.1 /
+    LaCT's rule ends."""
+    s = tiny_setup(kind="swiglu", d=4, h=6, V=7, L=2, static=True, T=12, m0=0.3)
+    E0 = np.zeros_like(s["E"])
+    model0 = O.make_model(s["d"], s["h"], s["V"], s["L"], "swiglu", 1e-6, E0, s["g"], s["static_w"])
+    W, M, _ = run_prefill(s, 4, update=rule, model=model0)
+    Wn, Mn = O.state_without_gradients(s["W0"], s["M0"], s["eta"][None], s["beta"][None], s["gamma"][None], 4,
+                                       update=rule)
+    np.testing.assert_allclose(W, Wn, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(M, Mn, rtol=1e-13, atol=1e-15)
+    # and a nonzero head moves the state away from it
+    W1, _, _ = run_prefill(s, 4, update=rule)
+    assert rel(W1, Wn) > 1e-6
+
+
+def test_state_without_gradients_matches_token_recursion():
+    """Per-token recursion of [E2-TTT] 原始公式 with G_t = 0, token by token:
+    M_t = beta_t M_{t-1}, W_t = gamma_t W_{t-1} + M_t; includes a beta = 0 and a
+    gamma = 1 inside a chunk, and two sequences with their own scalars."""
+    rng = np.random.default_rng(3)
+    B, T, b, n = 2, 15, 5, 9
+    W0 = rng.normal(size=(B, n))
+    M0 = rng.normal(size=(B, n))
+    eta = rng.uniform(0.0, 0.1, (B, T))
+    beta = rng.uniform(0.5, 0.99, (B, T))
+    gamma = rng.uniform(0.9, 1.0, (B, T))
+    beta[0, 7] = 0.0
+    gamma[1, 3] = 1.0
+    Wn, Mn = O.state_without_gradients(W0, M0, eta, beta, gamma, b)
+    for s in range(B):
+        Wt, Mt = W0[s].copy(), M0[s].copy()
+        for t in range(T):
+            Mt = beta[s, t] * Mt
+            Wt = gamma[s, t] * Wt + Mt
+        np.testing.assert_allclose(Wn[s], Wt, rtol=1e-13)
+        np.testing.assert_allclose(Mn[s], Mt, rtol=1e-13)
+    # n_chunks stops early: two chunks = the recursion over the first 2 b tokens
+    W2, M2 = O.state_without_gradients(W0[0], M0[0], eta[:1], beta[:1], gamma[:1], b, n_chunks=2)
+    Wt, Mt = W0[0].copy(), M0[0].copy()
+    for t in range(2 * b):
+        Mt = beta[0, t] * Mt
+        Wt = gamma[0, t] * Wt + Mt
+    np.testing.assert_allclose(W2, Wt, rtol=1e-13)
+    np.testing.assert_allclose(M2, Mt, rtol=1e-13)
