@@ -167,12 +167,14 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
  * the library until the process exits; calls needing more scratch than that
  * (ttt_workspace_size() > 16 MiB) return TTT_ERR_WORKSPACE with the sizes in
  * ttt_last_error().  Launches run directly on `stream` (no CUDA graph).  The
- * first call on a device looks up the array's device address
+ * first call on a device (and the first after a device reset, which gives the
+ * device a new context) looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture.  All calls share the one array: calls whose work
  * overlaps on the GPU (other streams, other threads, other handles) race and
  * corrupt each other's results; serialise them.  Nothing in the array needs
- * to start at zero (every buffer is written before it is read in a call). */
+ * to start at zero: every buffer is written before it is read in a call, and
+ * the call clears its split-K arrival counters itself. */
 ttt_status ttt_prefill_noalloc(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* hidden,
                                const int32_t* tokens, float* W, float* M, const float* eta, const float* beta,
                                const float* gamma, float* chunk_loss, void* stream);

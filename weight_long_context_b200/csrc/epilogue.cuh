@@ -338,8 +338,6 @@ struct EpiCEPartial {
   const int* tokens;  // [B, T]
   TokenMap tm;
   int ntn;
-  float* logits;      // [rows, ld_logits] fp32 copy of the logits for pass B, or nullptr
-  int ld_logits;
   __device__ void row_begin(RowState& st, int, int r) const {
     st.m = -INFINITY;
     st.s = 0.f;
@@ -358,15 +356,6 @@ struct EpiCEPartial {
     if (k >= 0 && k < nv) {
 #pragma unroll
       for (int j = 0; j < 32; ++j) if (j == k) tgt[r] = v[j];
-    }
-    if (logits) {
-      float* o = logits + (int64_t)r * ld_logits + c0;
-      if (nv == 32) {
-        vst<32>(o, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) if (j < nv) o[j] = v[j];
-      }
     }
   }
   __device__ void row_end(RowState& st, int, int r, int part_index) const {

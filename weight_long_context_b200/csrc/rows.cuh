@@ -290,37 +290,6 @@ __global__ void scalar_heads_kernel(const float* __restrict__ x, int64_t rows, i
   }
 }
 
-// Cross-entropy pass B from the logits kept by pass A (fp32):
-// P[r, j] = exp(logit[r, v0 + j] - lse[r]) - [v0 + j == y_r] for j < vs, the
-// operand slab of dz = P E_slab (row pitch Vs).  The same arithmetic as
-// recomputing the slab's logits, so the result is identical.  8 columns per thread.
-template <typename T>
-__global__ void ce_dlogits_kernel(const float* __restrict__ logits, int ld_logits, const float* __restrict__ lse,
-                                  const int* __restrict__ tokens, TokenMap tm, T* __restrict__ P, int Vs, int v0,
-                                  int vs, int64_t n) {
-  const int64_t groups = (vs + 7) / 8;
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n * groups) return;
-  const int64_t r = i / groups;
-  const int j0 = (int)(i - r * groups) * 8;
-  const float l = lse[r];
-  const int k = tokens[tm.index((int)r)] - v0 - j0;
-  const float* src = logits + r * ld_logits + v0 + j0;
-  T* dst = P + r * Vs + j0;
-  if (j0 + 8 <= vs) {
-    const float4 a = *reinterpret_cast<const float4*>(src);
-    const float4 b = *reinterpret_cast<const float4*>(src + 4);
-    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float p[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) p[q] = expf(x[q] - l) - (q == k ? 1.0f : 0.0f);
-    store4<T>(dst, make_float4(p[0], p[1], p[2], p[3]));
-    store4<T>(dst + 4, make_float4(p[4], p[5], p[6], p[7]));
-  } else {
-    for (int q = 0; q < vs - j0; ++q) dst[q] = from_f<T>(expf(src[q] - l) - (q == k ? 1.0f : 0.0f));
-  }
-}
-
 // Chunk mean of the token losses, one block per sequence, fixed reduction
 // order (the result does not depend on scheduling).
 __global__ void ce_mean_kernel(const float* __restrict__ ltok, int b, float* __restrict__ chunk_loss, int chunk,

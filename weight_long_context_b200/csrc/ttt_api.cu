@@ -115,7 +115,7 @@ struct Plan {
   float kscale;  // 1/b for the mean reduction, 1 for the sum
   bool swiglu, has_static;
   size_t esz;  // operand element size
-  size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, logits, P, dz, dout, dout_a,
+  size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
       doutW[2], doutM[2], dU, sk_partial, sk_counters, total;
   bool recon;           // reconstruction head: no LM-head buffers; yk, yq, qres below
   size_t yk, yq, qres;  // fp32 [n, d]: MLP outputs on the keys and queries, the query rows
@@ -147,15 +147,21 @@ static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
   p.esz = c.precision == TTT_PREC_FP32 ? 4 : 2;
   p.kscale = (c.loss_reduction == TTT_REDUCE_MEAN && b > 0) ? 1.0f / (float)b : 1.0f;
   p.ntn = head_parts(c.precision, p.V);
-  // vocabulary slab: the [n, Vs] slab of dl/dlogits.  Recomputing the logits
-  // (fp32 path): capped at 32 MiB so it stays resident in L2.  With the logits
-  // kept (bf16 path) pass B is elementwise and one dz GEMM over the whole
-  // vocabulary beats two smaller ones: capped at 128 MiB.
-  const size_t cap = (c.precision == TTT_PREC_BF16 ? 128ull : 32ull) << 20;
-  int64_t vs = p.n > 0 ? (int64_t)(cap / ((size_t)p.n * p.esz)) : 0;   // batch 0: no rows
-  vs = vs / 256 * 256;
-  if (vs < 256) vs = 256;
-  if (vs >= p.V) vs = p.V;
+  // vocabulary slab: CE pass B recomputes the logits of one slab of Vs
+  // columns at a time and writes softmax - onehot for it as the operand of
+  // dz += P_slab E_slab, so no [n, V] buffer exists.  A slab is at most 32 MiB
+  // (it stays resident in L2 between the two GEMMs); the vocabulary is cut
+  // into equal slabs of whole 256-column tiles.
+  const size_t cap = 32ull << 20;
+  int64_t vs = 0;
+  if (p.n > 0 && p.V > 0) {
+    const size_t full = (size_t)p.n * p.V * p.esz;
+    const int64_t ns = (int64_t)((full + cap - 1) / cap);
+    vs = ((p.V + ns - 1) / ns + 255) / 256 * 256;
+    const int64_t vmax = std::max<int64_t>(256, (int64_t)(cap / ((size_t)p.n * p.esz)) / 256 * 256);
+    if (vs > vmax) vs = vmax;
+    if (vs >= p.V) vs = p.V;
+  }
   p.Vs = (int)vs;
   p.nslabs = p.Vs > 0 ? (p.V + p.Vs - 1) / p.Vs : 0;
 
@@ -178,9 +184,6 @@ static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
   p.tgt = take(4 * n);
   p.lse = take(4 * n);
   p.ltok = take(4 * n);
-  // bf16 path: the head GEMM of CE pass A also keeps the fp32 logits [n, V],
-  // so pass B is elementwise instead of a second head GEMM.
-  p.logits = take(c.precision == TTT_PREC_BF16 ? 4ull * n * p.V : 0);
   p.P = take(e * n * p.Vs);
   p.dz = take(4 * n * d);
   p.dout = take(4 * n * d);
@@ -280,7 +283,7 @@ enum KernelClass {
 };
 static const char* kClassName[K_NCLASS] = {
     "scalar_scan", "w_shadow", "gather", "mlp_up", "mlp_down", "rmsnorm_fwd", "ce_logits_lse", "ce_rows",
-    "ce_mean", "ce_dlogits", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update", "recon_rows",
+    "ce_mean", "ce_logits_grad", "ce_dz", "rmsnorm_bwd", "mlp_bwd_dA", "mlp_bwd_dX", "agg_update", "recon_rows",
     "attn_proj", "attn_scores", "attn_rows"};
 
 struct Prof {
@@ -410,7 +413,6 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
   float* lse = reinterpret_cast<float*>(ws + p.lse);
   float* ltok = reinterpret_cast<float*>(ws + p.ltok);
   T* P = reinterpret_cast<T*>(ws + p.P);
-  float* logits = std::is_same<T, float>::value ? nullptr : reinterpret_cast<float*>(ws + p.logits);
   float* dz = reinterpret_cast<float*>(ws + p.dz);
   float* dout = reinterpret_cast<float*>(ws + p.dout);
   T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
@@ -428,7 +430,7 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
     Operand A = opnd(z, d, 0, 1, n);
     Operand Be = opnd(E, d, 0, 1, V);
     LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-           TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, logits, V}, st, status, ss))));
+           TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
   }
   LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
          (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
@@ -437,12 +439,7 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
   for (int sl = 0; sl < p.nslabs; ++sl) {
     const int v0 = sl * p.Vs;
     const int vs = V - v0 < p.Vs ? V - v0 : p.Vs;
-    if (logits) {   // softmax - onehot from the kept logits
-      const int64_t work = (int64_t)n * ((vs + 7) / 8);
-      LAUNCH(K_CE_GRAD, 0, (4.0 + e) * n * vs,
-             (ce_dlogits_kernel<T><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(logits, V, lse, tokens, tm, P,
-                                                                                  p.Vs, v0, vs, n)));
-    } else {        // fp32 path: recompute the slab's logits
+    {   // recompute the slab's logits; the epilogue writes softmax - onehot
       GemmShape s{n, vs, d, 1};
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E + (int64_t)v0 * d, d, 0, 1, vs);
@@ -1156,7 +1153,7 @@ static cudaError_t enqueue_predict(ttt_handle* hd, const Plan& p, const float* h
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E, d, 0, 1, V);
       LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn, nullptr, V}, st, status, ss))));
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
     }
     LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + (token_loss ? 20.0 : 16.0) * n,
            (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status,
@@ -1262,20 +1259,50 @@ static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[64] = {};   // device address of the scratch, per device ordinal
+static void* g_noalloc_ptr[64] = {};                 // device address of the scratch, per device ordinal
+static unsigned long long g_noalloc_ctx[64] = {};    // id of the context that address belongs to
+
+// Unique id of this thread's current context (0 if none is current or the
+// driver cannot say).  A device reset replaces the context, and the array's
+// address in the new one has to be looked up again.
+static unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static bool resolved = false;
+  if (!resolved) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+    resolved = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the scratch for the current device.  In host code the
 // array's name is only a stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, once per device and context, with that device current.
 static ttt_status noalloc_scratch(void** out) {
   int dev = 0;
   TTT_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(TTT_ERR_UNSUPPORTED, "device ordinal above 63");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* ptr = nullptr;
     TTT_CUDA_TRY(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
     g_noalloc_ptr[dev] = ptr;
+    g_noalloc_ctx[dev] = current_context_id();   // the lookup made the device's context current
   }
   *out = g_noalloc_ptr[dev];
   return TTT_OK;
