@@ -114,6 +114,27 @@ def input_bytes(w: I.Workload) -> int:
     return w.batch * w.T * (w.d * 4 + 4 + 12)
 
 
+def min_bytes_per_step(w: I.Workload) -> float:
+    """Algorithmic HBM bytes of one inner-loop pass: per chunk, every dynamic
+    parameter's fp32 W and M read and written once plus its bf16 (fp32 in fp32
+    mode) operand shadow written; the frozen LM head and static MLPs read once
+    per chunk (they are shared by the sequences of a batch); the inputs (hidden
+    rows, tokens, three scalars) read once."""
+    e = 4 if w.precision == "fp32" else 2
+    dyn = w.batch * w.n_blocks * w.block_params
+    frozen = (w.vocab * w.d + (w.n_blocks * w.block_params if w.has_static else 0)) * e
+    per_chunk = dyn * (16 + e) + frozen
+    return float(w.n_chunks * per_chunk + input_bytes(w))
+
+
+def hbm_line(w: I.Workload, ms: float, pk: dict) -> dict:
+    by = min_bytes_per_step(w)
+    gbs = by / (ms / 1e3) / 1e9
+    return {"algorithmic_bytes_per_step": by, "achieved_GBs": gbs, "frac": gbs / pk["hbm"],
+            "peak_GBs": pk["hbm"], "what": "state read+write and operand shadow per chunk, frozen head and "
+                                         "static MLPs once per chunk, inputs once"}
+
+
 def measured_peaks() -> dict:
     try:
         return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -394,44 +415,73 @@ def run_ours(args, w: I.Workload):
         rng = np.random.default_rng(100 + rank)
         heads = (T(rng.normal(0.0, 1.0 / np.sqrt(w.d), (3, w.d))), (0.0, 0.0, 0.0), 0.01, 1.0, 16.0)
 
-    def step():
+    # Every step is one prefill from the initial state: W and M are restored
+    # from W0 / M0 before each step, outside the timed events.
+    W0d, M0d = W.clone(), M.clone()
+
+    def step(g=None):
         if heads is not None:
             e_, b_, g_ = ttt.ttt_scalar_heads(hidden, *heads, stream=st)
             return h.prefill(hidden, tokens, W, M, e_, b_, g_, w.b, stream=st)
-        return h.prefill(hidden, tokens, W, M, eta, beta, gamma, w.b, stream=st)
+        return h.prefill(hidden, tokens, W, M, eta, beta, gamma if g is None else g, w.b, stream=st)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert h.device_status() == 0, "device status after warm-up"
+    def timed_steps(n_steps, g=None):
+        """args.warmup untimed steps, then n_steps steps each bracketed by CUDA
+        events on the launching stream (the state restore and the L2 flush sit
+        outside the events); returns per-step ms and the sampled clocks."""
+        for _ in range(args.warmup):
+            W.copy_(W0d)
+            M.copy_(M0d)
+            step(g)
+        torch.cuda.synchronize()
+        assert h.device_status() == 0, "device status after warm-up"
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
+        clocks = ClockSampler()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        if rank == 0:
+            clocks.start()
+        for i in range(n_steps):
+            W.copy_(W0d)
+            M.copy_(M0d)
+            if flush is not None:
+                flush.fill_(i & 0xff)
+            ev[i][0].record(st)
+            step(g)
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        clk = clocks.stop() if rank == 0 else None
+        return [a.elapsed_time(b) for a, b in ev], clk
 
     # ---- timed region: K steps, per-step CUDA events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    clocks = ClockSampler()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    if rank == 0:
-        clocks.start()
-    for i in range(args.steps):
-        if flush is not None:
-            flush.fill_(i & 0xff)
-        ev[i][0].record(st)
-        step()
-        ev[i][1].record(st)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop() if rank == 0 else None
-    step_ms = [a.elapsed_time(b) for a, b in ev]
+    step_ms, clk = timed_steps(args.steps)
     status = h.device_status()
     mean_ms = reduce_max(statistics.mean(step_ms), dev)
     tokens_per_step = w.batch * w.T
     value = whole_job_rate(tokens_per_step, world, mean_ms / 1e3)
+    state_norm = float(torch.linalg.vector_norm(W).item())
+
+    # ---- the same workload on a state that stays live (gamma = 1): under the
+    # E2-TTT draw W and M decay towards zero within a step, and GEMMs on zero
+    # operands draw less power; this timing shows what that is worth.
+    live = None
+    if w.scalars == "e2ttt" and heads is None and not args.no_live_state:
+        g1 = torch.ones_like(gamma)
+        live_ms, live_clk = timed_steps(max(3, min(args.steps, 10)), g1)
+        live_mean = reduce_max(statistics.mean(live_ms), dev)
+        live = {"value": whole_job_rate(tokens_per_step, world, live_mean / 1e3), "unit": UNIT,
+                "ms_per_step": live_mean, "steps": len(live_ms), "clocks": live_clk,
+                "scalars": "eta and beta of the workload's draw, gamma = 1 (no decay)",
+                "final_W_norm": float(torch.linalg.vector_norm(W).item())}
+        if live_clk and live_clk.get("sm_mhz"):
+            live["cycles_per_step"] = live_mean * 1e-3 * live_clk["sm_mhz"] * 1e6
 
     # ---- per-kernel breakdown from one profiled replay (same launches, eager, events per launch)
-    W2, M2 = W.clone(), M.clone()
+    W2, M2 = W0d.clone(), M0d.clone()
     _, stats = h.prefill_profiled(hidden, tokens, W2, M2, eta, beta, gamma, w.b, stream=st)
     del W2, M2
     launches_per_step = sum(s["launches"] for s in stats)
@@ -480,7 +530,7 @@ def run_ours(args, w: I.Workload):
           pin(x["beta"]), pin(x["gamma"])]
     h2d = sum(t.numel() * t.element_size() for t in (hx[:4] if heads is not None else hx))
     d2h = 2 * hx[2].numel() * 4 + w.batch * w.n_chunks * 4
-    del hidden, tokens, W, M, eta, beta, gamma
+    del hidden, tokens, W, M, W0d, M0d, eta, beta, gamma
     torch.cuda.empty_cache()
     h.prefill_host(*hx, b=w.b, stream=st, scalar_heads=heads)    # warm the host path once
     e_steps = max(1, min(args.steps, 3))
@@ -510,7 +560,13 @@ def run_ours(args, w: I.Workload):
                 "pct_of_bf16_peak": {"burst": tflops / world / pk["tflops"],
                                      "sustained": tflops / world / pk["tflops_sustained"], "source": pk["source"]},
                 "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
-                "roofline": roofline, "device_status": status}
+                "roofline": roofline, "device_status": status, "final_W_norm": state_norm,
+                "us_per_chunk": 1e3 * mean_ms / w.n_chunks,
+                "hbm": hbm_line(w, mean_ms, pk)}
+        if clk and clk.get("sm_mhz"):
+            line["cycles_per_step"] = mean_ms * 1e-3 * clk["sm_mhz"] * 1e6
+        if live is not None:
+            line["live_state"] = live
         if heads_line is not None:
             line["config"]["scalars"] = "input-dependent heads (eta_base 0.01, alpha_base 1, tau 16)"
             line["scalar_heads"] = heads_line
@@ -757,6 +813,10 @@ def main(argv=None):
                     choices=I.WORKLOAD_ORDER + ["e2ttt_layer_128k", "stack_128k_swa"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-live-state", action="store_true",
+                    help="skip the second timing on a state that stays live (gamma = 1)")
+    ap.add_argument("--scalars", default="", choices=["", "e2ttt_live"],
+                    help="override the workload's scalar recipe (e2ttt_live: the E2-TTT draw with gamma = 1)")
     ap.add_argument("--scalar-heads", action="store_true",
                     help="input-dependent scalars: eta, beta, gamma computed from the hidden rows on the device "
                          "inside every step (eta_base 0.01, alpha_base 1, tau 16, heads N(0, 1/d))")
@@ -778,6 +838,8 @@ def main(argv=None):
         w = w.with_(T=min(w.T, args.chunks * w.b))
     if args.update_rule != w.update_rule:
         w = w.with_(update_rule=args.update_rule)
+    if args.scalars and args.scalars != w.scalars:
+        w = w.with_(scalars=args.scalars, name=w.name + "_" + args.scalars)
     if args.impl == "reference":
         return run_reference(args, w)
     if args.final_prediction:

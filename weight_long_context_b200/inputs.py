@@ -17,7 +17,12 @@ them:
   CDF, because natural-text token frequencies are Zipf-like;
 * LM head, static MLPs and the initial fast weights W0 ~ N(0, 0.02^2);
 * scalars: plain SGD (eta = alpha, beta = 0, gamma = 1) or the E2-TTT draw
-  eta = 0.01 * sigmoid(N(0,1)), beta ~ U(0.8, 0.99), gamma ~ U(0.99, 1.0).
+  eta = 0.01 * sigmoid(N(0,1)), beta ~ U(0.8, 0.99), gamma ~ U(0.99, 1.0);
+  "e2ttt_live" is the same draw with gamma then set to 1 (no decay).  Under
+  the plain E2-TTT draw a chunk of 1024 tokens scales the state by a product
+  of gammas near 0.006, so over a long sequence W and M decay to zero; with
+  gamma = 1 the state keeps its size, which is what an added parity case and
+  a live-state timing need.
 
 Draw order (one numpy Generator seeded once): hidden, tokens, LM head, static
 weights, W0, M0 (only if requested), eta, beta, gamma.
@@ -48,7 +53,7 @@ class Workload:
     T: int
     b: int
     batch: int
-    scalars: str  # "sgd" or "e2ttt"
+    scalars: str  # "sgd", "e2ttt" or "e2ttt_live" (the e2ttt draw with gamma = 1)
     sgd_lr: float = 0.0
     token_dist: str = "zipf"
     rms_eps: float = 1e-6
@@ -208,6 +213,8 @@ def make_inputs(w: Workload, seed: int = 0, T: Optional[int] = None,
         eta = (0.01 / (1.0 + np.exp(-z))).astype(np.float32)
         beta = rng.uniform(0.8, 0.99, size=(B, T)).astype(np.float32)
         gamma = rng.uniform(0.99, 1.0, size=(B, T)).astype(np.float32)
+        if w.scalars == "e2ttt_live":
+            gamma = np.ones_like(gamma)
 
     return dict(hidden=hidden, tokens=tokens, lm_head=lm_head, rms_gain=rms_gain,
                 static_w=static_w, W0=W0, M0=M0, eta=eta, beta=beta, gamma=gamma)
