@@ -58,5 +58,5 @@ def test_heads_feed_the_inner_loop(dev, precision):
     re, rb, rg = oracle.scalar_heads(x["hidden"], Wh.astype(np.float32), bh.astype(np.float32),
                                      ETA_BASE, ALPHA_BASE, TAU)
     xr = dict(x, eta=re, beta=rb, gamma=rg)
-    e_ = H.compare(w, x, H.run_gpu(w, xg, dev), H.run_oracle(w, xr))
+    e_ = H.compare(w, xr, H.run_gpu(w, xg, dev), H.run_oracle(w, xr))
     print("heads", precision, e_)

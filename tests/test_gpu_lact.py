@@ -57,10 +57,16 @@ def test_lact_ragged_parity(dev, case, precision):
 
 def test_lact_full_dims_first_chunks(dev):
     """The 128K stack's shapes (the benchmark's launch configuration), first
-    two chunks, under the LaCT rule."""
+    two chunks, under the LaCT rule.  W0 and the static MLPs are drawn at a
+    quarter of the workload's scale: at the full draw float32 and float64 runs
+    of the oracle already differ by about 2 % on the gradient-driven part of W
+    (see test_stack_128k_first_chunks_against_fp64), which that part's bound
+    would measure instead of the kernels."""
     w = I.WORKLOADS["stack_128k"]
     w = w.with_(T=2 * w.b, update_rule="lact")
     x = I.make_inputs(w, seed=0, m0_scale=1e-3)
+    x["W0"] = x["W0"] * np.float32(0.25)
+    x["static_w"] = x["static_w"] * np.float32(0.25)
     e = H.compare(w, x, H.run_gpu(w, x, dev), H.run_oracle(w, x, dtype=np.float32))
     print("stack_128k lact", e)
 
