@@ -561,6 +561,10 @@ def run_ours(args, w: I.Workload):
                                      "sustained": tflops / world / pk["tflops_sustained"], "source": pk["source"]},
                 "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
                 "roofline": roofline, "device_status": status, "final_W_norm": state_norm,
+                "breakdown": {st_["name"]: {"launches": st_["launches"], "ms": round(st_["ms"], 3),
+                                            "us_per_launch": round(1e3 * st_["ms"] / st_["launches"], 2),
+                                            "share": round(st_["ms"] / step_total, 4)}
+                              for st_ in sorted(stats, key=lambda q: -q["ms"])},
                 "us_per_chunk": 1e3 * mean_ms / w.n_chunks,
                 "hbm": hbm_line(w, mean_ms, pk)}
         if clk and clk.get("sm_mhz"):

@@ -32,14 +32,35 @@ template <typename T>
 struct EpiStoreHeads {
   static constexpr bool kFixedHeadTile = false;
   static constexpr bool kPreload = false;
-  static constexpr bool kWarpRows = false;
+  static constexpr bool kWarpRows = true;
   using RowState = NoRowState;
+  using SpanRegs = NoSpanRegs;
   T* out;
   int b;
   int H;
   int dh;
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
+  // Row-walking form (tcgen05 engine): the lane's 4 columns lie in one head
+  // (dh % 16 == 0).
+  __device__ void load_span(SpanRegs&, int, int, int, int, int, int, int) const {}
+  __device__ void finish_span(const SpanRegs&, int half, int, int row0, int c0, const float* sv, int nv, int nrows,
+                              int lane) const {
+    const int cj = rw_col(lane);
+    if (cj >= nv) return;
+    const int c = c0 + cj, hh = c / dh, e = c - hh * dh;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = rw_row(half, k, lane);
+      if (i >= nrows) continue;
+      const int r = row0 + i, s = r / b, ii = r - s * b;
+      float a[4];
+      rw_read4(sv, i, cj, a);
+      T* o = out + (((int64_t)s * H + hh) * b + ii) * dh + e;
+      if (cj + 4 <= nv) store_x4(o, a);
+      else for (int j = 0; j < nv - cj; ++j) o[j] = from_f<T>(a[j]);
+    }
+  }
   __device__ void span(RowState&, int, int r, int c0, const float* v, const float*, int nv) const {
     const int s = r / b, i = r - s * b;
     const int h0 = c0 / dh, e0 = c0 - h0 * dh;

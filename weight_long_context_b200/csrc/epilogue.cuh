@@ -102,6 +102,29 @@ __device__ __forceinline__ void store_x4(float* p, const float* v) {
 __device__ __forceinline__ void store_x4(__nv_bfloat16* p, const float* v) {
   *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
+// ---------------------------------------------------------------------------
+// Row-walking form (kWarpRows), used by the tcgen05 engine for the plain
+// stores and the state update.  The engine stages a 32 x 32 span of the
+// accumulators in shared memory (element (row i, column j) at
+// sv[i * 32 + ((j + i) & 31)]) and calls load_span() / finish_span() for each
+// half of it (rows [16 half, 16 half + 16)).  Lane l covers columns
+// [4 (l % 8), 4 (l % 8) + 4) of the rows 16 half + 4 k + l / 8, k < 4, so a
+// warp instruction touches 4 rows x 32 contiguous columns.  row0 is the
+// span's first row inside batch entry z, c0 its first column; only rows
+// < nrows and columns < nv of the span are inside the matrix.  Measured on
+// B200, this form pays for stores only: epilogues that read per-row scalars
+// or per-element operands (the MLP and cross-entropy epilogues) keep the
+// one-row-per-thread form, where each thread loads its row once per tile and
+// a whole span's operands are in flight at once.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int rw_row(int half, int k, int lane) { return 16 * half + 4 * k + (lane >> 3); }
+__device__ __forceinline__ int rw_col(int lane) { return (lane & 7) * 4; }
+// Four consecutive staged values of span row i starting at span column c.
+__device__ __forceinline__ void rw_read4(const float* sv, int i, int c, float* a) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) a[j] = sv[i * 32 + ((c + j + i) & 31)];
+}
+struct NoSpanRegs {};
 
 // ---------------------------------------------------------------------------
 // F1: U = a W1^T (GELU: [n,h]; SwiGLU: [n,2h] in the interleaved layout).
@@ -434,13 +457,30 @@ struct EpiStoreF32 {
 struct EpiStoreBatched {
   static constexpr bool kFixedHeadTile = false;
   static constexpr bool kPreload = false;
-  static constexpr bool kWarpRows = false;
+  static constexpr bool kWarpRows = true;
   using RowState = NoRowState;
+  using SpanRegs = NoSpanRegs;
   float* out;
   int64_t ld;
   int64_t zstride;
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
+  __device__ void load_span(SpanRegs&, int, int, int, int, int, int, int) const {}
+  __device__ void finish_span(const SpanRegs&, int half, int z, int row0, int c0, const float* sv, int nv,
+                              int nrows, int lane) const {
+    const int cj = rw_col(lane);
+    if (cj >= nv) return;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = rw_row(half, k, lane);
+      if (i >= nrows) continue;
+      float a[4];
+      rw_read4(sv, i, cj, a);
+      float* o = out + (int64_t)z * zstride + (int64_t)(row0 + i) * ld + c0 + cj;
+      if (cj + 4 <= nv && (reinterpret_cast<uintptr_t>(o) & 15) == 0) store_x4(o, a);
+      else for (int j = 0; j < 4 && j < nv - cj; ++j) o[j] = a[j];
+    }
+  }
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
     float* o = out + (int64_t)z * zstride + (int64_t)r * ld + c0;
     if (nv == 32 && ((reinterpret_cast<uintptr_t>(o) & 15) == 0)) {
@@ -483,13 +523,14 @@ struct EpiUpdate {
   __device__ void row_begin(RowState&, int, int) const {}
   __device__ void row_end(RowState&, int, int, int) const {}
   // Row-walking epilogue (used by the tcgen05 engine): a warp updates a span
-  // of 32 rows x 32 columns, 8 lanes x 4 columns per row, so every W / M /
-  // shadow access of an instruction covers whole 128-byte rows.  load_span()
-  // issues the span's W and M loads into registers; finish_span() combines
-  // them with the accumulators staged in shared memory (sv / sv2: element
-  // (row i, column j) at [i * 32 + ((j + i) & 31)], rotated so both the
-  // staging writes and these reads are conflict-free) and stores the results.
-  // The engine calls them per half span (16 rows), 8 warps per CTA.
+  // of 32 rows x 32 columns, half a span (16 rows) per call, 8 lanes x 4
+  // columns per row, so every W / M / shadow access of an instruction covers
+  // whole 128-byte rows.  load_span() issues the half's W and M loads into
+  // registers; finish_span() combines them with the two accumulators staged
+  // in shared memory (sv: the half's row r of the first accumulator at
+  // buffer row r, of the second at buffer row 16 + r; element (buffer row i,
+  // column j) at [i * 32 + ((j + i) & 31)], rotated so both the staging
+  // writes and these reads are conflict-free) and stores the results.
   struct SpanRegs { float4 w[4], m[4]; };
   // half: rows [16 half, 16 half + 16) of the span (8 lanes x 4 rows per step).
   __device__ void load_span(SpanRegs& R, int half, int z, int row0, int c0, int nv, int nrows, int lane) const {
@@ -508,8 +549,8 @@ struct EpiUpdate {
       }
     }
   }
-  __device__ void finish_span(const SpanRegs& R, int half, int z, int row0, int c0, const float* sv,
-                              const float* sv2, int nv, int nrows, int lane) const {
+  __device__ void finish_span(const SpanRegs& R, int half, int z, int row0, int c0, const float* sv, int nv,
+                              int nrows, int lane) const {
     const float4 cs = *reinterpret_cast<const float4*>(consts + ((int64_t)z * nchunks + chunk) * 4);
     const float g0 = cs.x, b0 = cs.y, cM = cs.z;
     const int sub = lane >> 3, cj = (lane & 7) * 4;
@@ -523,11 +564,12 @@ struct EpiUpdate {
       if (i >= nrows || cj >= nv) continue;
       const int r = row0 + i;
       const int64_t off = (int64_t)(h > 0 ? swiglu_row_of_pos(r, h) : r) * cols;
+      const int b = 4 * k + sub;   // the row inside this half
       float a[4], a2[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        a[j] = sv[i * 32 + ((cj + j + i) & 31)];
-        a2[j] = sv2[i * 32 + ((cj + j + i) & 31)];
+        a[j] = sv[b * 32 + ((cj + j + b) & 31)];
+        a2[j] = sv[(16 + b) * 32 + ((cj + j + 16 + b) & 31)];
       }
       T* sp = Sz + (int64_t)r * cols;
       if (vec) {

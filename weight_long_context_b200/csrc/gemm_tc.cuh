@@ -41,7 +41,13 @@ constexpr int BK = 64;             // 64 bf16 = 128 bytes: one swizzle row
 constexpr int HEAD_BN = 256;       // N tile of the single-accumulator GEMMs
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_PARTS = EPI_WARPS / 4;   // column parts per tile row
-constexpr int THREADS = 64 + 32 * EPI_WARPS;
+// Epilogue warps of the two-accumulator state update (which streams 18 bytes
+// of fp32 W / M state per parameter).  Measured on B200 at the 128K stack's
+// shapes: 16 warps (four per TMEM lane quarter) run no faster than 8.
+constexpr int AGG_EPI_WARPS = 8;
+__host__ __device__ constexpr int epi_warps(int nacc, bool warprows) {
+  return (nacc == 2 && warprows) ? AGG_EPI_WARPS : EPI_WARPS;
+}
 constexpr uint64_t WAIT_NS = 4000000000ull;   // 4 s per wait before giving up
 
 // ---------------------------------------------------------------------------
@@ -180,21 +186,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n, int a_mn, int b_mn) {
 // ---------------------------------------------------------------------------
 template <int NACC, int BN, bool WARPROWS = false>
 struct Cfg {
-  // Epilogue warps: two per TMEM lane quarter, splitting the tile's columns.
-  static constexpr int EW = EPI_WARPS;
+  // Epilogue warps: two (four for the state update) per TMEM lane quarter,
+  // splitting the tile's columns.
+  static constexpr int EW = epi_warps(NACC, WARPROWS);
   static constexpr int PARTS = EW / 4;
   static constexpr int NTHREADS = 64 + 32 * EW;
   static constexpr int A_BYTES = BM * BK * 2;            // 16 KiB
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = NACC * A_BYTES + B_BYTES;
-  // Epilogues that walk rows per warp stage each warp's 32x32 span(s) in
-  // shared memory: NACC x 4 KiB per epilogue warp.
-  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EW * NACC * 32 * 32 * 4 : 0;
-  static constexpr int STAGES = ((WARPROWS ? 220 : 200) * 1024 - ROWSTAGE_BYTES) / STAGE_BYTES;
+  // Epilogues that walk rows stage each warp's 32x32 span in shared memory:
+  // 4 KiB per epilogue warp (the state update stages its two accumulators in turn).
+  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EW * 32 * 32 * 4 : 0;
+  // as many operand stages as the 227 KiB per CTA leave beside the staging,
+  // the 1 KiB alignment slack and the barriers
+  static constexpr int STAGES = (232448 - 1280 - ROWSTAGE_BYTES) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * NACC * BN;         // two accumulator buffers
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ROWSTAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-  static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(STAGES >= 2 && STAGES <= 16, "two to sixteen stages (the barriers take 256 bytes)");
   static_assert(SMEM_BYTES <= 232448, "shared memory above the 227 KiB per-CTA limit");
 };
 
@@ -249,20 +258,113 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   return x;
 }
 
-// Row-walking epilogue loop shared by both kernels: each 32 x 32 span of the
-// warp's accumulators is staged in shared memory (sv / sv2, rotated so the
-// staging writes and the row reads are conflict-free) and finished half a span
-// (16 rows) at a time, 8 lanes x 4 columns per row.  The tiles this CTA
-// processes are first, first + step, ...; tile rows start at
-// tm * rows_per_tile + row_off.  release(buf) frees the accumulator buffer once
-// every span of the tile is staged.  Epilogues of this kind keep no per-row state.
+// Row-walking epilogues.  The accumulators arrive one row per thread (the
+// TMEM lane layout); global rows are contiguous, so a thread writing its own
+// row would touch 32 separate lines per warp instruction.  Instead each warp
+// stages a 32 x 32 span in shared memory (element (row i, column j) at
+// [i * 32 + ((j + i) & 31)], rotated so the staging writes and the row reads
+// are both conflict-free) and the epilogue functor walks it row by row, half
+// a span (16 rows) at a time: 8 lanes x 4 columns per row, 4 rows per step,
+// so every global access of an instruction covers whole row segments.
+
+// Stage this thread's row of a 32-column span.
+__device__ __forceinline__ void stage_row32(float* sv, const float* v, int lane) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) sv[lane * 32 + ((j + lane) & 31)] = v[j];
+}
+
+// Walk a staged span: rows [row0, row0 + nrows) and columns [c0, c0 + nv) of
+// batch entry z, both halves.
+template <class Epi>
+__device__ __forceinline__ void finish_rows(const Epi& epi, int z, int row0, int c0, int nv, int nrows,
+                                            const float* sv, int lane) {
+  if (nrows <= 0 || nv <= 0) return;
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    typename Epi::SpanRegs R;
+    epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
+    epi.finish_span(R, half, z, row0, c0, sv, nv, nrows, lane);
+  }
+}
+
+// One tile of a row-walking epilogue read straight from TMEM (tbase: this
+// warp's lane quarter of the accumulator buffer).  The warp owns rows
+// [row0, row0 + 32) and the PART_COLS columns of its part.  release() frees
+// the accumulator buffer once every span of the tile is staged.
+// Stage columns [c, c + 32) of the accumulator at tbase (this thread's row).
+__device__ __forceinline__ void stage_tmem32(float* sv, uint32_t taddr, int lane) {
+#pragma unroll
+  for (int hc = 0; hc < 32; hc += 16) {
+    float v[16];
+    tmem_ld16(taddr + hc, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sv[lane * 32 + ((hc + j + lane) & 31)] = v[j];
+  }
+}
+
+template <int NACC, int BN, int PART_COLS, class Epi, class Release>
+__device__ __forceinline__ void rows_tile(const Epi& epi, const GemmShape& s, int z, int row0, int tn, uint32_t tbase,
+                                          float* sv, int part, int lane, Release release) {
+  constexpr int NSP = PART_COLS / 32;
+  const int nrows = min(32, s.M - row0);
+#pragma unroll 1
+  for (int spi = 0; spi < NSP; ++spi) {
+    const int c = part * PART_COLS + spi * 32;
+    const int c0 = tn * BN + c;
+    const int nv = min(32, s.N - c0);
+    if constexpr (NACC == 1) {
+      stage_tmem32(sv, tbase + c, lane);
+      if (spi == NSP - 1) {  // every accumulator of this tile is staged: free the buffer
+        tc_fence_before();
+        release();
+      }
+      __syncwarp();
+      finish_rows(epi, z, row0, c0, nv, nrows, sv, lane);
+      __syncwarp();
+    } else {
+      // Two accumulators through one 32 x 32 staging buffer, half a span at a
+      // time: rows [0, 16) of the buffer hold the half's rows of the first
+      // accumulator, rows [16, 32) the same rows of the second.  The half's
+      // global loads are issued before the TMEM reads.
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        typename Epi::SpanRegs R;
+        const bool live = nrows > 0 && nv > 0;
+        if (live) epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
+        const bool mine = (lane >> 4) == half;
+        const int r = lane & 15;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+#pragma unroll
+          for (int hc = 0; hc < 32; hc += 16) {
+            float v[16];
+            tmem_ld16(tbase + a * BN + c + hc, v);
+            if (mine) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sv[(16 * a + r) * 32 + ((hc + j + 16 * a + r) & 31)] = v[j];
+            }
+          }
+        }
+        if (half == 1 && spi == NSP - 1) {  // every accumulator of this tile is read: free the buffer
+          tc_fence_before();
+          release();
+        }
+        __syncwarp();
+        if (live) epi.finish_span(R, half, z, row0, c0, sv, nv, nrows, lane);
+        __syncwarp();
+      }
+    }
+  }
+}
+
+// Row-walking epilogue loop of the 1-SM kernel and of the pair kernel's
+// two-accumulator aggregation (never split): the tiles this CTA processes
+// are first, first + step, ...; tile rows start at tm * rows_per_tile + row_off.
 template <int NACC, int BN, int PART_COLS, class Epi, class Release>
 __device__ __forceinline__ void warp_rows_loop(const Epi& epi, const TcParams& p, int first, int step,
                                                int rows_per_tile, int row_off, uint32_t tmem_base,
-                                               uint64_t* tfull, float* sv, float* sv2, int q, int part, int lane,
+                                               uint64_t* tfull, float* sv, int q, int part, int lane,
                                                volatile int* abort_flag, Release release) {
-  constexpr int NSP = PART_COLS / 32;
-  const GemmShape& s = p.s;
   uint32_t tcount = 0;
   for (int t = first; t < p.num_tiles; t += step, ++tcount) {
     const uint32_t buf = tcount & 1u;
@@ -275,39 +377,8 @@ __device__ __forceinline__ void warp_rows_loop(const Epi& epi, const TcParams& p
     const int tn = rest % p.tiles_n;
     const int z = rest / p.tiles_n;
     const int row0 = tm * rows_per_tile + row_off + q * 32;
-    const int nrows = min(32, s.M - row0);
     const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
-#pragma unroll 1
-    for (int spi = 0; spi < NSP; ++spi) {
-      const int c = part * PART_COLS + spi * 32;
-      const int c0 = tn * BN + c;
-      const int nv = min(32, s.N - c0);
-#pragma unroll
-      for (int hc = 0; hc < 32; hc += 16) {
-        float v[16], v2[16];
-        tmem_ld16(tbase + c + hc, v);
-        if (NACC == 2) tmem_ld16(tbase + BN + c + hc, v2);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          sv[lane * 32 + ((hc + j + lane) & 31)] = v[j];
-          if (NACC == 2) sv2[lane * 32 + ((hc + j + lane) & 31)] = v2[j];
-        }
-      }
-      if (spi == NSP - 1) {  // every accumulator of this tile is staged: free the buffer
-        tc_fence_before();
-        release(buf);
-      }
-      __syncwarp();
-      if (nrows > 0 && nv > 0) {
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          typename Epi::SpanRegs R;
-          epi.load_span(R, half, z, row0, c0, nv, nrows, lane);
-          epi.finish_span(R, half, z, row0, c0, sv, sv2, nv, nrows, lane);
-        }
-      }
-      __syncwarp();
-    }
+    rows_tile<NACC, BN, PART_COLS>(epi, p.s, z, row0, tn, tbase, sv, part, lane, [&]() { release(buf); });
   }
 }
 
@@ -466,9 +537,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     constexpr int PART_COLS = BN / C::PARTS;
     const int row_in_tile = q * 32 + lane;
     if constexpr (Epi::kWarpRows) {
-      float* sv = rowstage + (warp - 2) * (NACC * 1024);
-      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, blockIdx.x, gridDim.x, BM, 0, tmem_base, tfull, sv,
-                                          sv + (NACC - 1) * 1024, q, part, lane, abort_flag,
+      float* sv = rowstage + (warp - 2) * 1024;
+      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, blockIdx.x, gridDim.x, BM, 0, tmem_base, tfull, sv, q, part,
+                                          lane, abort_flag,
                                           [&](uint32_t b) { mbar_arrive(&tempty[b]); });
     } else {
       uint32_t tcount = 0;
@@ -592,25 +663,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m256(int n, int a_mn, int b_mn
 // and CTA 1's the whole B2 tile; otherwise [A1 | (A2) | B half].
 template <int NACC, int BN, bool WARPROWS = false, bool DUALB = false>
 struct Cfg2 {
+  static constexpr int EW = epi_warps(NACC, WARPROWS);
+  static constexpr int PARTS = EW / 4;
+  static constexpr int NTHREADS = 64 + 32 * EW;
   static constexpr int A_BYTES = BM * BK * 2;            // this CTA's 128 rows
   static constexpr int B_BYTES = (BN / 2) * BK * 2;      // this CTA's BN/2 columns
   static constexpr int NA = DUALB ? 1 : NACC;            // A slots per stage
   static constexpr int NB = DUALB ? 2 : 1;               // B slots per stage
   static constexpr int STAGE_BYTES = NA * A_BYTES + NB * B_BYTES;
-  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EPI_WARPS * NACC * 32 * 32 * 4 : 0;
-  static constexpr int STAGES = ((WARPROWS ? 220 : 200) * 1024 - ROWSTAGE_BYTES) / STAGE_BYTES;
+  static constexpr int ROWSTAGE_BYTES = WARPROWS ? EW * 32 * 32 * 4 : 0;
+  static constexpr int STAGES = (232448 - 1280 - ROWSTAGE_BYTES) / STAGE_BYTES;
   static constexpr int TMEM_COLS = 2 * NACC * BN;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + ROWSTAGE_BYTES + 1024 + 256;
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
   static_assert(BN % 128 == 0, "each CTA loads whole 64-column boxes of B");
   static_assert(!DUALB || NACC == 2, "dual B operands need two accumulators");
-  static_assert(STAGES >= 2, "need at least two stages");
+  static_assert(STAGES >= 2 && STAGES <= 16, "two to sixteen stages (the barriers take 256 bytes)");
   static_assert(SMEM_BYTES <= 232448, "shared memory above the 227 KiB per-CTA limit");
 };
 
 // mapA2: the second A operand, or with DUALB the second B operand.
 template <int NACC, int BN, class Epi, bool DUALB = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg2<NACC, BN, Epi::kWarpRows, DUALB>::NTHREADS, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapA2,
                 const __grid_constant__ CUtensorMap mapB, const TcParams p, const Epi epi) {
   using C = Cfg2<NACC, BN, Epi::kWarpRows, DUALB>;
@@ -635,7 +709,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2 * 32 * EPI_WARPS); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2 * 32 * C::EW); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -757,15 +831,15 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     // ------------------------------ epilogue (both CTAs) ------------------------------
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;
-    constexpr int PART_COLS = BN / EPI_PARTS;
+    constexpr int PART_COLS = BN / C::PARTS;
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    float* sv = rowstage + (warp - 2) * 1024;   // row-walk staging (row-walking epilogues only)
     uint32_t tcount = 0;
-    if constexpr (Epi::kWarpRows) {   // never split: the launcher keeps splits == 1
-      float* sv = rowstage + (warp - 2) * (NACC * 1024);
-      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, pair, npairs, 2 * BM, (int)rank * BM, tmem_base, tfull, sv,
-                                          sv + (NACC - 1) * 1024, q, part, lane, abort_flag, [&](uint32_t b) {
+    if constexpr (Epi::kWarpRows && NACC == 2) {   // the aggregation: never split
+      warp_rows_loop<NACC, BN, PART_COLS>(epi, p, pair, npairs, 2 * BM, (int)rank * BM, tmem_base, tfull, sv, q,
+                                          part, lane, abort_flag, [&](uint32_t b) {
                                             mbar_arrive_remote(b ? tempty_leader1 : tempty_leader0);
                                           });
     } else
@@ -781,26 +855,49 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
       if (!ready) break;
       tc_fence_after();
-      const int r = tm * 2 * BM + (int)rank * BM + row_in_tile;
+      const int row0 = tm * 2 * BM + (int)rank * BM + q * 32;   // this warp's 32 rows
+      const int nrows = min(32, s.M - row0);
+      const int r = row0 + lane;                                 // this thread's row
       const bool row_ok = r < s.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
-      if (!un.split) {
-        typename Epi::RowState rs;
-        if (row_ok) epi.row_begin(rs, z, r);
-#pragma unroll 1
-        for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
-          float v[32], v2[32];
-          const int c0 = tn * BN + c;
+      // The finished fp32 values of one 32-column span of this thread's row
+      // go to the epilogue functor: staged and walked by rows, or per row.
+      auto emit_span = [&](typename Epi::RowState& rs, int c0, const float* v) {
+        if constexpr (Epi::kWarpRows) {
+          stage_row32(sv, v, lane);
+          __syncwarp();
+          finish_rows(epi, z, row0, c0, min(32, s.N - c0), nrows, sv, lane);
+          __syncwarp();
+        } else {
           if constexpr (Epi::kPreload) {
             if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
           }
-          tmem_ld32(tbase + c, v);
-          if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
-          if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+          if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
         }
-        if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
-        tc_fence_before();
-        mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+      };
+      if (!un.split) {
+        if constexpr (Epi::kWarpRows) {
+          rows_tile<NACC, BN, PART_COLS>(epi, s, z, row0, tn, tbase, sv, part, lane, [&]() {
+            mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+          });
+        } else {
+          typename Epi::RowState rs;
+          if (row_ok) epi.row_begin(rs, z, r);
+#pragma unroll 1
+          for (int c = part * PART_COLS; c < (part + 1) * PART_COLS; c += 32) {
+            float v[32], v2[32];
+            const int c0 = tn * BN + c;
+            if constexpr (Epi::kPreload) {
+              if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
+            }
+            tmem_ld32(tbase + c, v);
+            if (NACC == 2) tmem_ld32(tbase + BN + c, v2);
+            if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, NACC == 2 ? v2 : v, min(32, s.N - c0));
+          }
+          if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+          tc_fence_before();
+          mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
+        }
       } else if (p.pair_finish) {
         // Two splits resident at once: each finishes half of the tile's rows.
         // The warp whose rows the partner finishes parks its fp32 partial and
@@ -845,7 +942,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
           __threadfence();
           if (ok) {
             typename Epi::RowState rs;
-            if (row_ok) epi.row_begin(rs, z, r);
+            if (!Epi::kWarpRows && row_ok) epi.row_begin(rs, z, r);
 #pragma unroll 1
             for (int c = part * PART_COLS, sp = 0; c < (part + 1) * PART_COLS; c += 32, ++sp) {
               float v[32];
@@ -855,13 +952,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
                 const float4 x = __ldcg(region + (sp * 8 + i) * 32);
                 v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
               }
-              const int c0 = tn * BN + c;
-              if constexpr (Epi::kPreload) {
-                if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
-              }
-              if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
+              emit_span(rs, tn * BN + c, v);
             }
-            if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+            if (!Epi::kWarpRows && row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
           }
           tc_fence_before();
           mbar_arrive_remote(buf ? tempty_leader1 : tempty_leader0);
@@ -898,7 +991,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
         if (old == p.splits - 1) {
           __threadfence();
           typename Epi::RowState rs;
-          if (row_ok) epi.row_begin(rs, z, r);
+          if (!Epi::kWarpRows && row_ok) epi.row_begin(rs, z, r);
           const float4* base = reinterpret_cast<const float4*>(p.partial + ((size_t)t * p.splits * 2 + rank) * slab) +
                                (size_t)ew * (PART_COLS / 4) * 32 + lane;
 #pragma unroll 1
@@ -914,13 +1007,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
                 v[4 * i] += x.x; v[4 * i + 1] += x.y; v[4 * i + 2] += x.z; v[4 * i + 3] += x.w;
               }
             }
-            const int c0 = tn * BN + c;
-            if constexpr (Epi::kPreload) {
-              if (row_ok && c0 < s.N) epi.preload(rs, z, r, c0, min(32, s.N - c0));
-            }
-            if (row_ok && c0 < s.N) epi.span(rs, z, r, c0, v, v, min(32, s.N - c0));
+            emit_span(rs, tn * BN + c, v);
           }
-          if (row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
+          if (!Epi::kWarpRows && row_ok) epi.row_end(rs, z, r, tn * EPI_PARTS + part);
           __syncwarp();
           if (lane == 0) *ctr = 0;
         }
@@ -1175,7 +1264,7 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   p.num_tiles = p.tiles_m * p.tiles_n * s.batch;
   p.num_kb = (s.K + BK - 1) / BK;
   p.status = status;
-  const bool may_split = NACC == 1 && BN == 256 && !Epi::kWarpRows;
+  const bool may_split = NACC == 1 && BN == 256;
   const long full = may_split ? paired_finish_plan(p.num_tiles, p.num_kb, ss) : -1;
   if (full >= 0) {   // whole waves, then the last wave's tiles as paired halves
     p.pair_finish = 1;
@@ -1195,7 +1284,7 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   const int pairs = num_sms() / 2;
   const int units = p.num_units;
   const int grid = 2 * (units < pairs ? units : pairs);
-  gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, THREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
+  gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
   return cudaGetLastError();
 }
 
