@@ -2,10 +2,13 @@
 // ("TTT-E2E：端到端测试时训练的长上下文语言建模": the sketch's TTTE2EBlock,
 // TTTSelfAttention and RotaryEmbedding; 滑动窗口注意力, 关键设计参数).
 //
-// Row kernels around the attention GEMMs (which run on the same engines as
-// the MLP GEMMs, batched over heads): LayerNorm with frozen gain and bias,
-// the rotary embedding and the split of the fused q|k|v projection into
-// head-major operands, the window-masked softmax, its backward, the rotary
+// Epilogues and row kernels around the attention GEMMs (which run on the same
+// engines as the MLP GEMMs, batched over heads).  The scores never reach HBM:
+// a first score pass leaves masked online-softmax partials, a second one
+// recomputes the scores and writes the probabilities, and the dP GEMM forms
+// dS in its epilogue.  Row kernels: LayerNorm with frozen gain and bias, the
+// rotary embedding and the split of the fused q|k|v projection into
+// head-major operands, the rows' log-sum-exp and D = dO . O, the rotary
 // backward that packs dq|dk|dv for the input projection's backward, and the
 // split of the residual-stream gradient into the two weighted cotangent
 // streams the chunk update needs once attention mixes the rows.
@@ -14,8 +17,8 @@
 //   q of the chunk       [B][H][b][dh]  T, rotated
 //   key/value history    [L][B][H][T][dh] T per block; keys rotated, at their
 //                        absolute positions, written when their chunk runs
-//   scores, dP           [H][b][ldS] fp32 for one sequence, ldS % 8 == 0
-//   P, dS                [H][b][ldS] T, zero outside the window
+//   score partials       [H][b][ntn][2] fp32 for one sequence; lse, D [H][b]
+//   P, dS                [H][b][ldS] T, zero outside the window, ldS % 8 == 0
 //   o, dq, dk, dv        [rows][d] fp32, token-major (head h at columns h*dh)
 //   rotary table         [T][dh/2] (cos, sin) fp32, angles in fp64
 #pragma once
@@ -75,6 +78,150 @@ struct EpiStoreHeads {
     }
   }
 };
+
+// Scores pass A: per (head, query) row and column part of the tile, the
+// online-softmax partial (max, sum exp) of scale * s over the keys inside the
+// window (empty parts give (-inf, 0)).  The scores never reach HBM.
+struct EpiScorePartial {
+  static constexpr bool kFixedHeadTile = true;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
+  struct RowState { float m, s; };
+  float* part;     // [H][b][ntn][2]
+  int b;
+  int ntn;
+  int64_t q0, j0;  // positions of query row 0 and key column 0
+  int window;
+  float scale;
+  __device__ void row_begin(RowState& st, int, int) const { st.m = -INFINITY; st.s = 0.f; }
+  __device__ void span(RowState& st, int, int r, int c0, const float* v, const float*, int nv) const {
+    const int64_t qpos = q0 + r;
+    float x[32];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int64_t dlt = qpos - (j0 + c0 + j);
+      x[j] = (j < nv && dlt >= 0 && dlt < window) ? v[j] * scale : -INFINITY;
+      mx = fmaxf(mx, x[j]);
+    }
+    if (mx == -INFINITY) return;
+    if (mx > st.m) { st.s *= expf(st.m - mx); st.m = mx; }
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc += expf(x[j] - st.m);
+    st.s += acc;
+  }
+  __device__ void row_end(RowState& st, int z, int r, int part_index) const {
+    float* p = part + (((int64_t)z * b + r) * ntn + part_index) * 2;
+    *reinterpret_cast<float2*>(p) = make_float2(st.m, st.s);
+  }
+};
+
+// Scores pass B: the probabilities from the recomputed scores and each row's
+// log-sum-exp, P = exp(scale * s - lse) inside the window, 0 outside; stored
+// in the operand type for P V and the backward.
+template <typename T>
+struct EpiScoreP {
+  static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
+  using RowState = NoRowState;
+  T* P;                // [H][b][ldS]
+  const float* lse;    // [H][b]
+  int b;
+  int ldS;
+  int64_t q0, j0;
+  int window;
+  float scale;
+  __device__ void row_begin(RowState&, int, int) const {}
+  __device__ void row_end(RowState&, int, int, int) const {}
+  __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
+    const int64_t row = (int64_t)z * b + r;
+    const float l = lse[row];
+    const int64_t qpos = q0 + r;
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int64_t dlt = qpos - (j0 + c0 + j);
+      x[j] = (dlt >= 0 && dlt < window) ? expf(v[j] * scale - l) : 0.f;
+    }
+    T* o = P + row * ldS + c0;
+    if (nv == 32 && (ldS & 7) == 0 && (c0 & 7) == 0) {
+      vst<32>(o, x);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) o[j] = from_f<T>(x[j]);
+    }
+  }
+};
+
+// dP epilogue: dS = P (dP - D) * scale from the kept probabilities and each
+// row's D = sum_e dO O, stored in the operand type; dP never reaches HBM.
+template <typename T>
+struct EpiDScore {
+  static constexpr bool kFixedHeadTile = false;
+  static constexpr bool kPreload = false;
+  static constexpr bool kWarpRows = false;
+  using RowState = NoRowState;
+  T* dS;               // [H][b][ldS]
+  const T* P;          // [H][b][ldS]
+  const float* D;      // [H][b]
+  int b;
+  int ldS;
+  float scale;
+  __device__ void row_begin(RowState&, int, int) const {}
+  __device__ void row_end(RowState&, int, int, int) const {}
+  __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
+    const int64_t row = (int64_t)z * b + r;
+    const float dd = D[row];
+    const T* pr = P + row * ldS + c0;
+    T* o = dS + row * ldS + c0;
+    float x[32];
+    if (nv == 32 && (ldS & 7) == 0 && (c0 & 7) == 0) {
+      float p[32];
+      vld<32>(pr, p);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = p[j] * (v[j] - dd) * scale;
+      vst<32>(o, x);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) if (j < nv) o[j] = from_f<T>(to_f<T>(pr[j]) * (v[j] - dd) * scale);
+    }
+  }
+};
+
+// Log-sum-exp of each (head, query) row from its pass-A partials.
+__global__ void attn_lse_kernel(const float* __restrict__ part, int ntn, int64_t rows, float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float2* p = reinterpret_cast<const float2*>(part + row * ntn * 2);
+  float m = -INFINITY;
+  for (int t = lane; t < ntn; t += 32) m = fmaxf(m, p[t].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+  for (int t = lane; t < ntn; t += 32) { const float2 q = p[t]; if (q.y > 0.f) sum += q.y * expf(q.x - m); }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) lse[row] = m + logf(sum);
+}
+
+// D = sum_e dO[e] O[e] over each head's columns, one warp per (head, query) of
+// one sequence.
+template <typename T>
+__global__ void attn_rowdot_kernel(const T* __restrict__ dO, const float* __restrict__ O, int rows, int b, int d,
+                                   int dh, float* __restrict__ D) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int h = (int)(row / b), i = (int)(row % b);
+  float acc = 0.f;
+  for (int e = lane; e < dh; e += 32) acc += to_f<T>(dO[row * dh + e]) * O[(int64_t)i * d + h * dh + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) D[row] = acc;
+}
 
 // LayerNorm with frozen gain and bias, one warp per row (two passes over the
 // row: mean, then the centred variance).  Keeps x_hat and 1/sigma for the
@@ -195,58 +342,6 @@ __global__ void rope_split_kernel(const float* __restrict__ qkv, const float2* _
     kh[hist + half + i] = from_f<T>(k1 * cs.y + k2 * cs.x);
     vh[hist + i] = from_f<T>(src[2 * d + i]);
     vh[hist + half + i] = from_f<T>(src[2 * d + half + i]);
-  }
-}
-
-// Window-masked softmax of one sequence's scores, one warp per (head, query):
-// query at position q0 + i sees the keys at positions j0 + j with
-// 0 <= (q0 + i) - (j0 + j) < window.  P is zero elsewhere, pad columns included.
-template <typename T>
-__global__ void attn_softmax_kernel(const float* __restrict__ S, T* __restrict__ P, int rows, int b, int nk,
-                                    int ldS, int64_t q0, int64_t j0, int window, float scale) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int i = (int)(row % b);
-  const int64_t qpos = q0 + i;
-  const int hi = (int)(qpos - j0);                                   // last visible column
-  int lo = (int)(qpos - window + 1 - j0);
-  if (lo < 0) lo = 0;
-  const float* sr = S + row * ldS;
-  T* pr = P + row * ldS;
-  float m = -INFINITY;
-  for (int j = lo + lane; j <= hi; j += 32) m = fmaxf(m, sr[j] * scale);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float sum = 0.f;
-  for (int j = lo + lane; j <= hi; j += 32) sum += expf(sr[j] * scale - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float inv = 1.f / sum;
-  for (int j = lane; j < ldS; j += 32)
-    pr[j] = from_f<T>((j >= lo && j <= hi) ? expf(sr[j] * scale - m) * inv : 0.f);
-}
-
-// Softmax backward of one sequence, one warp per (head, query):
-// dS = P (dP - D) * scale with D = sum_e dO[e] O[e] over the head's columns.
-template <typename T>
-__global__ void attn_dsoftmax_kernel(const float* __restrict__ dP, const T* __restrict__ P,
-                                     const T* __restrict__ dO, const float* __restrict__ O, T* __restrict__ dS,
-                                     int rows, int b, int ldS, int d, int dh, float scale) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int h = (int)(row / b), i = (int)(row % b);
-  float D = 0.f;
-  for (int e = lane; e < dh; e += 32) D += to_f<T>(dO[row * dh + e]) * O[(int64_t)i * d + h * dh + e];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
-  const float* gr = dP + row * ldS;
-  const T* pr = P + row * ldS;
-  T* sr = dS + row * ldS;
-  for (int j = lane; j < ldS; j += 32) {
-    const float p = to_f<T>(pr[j]);
-    sr[j] = from_f<T>(p == 0.f ? 0.f : p * (gr[j] - D) * scale);
   }
 }
 

@@ -122,8 +122,9 @@ struct Plan {
   size_t sk_partial_bytes, sk_counter_count;
   // frozen sliding-window attention (attn_heads > 0)
   int H, dh, window, ldS;
-  size_t rope_tab, xhat, lnr, qkv, qh, kh, vh, S, Pa, Of, Oc, dOh, dSa, dq, dk, dv, dqkv, da, sdout[2], sdoutT[2][2],
-      sdU[2];
+  int ntnS;   // score partials per (head, query) row
+  size_t rope_tab, xhat, lnr, qkv, qh, kh, vh, spart, slse, sD, Pa, Of, Oc, dOh, dSa, dq, dk, dv, dqkv, da, sdout[2],
+      sdoutT[2][2], sdU[2];
 };
 
 static inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -193,8 +194,8 @@ static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
   p.yk = take(p.recon ? 4 * n * d : 0);
   p.yq = take(p.recon ? 4 * n * d : 0);
   p.qres = take(p.recon ? 4 * n * d : 0);
-  // split-K scratch of the CTA-pair GEMMs (only when 256-row pair tiles exist)
-  p.sk_partial_bytes = (c.precision == TTT_PREC_BF16 && n >= 256) ? std::min<size_t>(64ull << 20, 64ull * 1024 * n) : 0;
+  // split-K scratch of the CTA-pair GEMMs (bf16 path)
+  p.sk_partial_bytes = c.precision == TTT_PREC_BF16 ? std::min<size_t>(64ull << 20, 64ull * 1024 * std::max<size_t>(n, 64)) : 0;
   p.sk_counter_count = p.sk_partial_bytes ? 65536 : 0;
   p.sk_partial = take(p.sk_partial_bytes);
   p.sk_counters = take(4 * p.sk_counter_count);
@@ -216,7 +217,10 @@ static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
     p.qh = take(e * L * n * d);
     p.kh = take(e * L * B * T * d);
     p.vh = take(e * L * B * T * d);
-    p.S = take(4 * H * b * ldS);
+    p.ntnS = head_parts(c.precision, p.ldS);
+    p.spart = take(8 * H * b * (size_t)p.ntnS);
+    p.slse = take(4 * H * b);
+    p.sD = take(4 * H * b);
     p.Pa = take(e * L * B * H * b * ldS);
     p.Of = take(4 * L * n * d);
     p.Oc = take(e * n * d);
@@ -629,7 +633,9 @@ static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const floa
   T* qh = reinterpret_cast<T*>(ws + p.qh);
   T* kh = reinterpret_cast<T*>(ws + p.kh);
   T* vh = reinterpret_cast<T*>(ws + p.vh);
-  float* Sc = reinterpret_cast<float*>(ws + p.S);
+  float* spart = reinterpret_cast<float*>(ws + p.spart);
+  float* slse = reinterpret_cast<float*>(ws + p.slse);
+  float* sD = reinterpret_cast<float*>(ws + p.sD);
   T* Pa = reinterpret_cast<T*>(ws + p.Pa);
   float* Of = reinterpret_cast<float*>(ws + p.Of);
   T* Oc = reinterpret_cast<T*>(ws + p.Oc);
@@ -714,15 +720,21 @@ static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const floa
         T* vs = vb + (int64_t)s * H * Tn * dh + j0 * dh;
         T* ps = Pa + l * pblk + (int64_t)s * H * b * ldS;
         {
+          // pass A: masked (max, sum exp) partials per row and column part;
+          // pass B recomputes the scores and writes P = exp(scale s - lse)
           GemmShape g{b, nk, dh, H};
-          LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 4.0 * H * b * nk,
-                 TRY((gemm<T, 1>(g, opnd(qs, dh, (int64_t)b * dh, 1, b), opnd(qs, dh, (int64_t)b * dh, 1, b),
-                                 opnd(ks, dh, Tn * dh, 1, nk), EpiStoreBatched{Sc, ldS, (int64_t)b * ldS}, st,
-                                 status, ss))));
+          const int ntn = head_parts(hd->cfg.precision, nk);
+          Operand Aq = opnd(qs, dh, (int64_t)b * dh, 1, b);
+          Operand Bk = opnd(ks, dh, Tn * dh, 1, nk);
+          LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 8.0 * H * b * ntn,
+                 TRY((gemm<T, 1>(g, Aq, Aq, Bk, EpiScorePartial{spart, b, ntn, q0, j0, p.window, scale}, st, status,
+                                 ss))));
+          LAUNCH(K_ATTN_ROWS, 0, 8.0 * H * b * ntn + 4.0 * H * b,
+                 (attn_lse_kernel<<<(H * b + 7) / 8, 256, 0, st>>>(spart, ntn, (int64_t)H * b, slse)));
+          LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + e * H * b * nk,
+                 TRY((gemm<T, 1>(g, Aq, Aq, Bk, EpiScoreP<T>{ps, slse, b, ldS, q0, j0, p.window, scale}, st, status,
+                                 ss))));
         }
-        LAUNCH(K_ATTN_ROWS, 0, (4.0 + e) * H * b * nk,
-               (attn_softmax_kernel<T><<<(H * b + 7) / 8, 256, 0, st>>>(Sc, ps, H * b, b, nk, ldS, q0, j0,
-                                                                        p.window, scale)));
         {
           GemmShape g{b, dh, nk, H};
           LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b * nk + (double)nk * dh) * H + 4.0 * b * d,
@@ -871,16 +883,17 @@ static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const floa
           T* vs = vb + (int64_t)s * H * Tn * dh + j0 * dh;
           T* ps = Pa + l * pblk + (int64_t)s * H * b * ldS;
           T* dos = dOh + (int64_t)s * H * b * dh;
+          LAUNCH(K_ATTN_ROWS, 0, (e + 4.0) * H * b * dh + 4.0 * H * b,
+                 (attn_rowdot_kernel<T><<<(H * b + 7) / 8, 256, 0, st>>>(dos, ob + (int64_t)s * b * d, H * b, b, d, dh,
+                                                                         sD)));
           {
+            // dP = dO V^T, turned into dS = P (dP - D) scale in the epilogue
             GemmShape g{b, nk, dh, H};
-            LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 4.0 * H * b * nk,
+            LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 2.0 * e * H * b * nk,
                    TRY((gemm<T, 1>(g, opnd(dos, dh, (int64_t)b * dh, 1, b), opnd(dos, dh, (int64_t)b * dh, 1, b),
-                                   opnd(vs, dh, Tn * dh, 1, nk), EpiStoreBatched{Sc, ldS, (int64_t)b * ldS}, st,
-                                   status, ss))));
+                                   opnd(vs, dh, Tn * dh, 1, nk), EpiDScore<T>{dSa, ps, sD, b, ldS, scale}, st, status,
+                                   ss))));
           }
-          LAUNCH(K_ATTN_ROWS, 0, (4.0 + 2.0 * e) * H * b * nk,
-                 (attn_dsoftmax_kernel<T><<<(H * b + 7) / 8, 256, 0, st>>>(Sc, ps, dos, ob + (int64_t)s * b * d, dSa,
-                                                                           H * b, b, ldS, d, dh, scale)));
           {
             GemmShape g{b, dh, nk, H};
             LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b * nk + (double)nk * dh) * H + 4.0 * b * d,
