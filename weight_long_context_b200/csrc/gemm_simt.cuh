@@ -49,20 +49,41 @@ gemm_simt_kernel(GemmShape s, Operand A, Operand A2, Operand B, Epi epi, int dua
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[a][i][j] = 0.f;
 
-  for (int k0 = 0; k0 < s.K; k0 += BK) {
+  // The next k-tile's operands are loaded into registers while the current
+  // tile is multiplied (one global-load latency per tile is hidden).
+  constexpr int PER = (BM * BK) / THREADS;
+  float ra[2][PER], rb[PER];
+  auto load_tile = [&](int k0) {
 #pragma unroll
-    for (int i = 0; i < (BM * BK) / THREADS; ++i) {
-      int idx = tid + i * THREADS;
-      int mm, kk;
+    for (int i = 0; i < PER; ++i) {
+      const int idx = tid + i * THREADS;
+      int mm, kk, nn;
       if (A.kmajor) { mm = idx / BK; kk = idx % BK; } else { kk = idx / BM; mm = idx % BM; }
-      As[0][kk][mm] = simt_load<T>(A, z, m0 + mm, k0 + kk, s.M, s.K);
-      if (NACC == 2 && !dualb) As[NACC - 1][kk][mm] = simt_load<T>(A2, z, m0 + mm, k0 + kk, s.M, s.K);
-      int nn;
+      ra[0][i] = simt_load<T>(A, z, m0 + mm, k0 + kk, s.M, s.K);
+      if (NACC == 2 && !dualb) ra[1][i] = simt_load<T>(A2, z, m0 + mm, k0 + kk, s.M, s.K);
       if (B.kmajor) { nn = idx / BK; kk = idx % BK; } else { kk = idx / BN; nn = idx % BN; }
-      Bs[kk][nn] = simt_load<T>(B, z, n0 + nn, k0 + kk, s.N, s.K);
-      if (NACC == 2 && dualb) As[NACC - 1][kk][nn] = simt_load<T>(A2, z, n0 + nn, k0 + kk, s.N, s.K);
+      rb[i] = simt_load<T>(B, z, n0 + nn, k0 + kk, s.N, s.K);
+      if (NACC == 2 && dualb) ra[1][i] = simt_load<T>(A2, z, n0 + nn, k0 + kk, s.N, s.K);
     }
+  };
+  auto store_tile = [&]() {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int idx = tid + i * THREADS;
+      int mm, kk, nn;
+      if (A.kmajor) { mm = idx / BK; kk = idx % BK; } else { kk = idx / BM; mm = idx % BM; }
+      As[0][kk][mm] = ra[0][i];
+      if (NACC == 2 && !dualb) As[NACC - 1][kk][mm] = ra[1][i];
+      if (B.kmajor) { nn = idx / BK; kk = idx % BK; } else { kk = idx / BN; nn = idx % BN; }
+      Bs[kk][nn] = rb[i];
+      if (NACC == 2 && dualb) As[NACC - 1][kk][nn] = ra[1][i];
+    }
+  };
+  if (s.K > 0) load_tile(0);
+  for (int k0 = 0; k0 < s.K; k0 += BK) {
+    store_tile();
     __syncthreads();
+    if (k0 + BK < s.K) load_tile(k0 + BK);
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {
       float b[NACC][4];

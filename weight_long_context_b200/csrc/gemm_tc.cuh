@@ -832,7 +832,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;
     constexpr int PART_COLS = BN / C::PARTS;
-    const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     float* sv = rowstage + (warp - 2) * 1024;   // row-walk staging (row-walking epilogues only)
@@ -1191,7 +1190,7 @@ inline long paired_finish_plan(long tiles, int num_kb, const SplitScratch& ss, d
 // Split count for a pair-kernel GEMM: minimise waves x (k-blocks per split +
 // a fixed cost for parking and reducing a partial), with no empty split and
 // within the partial-tile scratch.
-inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
+inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss, double* cost_out = nullptr) {
   static int forced = -1;
   if (forced < 0) {
     const char* e = getenv("TTT_GEMM_SPLITS");   // tuning knob: force a split count
@@ -1209,7 +1208,10 @@ inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
   // Measured on B200: splitting pays only when unsplit tiles leave most pairs
   // idle; with 1-2 waves of tiles the partial round trip costs more than the
   // quantisation it removes.
-  if (tiles >= (long)(0.6 * pairs)) return 1;
+  if (tiles >= (long)(0.6 * pairs)) {
+    if (cost_out) *cost_out = (double)((tiles + pairs - 1) / pairs) * num_kb;
+    return 1;
+  }
   int best = 1;
   double best_cost = 1e30;
   for (int S = 1; S <= 8 && S <= num_kb; ++S) {
@@ -1226,6 +1228,7 @@ inline int choose_splits(long tiles, int num_kb, const SplitScratch& ss) {
     const double cost = (double)waves * (kbps + (S > 1 ? 4 : 0));
     if (cost < best_cost - 1e-9) { best_cost = cost; best = S; }
   }
+  if (cost_out) *cost_out = best_cost;
   return best;
 }
 
@@ -1265,7 +1268,10 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   p.num_kb = (s.K + BK - 1) / BK;
   p.status = status;
   const bool may_split = NACC == 1 && BN == 256;
-  const long full = may_split ? paired_finish_plan(p.num_tiles, p.num_kb, ss) : -1;
+  double pf_cost = 0.0, split_cost = 1e30;
+  long full = may_split ? paired_finish_plan(p.num_tiles, p.num_kb, ss, &pf_cost) : -1;
+  const int split_S = may_split ? choose_splits(p.num_tiles, p.num_kb, ss, &split_cost) : 1;
+  if (full >= 0 && split_S > 1 && split_cost < pf_cost) full = -1;   // few tiles, long K: plain split-K
   if (full >= 0) {   // whole waves, then the last wave's tiles as paired halves
     p.pair_finish = 1;
     p.full_tiles = (int)full;
@@ -1275,7 +1281,7 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   } else {
     p.pair_finish = 0;
     p.full_tiles = p.num_tiles;
-    p.splits = may_split ? choose_splits(p.num_tiles, p.num_kb, ss) : 1;
+    p.splits = split_S;
     p.kb_per_split = (p.num_kb + p.splits - 1) / p.splits;
     p.num_units = p.num_tiles * p.splits;
   }
@@ -1320,6 +1326,17 @@ cudaError_t launch_gemm_tc(const GemmShape& s, const Operand& A, const Operand& 
     // the tile shape under the operand-feed limit (pair 256x256: 1.3,
     // 1-SM 128x256: 1.0, 1-SM 128x128: 0.78, already in tile_efficiency).
     // The pair kernel may split K, which lifts its occupancy.
+    // A few row tiles and a long K (the cross-entropy dz of a short chunk:
+    // M = b rows, K = the vocabulary): one SM per tile would walk the whole K
+    // alone, so the pair kernel runs it split over K across many pairs
+    // (its 256-row tile reads zeros past row M and stores only rows < M).
+    if (pair_mode() && s.M <= BM && ss.partial && ss.counters) {
+      const long ptiles = (long)((s.N + 255) / 256) * s.batch;
+      const int num_kb = (s.K + BK - 1) / BK;
+      // measured on B200: pays from K = 8192 (128 k-blocks: 49.6 -> 31 us for
+      // the dz of a 64-row chunk), loses at K = 2048 (20.9 -> 29.4 us)
+      if (ptiles * 4 <= num_sms() / 2 && num_kb >= 64) return launch_tc2<1, 256, Epi>(s, A, A2, B, epi, st, status, ss);
+    }
     double s_pair = 0.0;
     if (pair_mode() && s.M > BM) {
       const long tiles = (long)((s.M + 2 * BM - 1) / (2 * BM)) * ((s.N + 255) / 256) * s.batch;
