@@ -107,6 +107,11 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
+// Bring a kernel-parameter tensor map into the TMA unit's descriptor cache
+// ahead of the first copy that uses it.
+__device__ __forceinline__ void tmap_prefetch(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -258,6 +263,26 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   return x;
 }
 
+// Tile t -> (row tile tm, column tile tn, batch entry z).  Consecutive tiles
+// run on consecutive CTAs (pairs) at the same time.  The GEMMs walk row tiles
+// first (the tiles in flight share a column block of B); the two-accumulator
+// state update walks column tiles first, so the state rows it streams at once
+// are whole rows (measured on B200: 3 % faster than row tiles first).
+template <int NACC>
+__device__ __forceinline__ void decode_tile(const TcParams& p, int t, int& tm, int& tn, int& z) {
+  if constexpr (NACC == 2) {
+    tn = t % p.tiles_n;
+    const int rest = t / p.tiles_n;
+    tm = rest % p.tiles_m;
+    z = rest / p.tiles_m;
+  } else {
+    tm = t % p.tiles_m;
+    const int rest = t / p.tiles_m;
+    tn = rest % p.tiles_n;
+    z = rest / p.tiles_n;
+  }
+}
+
 // Row-walking epilogues.  The accumulators arrive one row per thread (the
 // TMEM lane layout); global rows are contiguous, so a thread writing its own
 // row would touch 32 separate lines per warp instruction.  Instead each warp
@@ -372,10 +397,8 @@ __device__ __forceinline__ void warp_rows_loop(const Epi& epi, const TcParams& p
     const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
     if (!ready) break;
     tc_fence_after();
-    const int tm = t % p.tiles_m;
-    const int rest = t / p.tiles_m;
-    const int tn = rest % p.tiles_n;
-    const int z = rest / p.tiles_n;
+    int tm, tn, z;
+    decode_tile<NACC>(p, t, tm, tn, z);
     const int row0 = tm * rows_per_tile + row_off + q * 32;
     const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + buf * (NACC * BN);
     rows_tile<NACC, BN, PART_COLS>(epi, p.s, z, row0, tn, tbase, sv, part, lane, [&]() { release(buf); });
@@ -402,6 +425,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    tmap_prefetch(&mapA);
+    tmap_prefetch(&mapA2);
+    tmap_prefetch(&mapB);
     for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 32 * C::EW); }
     mbar_init(drain, 1);
@@ -422,10 +448,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       uint32_t it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const int tm = t % p.tiles_m;
-        const int rest = t / p.tiles_m;
-        const int tn = rest % p.tiles_n;
-        const int z = rest / p.tiles_n;
+        int tm, tn, z;
+        decode_tile<NACC>(p, t, tm, tn, z);
         const int m0 = tm * BM, n0 = tn * BN;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const int st = it % C::STAGES;
@@ -544,10 +568,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
     } else {
       uint32_t tcount = 0;
       for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
-        const int tm = t % p.tiles_m;
-        const int rest = t / p.tiles_m;
-        const int tn = rest % p.tiles_n;
-        const int z = rest / p.tiles_n;
+        int tm, tn, z;
+        decode_tile<NACC>(p, t, tm, tn, z);
         const uint32_t buf = tcount & 1u;
         const uint32_t aph = (tcount >> 1) & 1u;
         // Warp-uniform decision: tcgen05.ld below is .sync.aligned.
@@ -708,6 +730,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   const int npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
+    tmap_prefetch(&mapA);
+    tmap_prefetch(&mapA2);
+    tmap_prefetch(&mapB);
     for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2 * 32 * C::EW); }
     mbar_init(drain, 1);
@@ -729,10 +754,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
       for (int u = pair; u < p.num_units && ok; u += npairs) {
         const Unit un = decode_unit(p, u);
         const int t = un.t;
-        const int tm = t % p.tiles_m;
-        const int rest = t / p.tiles_m;
-        const int tn = rest % p.tiles_n;
-        const int z = rest / p.tiles_n;
+        int tm, tn, z;
+        decode_tile<NACC>(p, t, tm, tn, z);
         const int m0 = tm * 2 * BM + (int)rank * BM;     // this CTA's 128 rows
         const int n0 = tn * BN + (int)rank * HBN;        // this CTA's BN/2 columns
         for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
@@ -845,10 +868,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
     for (int u = pair; u < p.num_units; u += npairs, ++tcount) {
       const Unit un = decode_unit(p, u);
       const int t = un.t, ks = un.ks;
-      const int tm = t % p.tiles_m;
-      const int rest = t / p.tiles_m;
-      const int tn = rest % p.tiles_n;
-      const int z = rest / p.tiles_n;
+      int tm, tn, z;
+      decode_tile<NACC>(p, t, tm, tn, z);
       const uint32_t buf = tcount & 1u;
       const uint32_t aph = (tcount >> 1) & 1u;
       const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aph, abort_flag, p.status));
