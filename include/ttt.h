@@ -156,6 +156,34 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b,
                        const float* eta, const float* beta, const float* gamma,
                        float* chunk_loss, void* workspace, size_t ws_bytes, void* stream);
 
+/* ttt_prefill on HOST buffers, end to end: the inputs go to the device and the
+ * results come back inside the call, which returns once W, M and chunk_loss
+ * are in host memory.  Same operation as ttt_prefill ([TTT-E2E] 内层循环:
+ * 测试时训练; [E2-TTT] Algorithm 1, Proposition 3.1).
+ *   hidden [batch, T, d], tokens [batch, T], eta/beta/gamma [batch, T]:
+ *     host arrays, read only.
+ *   W0, M0: host arrays (packed as for ttt_prefill), the initial state, read
+ *     only; W, M: host arrays receiving the final state (they may be W0 and
+ *     M0 themselves).  chunk_loss [batch, T/b]: host, written.
+ *   seg_chunks: the sequence is streamed in segments of seg_chunks chunks
+ *     (0: about 8 segments); segment s + 1's inputs are copied while segment
+ *     s runs, through two device slots.  With attention blocks the whole
+ *     sequence is one segment (a chunk reads earlier chunks' keys).  Chunk-end
+ *     state is the only carried state, so the result is ttt_prefill's bit for
+ *     bit whatever the segment length.
+ *   device_buffer: caller-owned device memory of ttt_host_buffer_size() bytes,
+ *     256-byte aligned (state, losses, two input slots, the workspace).
+ * Copies overlap the compute only from page-locked (pinned) host memory;
+ * pageable buffers work but serialise the copies.  Argument errors return
+ * without copying or launching; device-side errors go to the status word
+ * (ttt_get_device_status).  The call synchronises `stream`. */
+ttt_status ttt_host_buffer_size(const ttt_handle* h, int32_t batch, int32_t T, int32_t b, int32_t seg_chunks,
+                                size_t* bytes);
+ttt_status ttt_prefill_host(ttt_handle* h, int32_t batch, int32_t T, int32_t b, int32_t seg_chunks,
+                            const float* hidden, const int32_t* tokens, const float* W0, const float* M0, float* W,
+                            float* M, const float* eta, const float* beta, const float* gamma, float* chunk_loss,
+                            void* device_buffer, size_t buffer_bytes, void* stream);
+
 /* ttt_prefill without a caller-provided workspace and without allocating:
  * for callers that must not allocate device memory while they run (memory
  * budgeted once at start-up, a host that owns the allocator, or a loop that

@@ -288,6 +288,23 @@ def test_resume_and_determinism_bitwise(dev):
     assert np.array_equal(np.concatenate([L1, L2], axis=1), La)
 
 
+@pytest.mark.parametrize("seg", [0, 1, 3])
+def test_host_prefill_matches_device_prefill_bitwise(dev, seg):
+    """ttt_prefill_host streams the sequence in segments of seg chunks with
+    the copies overlapping the compute; chunk-end state is the only carried
+    state, so it must give ttt_prefill's results bit for bit (two sequences:
+    strided segment copies; seg = 3 of 4 chunks leaves a ragged last segment)."""
+    w = W("batched_16", T=1024, batch=2)
+    x = I.make_inputs(w, seed=2, m0_scale=1e-3, w0_per_sequence=True)
+    Wa, Ma, La, st, h = H.run_gpu(w, x, dev, return_handle=True)
+    pin = lambda a, dt=None: torch.from_numpy(np.ascontiguousarray(a if dt is None else a.astype(dt))).pin_memory()
+    Wh, Mh, Lh = h.prefill_host(pin(x["hidden"]), pin(x["tokens"], np.int32), pin(x["W0"]), pin(x["M0"]),
+                                pin(x["eta"]), pin(x["beta"]), pin(x["gamma"]), w.b, seg_chunks=seg)
+    assert h.device_status() == 0
+    assert np.array_equal(Wh.numpy(), Wa) and np.array_equal(Mh.numpy(), Ma) and np.array_equal(Lh.numpy(), La)
+    h.close()
+
+
 def test_zero_head_gives_log_v(dev):
     w = I.Workload("zh", 64, 96, 160, 1, "swiglu", False, "bf16", 64, 32, 1, "e2ttt")
     x = I.make_inputs(w, seed=1, m0_scale=0.01)

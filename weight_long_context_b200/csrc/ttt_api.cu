@@ -79,7 +79,9 @@ struct GraphSlot {
   CallKey key;
   bool have = false;
 };
-enum { SLOT_PREFILL, SLOT_RECON, SLOT_PREDICT, N_SLOTS };
+// SLOT_HOST0/1: the host-buffer prefill's segments in input slot 0 / 1;
+// SLOT_HOST_LAST: its last segment when that one is shorter.
+enum { SLOT_PREFILL, SLOT_RECON, SLOT_PREDICT, SLOT_HOST0, SLOT_HOST1, SLOT_HOST_LAST, N_SLOTS };
 
 }  // namespace ttt
 
@@ -92,6 +94,10 @@ struct ttt_handle {
   int* status = nullptr;    // device status word
   int* zero_flag = nullptr; // a device int that stays 0 (bounded-wait self-test)
   cudaStream_t cap = nullptr;
+  // host-buffer prefill: copy stream and the two input slots' events
+  cudaStream_t copy = nullptr;
+  cudaEvent_t ev_copied[2] = {nullptr, nullptr};
+  cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
   ttt::GraphSlot graph[ttt::N_SLOTS];
   bool use_graph = true;
   // Frozen sliding-window attention in front of every updated block
@@ -1322,6 +1328,134 @@ static ttt_status noalloc_scratch(void** out) {
 }
 
 // ---------------------------------------------------------------------------
+// Host-buffer prefill: the sequence in segments of whole chunks, the copy of
+// segment s + 1's inputs (and of s + 2's, once slot s's compute is done)
+// overlapping the compute of segment s.  Chunk-end state is the only carried
+// state, so running the segments one after another on the same W and M gives
+// the whole call's result bit for bit.
+// ---------------------------------------------------------------------------
+struct HostPlan {
+  int seg_chunks = 0, nseg = 0, segT = 0, nchunks = 0;
+  int64_t per_seq = 0;               // fast-weight parameters per sequence
+  size_t W = 0, M = 0, loss = 0;     // offsets in the device buffer
+  size_t slot[2] = {0, 0};           // input slots
+  size_t hid = 0, tok = 0, eta = 0, beta = 0, gamma = 0;   // offsets inside a slot
+  size_t ws = 0, ws_bytes = 0, total = 0;
+};
+
+static HostPlan make_host_plan(const ttt_handle* h, int B, int T, int b, int seg_chunks) {
+  HostPlan q;
+  q.nchunks = b > 0 ? T / b : 0;
+  if (seg_chunks <= 0) seg_chunks = std::max(1, (q.nchunks + 7) / 8);
+  // with attention a chunk reads the keys of earlier chunks, kept in the
+  // workspace for one call: the whole sequence is one segment
+  if (h->attn_heads > 0) seg_chunks = q.nchunks;
+  seg_chunks = std::max(1, std::min(seg_chunks, std::max(q.nchunks, 1)));
+  q.seg_chunks = seg_chunks;
+  q.segT = seg_chunks * b;
+  q.nseg = q.nchunks > 0 ? (q.nchunks + seg_chunks - 1) / seg_chunks : 0;
+  const int m = h->cfg.mlp == TTT_MLP_SWIGLU ? 3 : 2;
+  q.per_seq = (int64_t)h->cfg.n_blocks * m * h->cfg.hidden * h->cfg.d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  q.W = take(4ull * B * q.per_seq);
+  q.M = take(4ull * B * q.per_seq);
+  q.loss = take(2 * 4ull * B * seg_chunks);   // one [B][seg_chunks] block per input slot
+  const size_t n = (size_t)B * q.segT;
+  size_t so = 0;
+  auto stake = [&](size_t bytes) { size_t o = so; so = align_up(so + bytes, 256); return o; };
+  q.hid = stake(4 * n * h->cfg.d);
+  q.tok = stake(4 * n);
+  q.eta = stake(4 * n);
+  q.beta = stake(4 * n);
+  q.gamma = stake(4 * n);
+  q.slot[0] = take(so);
+  q.slot[1] = take(so);
+  q.ws_bytes = make_plan(h, B, q.segT, b).total;
+  q.ws = take(q.ws_bytes);
+  q.total = off;
+  return q;
+}
+
+static ttt_status prefill_host_impl(ttt_handle* h, int B, int T, int b, const float* hidden, const int32_t* tokens,
+                                    const float* W0, const float* M0, float* W, float* M, const float* eta,
+                                    const float* beta, const float* gamma, float* chunk_loss, char* buf,
+                                    const HostPlan& q, cudaStream_t st) {
+  if (!h->copy) {
+    TTT_CUDA_TRY(cudaStreamCreateWithFlags(&h->copy, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      TTT_CUDA_TRY(cudaEventCreateWithFlags(&h->ev_copied[i], cudaEventDisableTiming));
+      TTT_CUDA_TRY(cudaEventCreateWithFlags(&h->ev_consumed[i], cudaEventDisableTiming));
+    }
+  }
+  const int64_t d = h->cfg.d;
+  const size_t state = 4ull * B * q.per_seq;
+  float* Wd = reinterpret_cast<float*>(buf + q.W);
+  float* Md = reinterpret_cast<float*>(buf + q.M);
+  TTT_CUDA_TRY(cudaMemcpyAsync(Wd, W0, state, cudaMemcpyHostToDevice, st));
+  TTT_CUDA_TRY(cudaMemcpyAsync(Md, M0, state, cudaMemcpyHostToDevice, st));
+  // segment s: chunks [s * seg_chunks, ...), Ts tokens per sequence
+  auto seg_T = [&](int s) { return std::min(q.seg_chunks, q.nchunks - s * q.seg_chunks) * b; };
+  auto copy_in = [&](int s) -> ttt_status {
+    const int slot = s & 1;
+    char* sb = buf + q.slot[slot];
+    const size_t t0 = (size_t)s * q.segT, Ts = (size_t)seg_T(s);
+    TTT_CUDA_TRY(cudaMemcpy2DAsync(sb + q.hid, 4 * Ts * d, hidden + t0 * d, 4 * (size_t)T * d, 4 * Ts * d, B,
+                                   cudaMemcpyHostToDevice, h->copy));
+    const void* src[4] = {tokens + t0, eta + t0, beta + t0, gamma + t0};
+    const size_t dst[4] = {q.tok, q.eta, q.beta, q.gamma};
+    for (int i = 0; i < 4; ++i)
+      TTT_CUDA_TRY(cudaMemcpy2DAsync(sb + dst[i], 4 * Ts, src[i], 4 * (size_t)T, 4 * Ts, B, cudaMemcpyHostToDevice,
+                                     h->copy));
+    TTT_CUDA_TRY(cudaEventRecord(h->ev_copied[slot], h->copy));
+    return TTT_OK;
+  };
+  ttt_status s0 = copy_in(0);
+  if (s0 != TTT_OK) return s0;
+  if (q.nseg > 1 && (s0 = copy_in(1)) != TTT_OK) return s0;
+  char* ws = buf + q.ws;
+  for (int s = 0; s < q.nseg; ++s) {
+    const int slot = s & 1;
+    const int Ts = seg_T(s);
+    const size_t nc = (size_t)Ts / b;
+    char* sb = buf + q.slot[slot];
+    float* loss_s = reinterpret_cast<float*>(buf + q.loss) + (size_t)slot * B * q.seg_chunks;
+    TTT_CUDA_TRY(cudaStreamWaitEvent(st, h->ev_copied[slot], 0));
+    Plan p = make_plan(h, B, Ts, b);
+    Prof prof;
+    const float* hid = reinterpret_cast<const float*>(sb + q.hid);
+    const int* tok = reinterpret_cast<const int*>(sb + q.tok);
+    const float* et = reinterpret_cast<const float*>(sb + q.eta);
+    const float* be = reinterpret_cast<const float*>(sb + q.beta);
+    const float* ga = reinterpret_cast<const float*>(sb + q.gamma);
+    auto enqueue = [&](cudaStream_t qs) -> cudaError_t {
+      return enqueue_lm(h, p, hid, tok, Wd, Md, et, be, ga, loss_s, ws, qs, prof);
+    };
+    // one cached graph per input slot (and one for a shorter last segment):
+    // the same pointers every segment and every call with these sizes
+    CallKey key;
+    key.batch = B; key.T = Ts; key.b = b; key.ws_bytes = q.ws_bytes;
+    const void* ptrs[] = {hid, tok, Wd, Md, et, be, ga, loss_s, ws};
+    std::copy(std::begin(ptrs), std::end(ptrs), key.ptr);
+    const int gslot = Ts != q.segT ? SLOT_HOST_LAST : (slot ? SLOT_HOST1 : SLOT_HOST0);
+    ttt_status r = run_graph(h, gslot, key, enqueue, st);
+    if (r != TTT_OK) return r;
+    // this segment's chunk losses out before the slot's next segment overwrites them
+    TTT_CUDA_TRY(cudaMemcpy2DAsync(chunk_loss + (size_t)s * q.seg_chunks, 4 * (size_t)q.nchunks, loss_s, 4 * nc,
+                                   4 * nc, B, cudaMemcpyDeviceToHost, st));
+    TTT_CUDA_TRY(cudaEventRecord(h->ev_consumed[slot], st));
+    if (s + 2 < q.nseg) {
+      TTT_CUDA_TRY(cudaStreamWaitEvent(h->copy, h->ev_consumed[slot], 0));
+      if ((s0 = copy_in(s + 2)) != TTT_OK) return s0;
+    }
+  }
+  TTT_CUDA_TRY(cudaMemcpyAsync(W, Wd, state, cudaMemcpyDeviceToHost, st));
+  TTT_CUDA_TRY(cudaMemcpyAsync(M, Md, state, cudaMemcpyDeviceToHost, st));
+  TTT_CUDA_TRY(cudaStreamSynchronize(st));
+  return TTT_OK;
+}
+
+// ---------------------------------------------------------------------------
 // C ABI
 // ---------------------------------------------------------------------------
 extern "C" {
@@ -1409,6 +1543,11 @@ void ttt_destroy(ttt_handle* h) {
   if (h->ln_gain) cudaFree(h->ln_gain);
   if (h->ln_bias) cudaFree(h->ln_bias);
   if (h->status) cudaFree(h->status);
+  if (h->copy) { cudaStreamSynchronize(h->copy); cudaStreamDestroy(h->copy); }
+  for (int i = 0; i < 2; ++i) {
+    if (h->ev_copied[i]) cudaEventDestroy(h->ev_copied[i]);
+    if (h->ev_consumed[i]) cudaEventDestroy(h->ev_consumed[i]);
+  }
   if (h->cap) cudaStreamDestroy(h->cap);
   delete h;
 }
@@ -1498,6 +1637,37 @@ ttt_status ttt_prefill(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const
   const void* ptrs[] = {hidden, tokens, W, M, eta, beta, gamma, chunk_loss, workspace};
   std::copy(std::begin(ptrs), std::end(ptrs), key.ptr);
   return run_graph(h, SLOT_PREFILL, key, enqueue, st);
+}
+
+ttt_status ttt_host_buffer_size(const ttt_handle* h, int32_t batch, int32_t T, int32_t b, int32_t seg_chunks,
+                                size_t* bytes) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (!bytes) return fail(TTT_ERR_INVALID_ARG, "bytes is NULL");
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the host-buffer prefill serves the LM head");
+  *bytes = make_host_plan(h, batch, T, b, seg_chunks).total;
+  return TTT_OK;
+}
+
+ttt_status ttt_prefill_host(ttt_handle* h, int32_t batch, int32_t T, int32_t b, int32_t seg_chunks,
+                            const float* hidden, const int32_t* tokens, const float* W0, const float* M0, float* W,
+                            float* M, const float* eta, const float* beta, const float* gamma, float* chunk_loss,
+                            void* device_buffer, size_t buffer_bytes, void* stream) {
+  ttt_status s = check_shape(h, batch, T, b);
+  if (s != TTT_OK) return s;
+  if (h->cfg.head != TTT_HEAD_LM) return fail(TTT_ERR_UNSUPPORTED, "the host-buffer prefill serves the LM head");
+  if (batch == 0 || T == 0) return TTT_OK;
+  if (!hidden || !tokens || !W0 || !M0 || !W || !M || !eta || !beta || !gamma || !chunk_loss)
+    return fail(TTT_ERR_INVALID_ARG, "a required pointer is NULL");
+  const HostPlan q = make_host_plan(h, batch, T, b, seg_chunks);
+  if (!device_buffer || buffer_bytes < q.total) return fail(TTT_ERR_WORKSPACE, "device buffer missing or too small");
+  if (reinterpret_cast<uintptr_t>(device_buffer) % 256)
+    return fail(TTT_ERR_INVALID_ARG, "device buffer must be 256-byte aligned");
+  int dev = 0;
+  TTT_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != h->device) return fail(TTT_ERR_INVALID_ARG, "the current device is not the handle's device");
+  return prefill_host_impl(h, batch, T, b, hidden, tokens, W0, M0, W, M, eta, beta, gamma, chunk_loss,
+                           static_cast<char*>(device_buffer), q, static_cast<cudaStream_t>(stream));
 }
 
 ttt_status ttt_prefill_recon(ttt_handle* h, int32_t batch, int32_t T, int32_t b, const float* K, const float* V,

@@ -27,6 +27,7 @@ RULE = {"e2ttt": 0, "lact": 1}
 HEAD = {"lm": 0, "recon": 1}
 
 EXPORTED = ["ttt_create", "ttt_destroy", "ttt_workspace_size", "ttt_prefill", "ttt_prefill_noalloc",
+            "ttt_prefill_host", "ttt_host_buffer_size",
             "ttt_prefill_profiled", "ttt_prefill_recon", "ttt_predict", "ttt_set_attention",
             "ttt_scalar_kernels", "ttt_scalar_heads", "ttt_gemm_bf16",
             "ttt_get_device_status", "ttt_selftest_bounded_wait", "ttt_status_string",
@@ -73,6 +74,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ttt_prefill.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill.restype = I32
     lib.ttt_prefill_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P]
+    lib.ttt_host_buffer_size.argtypes = [P, I32, I32, I32, I32, ctypes.POINTER(SZ)]
+    lib.ttt_host_buffer_size.restype = I32
+    lib.ttt_prefill_host.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.ttt_prefill_host.restype = I32
     lib.ttt_prefill_recon.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.ttt_prefill_recon.restype = I32
     lib.ttt_predict.argtypes = [P, I32, I32, I32, P, P, P, P, P, P, SZ, P]
@@ -245,6 +250,7 @@ class Handle:
         with torch.cuda.device(dev):
             self._h = ttt_create(self.cfg, lm_head, rms_gain, static_w)
         self._ws = None
+        self._hbuf = None   # device buffer of the host-buffer prefill, grown on demand
 
     def set_attention(self, n_heads: int, window: int, attn_w, ln_gain, ln_bias, ln_eps: float = 1e-5):
         """Frozen sliding-window attention in front of every updated block:
@@ -260,6 +266,7 @@ class Handle:
             _check(load_library().ttt_set_attention(self._h, n_heads, window, _ptr(attn_w), _ptr(ln_gain),
                                                     _ptr(ln_bias), ln_eps), "ttt_set_attention")
         self._ws = None
+        self._hbuf = None
 
     # workspace cached per handle, grown on demand
     def workspace(self, batch: int, T: int, b: int) -> torch.Tensor:
@@ -395,28 +402,50 @@ class Handle:
                     flops=stats[i].flops, bytes=stats[i].bytes) for i in range(n.value)]
         return loss, out
 
-    def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None, scalar_heads=None):
-        """End-to-end call on HOST tensors: copies the inputs to the device,
-        runs the inner loop, copies W, M and the chunk losses back.  Returns
-        (W, M, chunk_loss) as host tensors.  scalar_heads = (heads [3, d] CUDA
-        tensor, bias[3], eta_base, alpha_base, tau): the scalars come from
-        ttt_scalar_heads on the device (eta, beta, gamma are then ignored)."""
+    def prefill_host(self, hidden, tokens, W0, M0, eta, beta, gamma, b: int, stream=None, scalar_heads=None,
+                     seg_chunks: int = 0):
+        """End-to-end call on HOST tensors: the inputs go to the device, the
+        inner loop runs, W, M and the chunk losses come back.  Returns
+        (W, M, chunk_loss) as new host tensors (pinned).  Without scalar heads
+        this is ttt_prefill_host (the sequence streamed in segments of
+        seg_chunks chunks, copies overlapping the compute; pass pinned host
+        tensors).  scalar_heads = (heads [3, d] CUDA tensor, bias[3],
+        eta_base, alpha_base, tau): the scalars come from ttt_scalar_heads on
+        the device (eta, beta, gamma are then ignored), after a plain copy of
+        the inputs."""
         dev = self.device
         st = stream if stream is not None else torch.cuda.current_stream(dev)
-        with torch.cuda.stream(st):
-            if scalar_heads is None:
-                d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0, eta, beta, gamma)]
-            else:
+        if scalar_heads is not None:
+            with torch.cuda.stream(st):
                 d_in = [t.to(dev, non_blocking=True) for t in (hidden, tokens, W0, M0)]
                 d_in += list(ttt_scalar_heads(d_in[0], *scalar_heads, stream=st))
-            loss = self.prefill(*d_in, b=b, stream=st)
-            outs = []
-            for t in (d_in[2], d_in[3], loss):
-                o = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                o.copy_(t, non_blocking=True)
-                outs.append(o)
-        st.synchronize()
-        return tuple(outs)
+                loss = self.prefill(*d_in, b=b, stream=st)
+                outs = []
+                for t in (d_in[2], d_in[3], loss):
+                    o = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    o.copy_(t, non_blocking=True)
+                    outs.append(o)
+            st.synchronize()
+            return tuple(outs)
+        for name, t, dt in (("hidden", hidden, torch.float32), ("tokens", tokens, torch.int32),
+                            ("W0", W0, torch.float32), ("M0", M0, torch.float32), ("eta", eta, torch.float32),
+                            ("beta", beta, torch.float32), ("gamma", gamma, torch.float32)):
+            if t.device.type != "cpu" or t.dtype != dt or not t.is_contiguous():
+                raise ValueError(f"{name}: expected a contiguous {dt} host tensor")
+        B, T = hidden.shape[0], hidden.shape[1]
+        lib = load_library()
+        need = ctypes.c_size_t(0)
+        _check(lib.ttt_host_buffer_size(self._h, B, T, b, seg_chunks, ctypes.byref(need)), "ttt_host_buffer_size")
+        if self._hbuf is None or self._hbuf.numel() < need.value:
+            self._hbuf = torch.empty(need.value, dtype=torch.uint8, device=dev)
+        W = torch.empty(W0.shape, dtype=torch.float32, pin_memory=True)
+        M = torch.empty(M0.shape, dtype=torch.float32, pin_memory=True)
+        loss = torch.empty((B, T // b if b > 0 else 0), dtype=torch.float32, pin_memory=True)
+        with torch.cuda.device(dev):
+            _check(lib.ttt_prefill_host(self._h, B, T, b, seg_chunks, _ptr(hidden), _ptr(tokens), _ptr(W0),
+                                        _ptr(M0), _ptr(W), _ptr(M), _ptr(eta), _ptr(beta), _ptr(gamma), _ptr(loss),
+                                        _ptr(self._hbuf), self._hbuf.numel(), _stream_ptr(st)), "ttt_prefill_host")
+        return W, M, loss
 
     def device_status(self, stream=None) -> int:
         return load_library().ttt_get_device_status(self._h, _stream_ptr(stream))
@@ -430,6 +459,7 @@ class Handle:
             ttt_destroy(self._h)
             self._h = None
         self._ws = None
+        self._hbuf = None
 
     def __del__(self):
         try:
