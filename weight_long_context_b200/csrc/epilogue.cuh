@@ -14,6 +14,8 @@
 //   Proposition 3.1 state update (same page, 命题3.1 and Algorithm 1).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace ttt {
@@ -278,18 +280,47 @@ struct EpiB1 {
     } else {
       // h % 16 == 0 and c0 % 32 == 0: nv is 16 or 32, whole groups of 16.
       // dA columns c0 + 16 g + k own positions 2 c0 + 32 g + k (gate) and + 16 (up).
+      // bf16: both groups' factors are loaded (packed) before either dU
+      // group is stored, so their latencies overlap.
+      const int ng = nv > 16 ? 2 : 1;
+      const int64_t p0 = ob + 2 * (int64_t)c0;
+      if constexpr (!std::is_same<T, __nv_bfloat16>::value) {
+        for (int g = 0; g < ng; ++g) {
+          float f[32], du[32];
+          vld<32>(fac + p0 + 32 * g, f);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            du[k] = v[16 * g + k] * f[k];
+            du[16 + k] = v[16 * g + k] * f[16 + k];
+          }
+          vst<32>(dU + p0 + 32 * g, du);
+        }
+        return;
+      }
+      uint4 fr[2][4];
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+        if (g < ng) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) fr[g][i] = reinterpret_cast<const uint4*>(fac + p0 + 32 * g)[i];
+        }
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
-        if (16 * g >= nv) break;
-        const int64_t p0 = ob + 2 * (int64_t)c0 + 32 * g;
+        if (g >= ng) break;
         float f[32], du[32];
-        vld<32>(fac + p0, f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 a = unpack_bf16x2(fr[g][i].x), b = unpack_bf16x2(fr[g][i].y);
+          const float2 c = unpack_bf16x2(fr[g][i].z), e = unpack_bf16x2(fr[g][i].w);
+          f[8 * i] = a.x; f[8 * i + 1] = a.y; f[8 * i + 2] = b.x; f[8 * i + 3] = b.y;
+          f[8 * i + 4] = c.x; f[8 * i + 5] = c.y; f[8 * i + 6] = e.x; f[8 * i + 7] = e.y;
+        }
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           du[k] = v[16 * g + k] * f[k];
           du[16 + k] = v[16 * g + k] * f[16 + k];
         }
-        vst<32>(dU + p0, du);
+        vst<32>(dU + p0 + 32 * g, du);
       }
     }
   }
