@@ -30,6 +30,20 @@ __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ----------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialisation attribute (launch_dependent below) may be scheduled
+// while the previous kernel of its stream still runs, once every CTA of that
+// kernel has called grid_launch_dependents() or exited.  It may set up shared
+// memory, barriers and TMEM, but must not read or write global memory before
+// grid_dependency_wait() returns: that waits for the previous kernel to
+// complete with its writes visible (to TMA loads too).  Both are no-ops in a
+// kernel launched the ordinary way.  Because every kernel so launched waits
+// before it completes, completion stays ordered along the whole stream.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // SwiGLU layout of the fused [gate; up] dimension inside the library:
 // 32-wide groups, gate columns j in [16g, 16g+16) at positions [32g, 32g+16),
 // up columns at [32g+16, 32g+32).  h must be a multiple of 16.

@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 
 #include <cstdlib>
+#include <utility>
 
 #include "common.cuh"
 #include "gemm_types.cuh"
@@ -439,6 +440,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Barriers and TMEM are set up: wait for the previous kernel of the stream
+  // before the first global access, then let the next one be scheduled onto
+  // SMs as they free up.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   const GemmShape& s = p.s;
 
@@ -744,6 +750,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant_
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Barriers and TMEM are set up: wait for the previous kernel of the stream
+  // before the first global access, then let the next one be scheduled onto
+  // SMs as they free up.
+  grid_dependency_wait();
+  grid_launch_dependents();
   const GemmShape& s = p.s;
 
   if (warp == 0) {
@@ -1082,6 +1093,36 @@ inline int num_sms() {
   return n;
 }
 
+// 1: GEMMs are launched as programmatic dependents of the previous kernel in
+// their stream, so their launch and set-up overlap its tail (env TTT_PDL=0
+// launches them the ordinary way, for A/B timing).
+inline int pdl_mode() {
+  static int m = -1;
+  if (m < 0) {
+    const char* e = getenv("TTT_PDL");
+    m = (e && e[0] == '0') ? 0 : 1;
+  }
+  return m;
+}
+
+// Launch `kernel` with the programmatic stream-serialisation attribute (see
+// grid_dependency_wait); the kernel must wait before its first global access.
+template <class... KArgs, class... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_mode() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // 3-D map of a bf16 operand: dims (inner, outer, batch).  K-major: inner = K,
 // outer = MN rows; MN-major: inner = MN, outer = K rows.  Box: 64 inner
 // elements (128 bytes, 128-byte swizzle) by box_outer rows.
@@ -1158,8 +1199,7 @@ cudaError_t launch_tc(const GemmShape& s, const Operand& A, const Operand& A2, c
   p.partial = nullptr;
   p.counters = nullptr;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  gemm_tc_kernel<NACC, BN, Epi><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
-  return cudaGetLastError();
+  return launch_dependent(gemm_tc_kernel<NACC, BN, Epi>, grid, C::NTHREADS, C::SMEM_BYTES, st, ma, ma2, mb, p, epi);
 }
 
 // Fraction of the machine a GEMM keeps busy with N tile `bn`: tiles over
@@ -1311,8 +1351,8 @@ cudaError_t launch_tc2(const GemmShape& s, const Operand& A, const Operand& A2, 
   const int pairs = num_sms() / 2;
   const int units = p.num_units;
   const int grid = 2 * (units < pairs ? units : pairs);
-  gemm_tc2_kernel<NACC, BN, Epi, DUALB><<<grid, C::NTHREADS, C::SMEM_BYTES, st>>>(ma, ma2, mb, p, epi);
-  return cudaGetLastError();
+  return launch_dependent(gemm_tc2_kernel<NACC, BN, Epi, DUALB>, grid, C::NTHREADS, C::SMEM_BYTES, st, ma, ma2, mb, p,
+                          epi);
 }
 
 // 0: 1-SM kernel, 1: CTA-pair kernel (env TTT_GEMM_PAIR=0 forces 1-SM, for A/B timing).

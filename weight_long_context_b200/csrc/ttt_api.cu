@@ -98,6 +98,13 @@ struct ttt_handle {
   cudaStream_t copy = nullptr;
   cudaEvent_t ev_copied[2] = {nullptr, nullptr};
   cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
+  // the plain prefill's aggregation stream: each dynamic MLP's two
+  // aggregations run on it beside the next MLPs' backward GEMMs
+  cudaStream_t agg = nullptr;
+  bool agg_stream = true;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_up[3] = {nullptr, nullptr, nullptr};    // dU buffer k read by its aggregation
+  cudaEvent_t ev_out[3] = {nullptr, nullptr, nullptr};   // doutW/doutM buffer k read by its aggregation
   ttt::GraphSlot graph[ttt::N_SLOTS];
   bool use_graph = true;
   // Frozen sliding-window attention in front of every updated block
@@ -122,7 +129,7 @@ struct Plan {
   bool swiglu, has_static;
   size_t esz;  // operand element size
   size_t KW, KM, consts, Wsh, resid, actin, aw, am, act, fac, z, rstd, part, tgt, lse, ltok, P, dz, dout, dout_a,
-      doutW[2], doutM[2], dU, sk_partial, sk_counters, total;
+      doutW[3], doutM[3], dU, dUx[2], sk_partial, sk_counters, total;
   bool recon;           // reconstruction head: no LM-head buffers; yk, yq, qres below
   size_t yk, yq, qres;  // fp32 [n, d]: MLP outputs on the keys and queries, the query rows
   size_t sk_partial_bytes, sk_counter_count;
@@ -195,8 +202,9 @@ static Plan make_plan(const ttt_handle* hd, int B, int T, int b) {
   p.dz = take(4 * n * d);
   p.dout = take(4 * n * d);
   p.dout_a = take(e * n * d);
-  for (int i = 0; i < 2; ++i) { p.doutW[i] = take(e * n * d); p.doutM[i] = take(e * n * d); }
+  for (int i = 0; i < 3; ++i) { p.doutW[i] = take(e * n * d); p.doutM[i] = take(e * n * d); }
   p.dU = take(e * n * H2);
+  for (int i = 0; i < 2; ++i) p.dUx[i] = take(e * n * H2);
   p.yk = take(p.recon ? 4 * n * d : 0);
   p.yq = take(p.recon ? 4 * n * d : 0);
   p.qres = take(p.recon ? 4 * n * d : 0);
@@ -408,12 +416,12 @@ static cudaError_t enqueue_forward(ttt_handle* hd, const Plan& p, const float* h
 // partials), the per-token and chunk losses, CE pass B and dz per vocabulary
 // slab, RMSNorm backward.  Leaves the residual-stream gradient in dout (fp32),
 // its operand copy in dout_a and the K-scaled copies for the top MLP in
-// doutW / doutM [(nM - 1) & 1].
+// doutW / doutM [top_buf].
 // ---------------------------------------------------------------------------
 template <typename T>
 static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens, float* chunk_loss, int c,
                                 const float* KW, const float* KM, char* ws, const SplitScratch& ss,
-                                cudaStream_t st, Prof& prof) {
+                                cudaStream_t st, Prof& prof, int top_buf) {
   const int B = p.B, b = p.b, n = p.n, d = p.d, V = p.V;
   float* resid = reinterpret_cast<float*>(ws + p.resid);
   T* z = reinterpret_cast<T*>(ws + p.z);
@@ -426,8 +434,8 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
   float* dz = reinterpret_cast<float*>(ws + p.dz);
   float* dout = reinterpret_cast<float*>(ws + p.dout);
   T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
-  T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
-  T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
+  T* doutW = reinterpret_cast<T*>(ws + p.doutW[top_buf]);
+  T* doutM = reinterpret_cast<T*>(ws + p.doutM[top_buf]);
   const T* E = static_cast<const T*>(hd->E);
   int* status = hd->status;
   cudaError_t err;
@@ -464,12 +472,9 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
              TRY((gemm<T, 1>(s, A, A, Be, EpiStoreF32{dz, d, sl > 0 ? 1 : 0}, st, status, ss))));
     }
   }
-  {
-    const int top = p.nM - 1;  // always dynamic
-    LAUNCH(K_RMS_BWD, 0, (12.0 + 3.0 * e) * n * d,
-           (rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a,
-                                                               doutW[top & 1], doutM[top & 1], KW, KM, p.kscale, tm)));
-  }
+  LAUNCH(K_RMS_BWD, 0, (12.0 + 3.0 * e) * n * d,
+         (rmsnorm_bwd_kernel<T><<<(n + 7) / 8, 256, 0, st>>>(dz, resid, rstd, hd->gain, n, d, dout, dout_a, doutW,
+                                                             doutM, KW, KM, p.kscale, tm)));
   return cudaSuccess;
 }
 
@@ -492,9 +497,16 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   T* fac = reinterpret_cast<T*>(ws + p.fac);
   float* dout = reinterpret_cast<float*>(ws + p.dout);
   T* dout_a = reinterpret_cast<T*>(ws + p.dout_a);
-  T* doutW[2] = {reinterpret_cast<T*>(ws + p.doutW[0]), reinterpret_cast<T*>(ws + p.doutW[1])};
-  T* doutM[2] = {reinterpret_cast<T*>(ws + p.doutM[0]), reinterpret_cast<T*>(ws + p.doutM[1])};
-  T* dU = reinterpret_cast<T*>(ws + p.dU);
+  // three rotating buffers each: an aggregation on the side stream may still
+  // read the ones of the MLP two levels up while this level writes its own
+  T* doutW[3];
+  T* doutM[3];
+  T* dUb[3];
+  for (int k = 0; k < 3; ++k) {
+    doutW[k] = reinterpret_cast<T*>(ws + p.doutW[k]);
+    doutM[k] = reinterpret_cast<T*>(ws + p.doutM[k]);
+    dUb[k] = reinterpret_cast<T*>(ws + (k == 0 ? p.dU : p.dUx[k - 1]));
+  }
   const T* S = static_cast<const T*>(hd->S);
   int* status = hd->status;
   SplitScratch ss;
@@ -524,11 +536,20 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   auto is_dyn = [&](int i) { return (i % per_blk) == per_blk - 1; };
   auto blk_of = [&](int i) { return i / per_blk; };
 
+  // Each dynamic MLP's two aggregations depend only on its own backward
+  // (dU, the K-scaled copies) and write only its own weights, so they run on
+  // the handle's aggregation stream beside the backward GEMMs of the MLPs
+  // below, which fill each other's last waves.  The forward of the next chunk
+  // waits for all of them.  Serial when the launches are timed one by one.
+  const bool conc = hd->agg_stream && hd->agg && !prof.timing;
+  const cudaStream_t ast = conc ? hd->agg : st;
+  bool up_pend[3] = {false, false, false}, out_pend[3] = {false, false, false};
+
   for (int c = 0; c < p.nchunks; ++c) {
     TokenMap tm{b, p.T, c};
     TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, true, KW, KM, ws, ss, st, prof));
 
-    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof));
+    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof, (p.nM - 1) % 3));
 
     // ---- backward, top down ----
     for (int i = p.nM - 1; i >= i_min; --i) {
@@ -540,6 +561,12 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
       const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
       const bool need_dx = i > i_min;
       T* fi = fac + (int64_t)i * n * H2;
+      const int k = i % 3;
+      T* dU = dUb[k];
+      if (up_pend[k]) {   // the aggregation of MLP i + 3 still reads dU[k]
+        TRY(cudaStreamWaitEvent(st, hd->ev_up[k], 0));
+        up_pend[k] = false;
+      }
       {  // B1: dA = dOut W2 -> dU
         GemmShape s{Mz, h, d, Bz};
         Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
@@ -554,8 +581,13 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         Operand A = opnd(dU, H2, (int64_t)Mz * H2, 1, Mz);
         Operand Bw = opnd(w1, d, wstride, 0, H2);
         const bool below_dyn = is_dyn(i - 1);
-        T* ow = below_dyn ? doutW[(i - 1) & 1] : nullptr;
-        T* om = below_dyn ? doutM[(i - 1) & 1] : nullptr;
+        const int ko = (i - 1) % 3;
+        if (below_dyn && out_pend[ko]) {   // the aggregation of MLP i + 2 still reads doutW/doutM[ko]
+          TRY(cudaStreamWaitEvent(st, hd->ev_out[ko], 0));
+          out_pend[ko] = false;
+        }
+        T* ow = below_dyn ? doutW[ko] : nullptr;
+        T* om = below_dyn ? doutM[ko] : nullptr;
         LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
                e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
                TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status, ss))));
@@ -565,6 +597,12 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
         float* Wl = W + l * blk;
         float* Ml = M + l * blk;
         T* Sl = Wsh + l * blk;
+        // after this MLP's dA and dX, which read the shadow rows these update
+        if (conc) {
+          TRY(cudaEventRecord(hd->ev_fork, st));
+          TRY(cudaStreamWaitEvent(ast, hd->ev_fork, 0));
+        }
+        const cudaStream_t st = ast;
         {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens:
            // sum_t dU_t (x) (-K_t x_t), A = dU shared by both accumulators
           GemmShape s{H2, d, b, B};
@@ -576,10 +614,14 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
                  (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
                  TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
         }
+        if (conc) {
+          TRY(cudaEventRecord(hd->ev_up[k], st));
+          up_pend[k] = true;
+        }
         {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
           GemmShape s{d, h, b, B};
-          Operand A = opnd(doutW[i & 1], d, (int64_t)b * d, 0, b);
-          Operand A2 = opnd(doutM[i & 1], d, (int64_t)b * d, 0, b);
+          Operand A = opnd(doutW[k], d, (int64_t)b * d, 0, b);
+          Operand A2 = opnd(doutM[k], d, (int64_t)b * d, 0, b);
           Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
           EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
                           consts, c, p.nchunks, h, 0};
@@ -587,7 +629,16 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
                  (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
                  TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
         }
+        if (conc) {
+          TRY(cudaEventRecord(hd->ev_out[k], st));
+          out_pend[k] = true;
+        }
       }
+    }
+    if (conc) {   // the next chunk's forward reads the updated shadow
+      TRY(cudaEventRecord(hd->ev_join, ast));
+      TRY(cudaStreamWaitEvent(st, hd->ev_join, 0));
+      for (int k = 0; k < 3; ++k) up_pend[k] = out_pend[k] = false;
     }
   }
   return cudaSuccess;
@@ -804,7 +855,7 @@ static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const floa
     }
 
     // ---- head ----
-    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof));
+    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof, (p.nM - 1) & 1));
 
     // ---- backward of the top block's MLPs (row-local) ----
     for (int i = p.nM - 1; i >= std::max(i_top, i_min); --i) {
@@ -1504,6 +1555,15 @@ ttt_status ttt_create(const ttt_config* cfg, const float* lm_head, const float* 
   h->zero_flag = h->status + 1;
   CTRY(cudaMemset(h->status, 0, 8));
   CTRY(cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking));
+  const char* env_agg = getenv("TTT_AGG_STREAM");   // 0: aggregations on the caller's stream (A/B timing)
+  h->agg_stream = !(env_agg && env_agg[0] == '0');
+  CTRY(cudaStreamCreateWithFlags(&h->agg, cudaStreamNonBlocking));
+  CTRY(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+  CTRY(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
+  for (int i = 0; i < 3; ++i) {
+    CTRY(cudaEventCreateWithFlags(&h->ev_up[i], cudaEventDisableTiming));
+    CTRY(cudaEventCreateWithFlags(&h->ev_out[i], cudaEventDisableTiming));
+  }
   if (!recon) {   // the frozen LM head and RMSNorm gain
     CTRY(cudaMalloc(&h->E, esz * V * d));
     CTRY(cudaMalloc(&h->gain, 4 * d));
@@ -1548,6 +1608,10 @@ void ttt_destroy(ttt_handle* h) {
     if (h->ev_copied[i]) cudaEventDestroy(h->ev_copied[i]);
     if (h->ev_consumed[i]) cudaEventDestroy(h->ev_consumed[i]);
   }
+  if (h->agg) { cudaStreamSynchronize(h->agg); cudaStreamDestroy(h->agg); }
+  for (cudaEvent_t ev : {h->ev_fork, h->ev_join, h->ev_up[0], h->ev_up[1], h->ev_up[2], h->ev_out[0], h->ev_out[1],
+                         h->ev_out[2]})
+    if (ev) cudaEventDestroy(ev);
   if (h->cap) cudaStreamDestroy(h->cap);
   delete h;
 }
