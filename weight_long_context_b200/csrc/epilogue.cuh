@@ -45,6 +45,16 @@ __device__ __forceinline__ float gelu_grad_f(float u) {
   return cdf + u * pdf;
 }
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+// The exponential and the logistic function inside the GEMM epilogues: the
+// accurate library forms with fp32 operands; with bf16 operands, whose
+// results are rounded to 8 significant bits or only feed the chunk loss, the
+// hardware approximations __expf and __frcp_rn (relative error about 1e-6
+// over the arguments met here), which keep the epilogue of the cross-entropy
+// and SwiGLU tiles off the critical path of the next tile's MMAs.
+template <typename T> __device__ __forceinline__ float exp_op(float x) { return expf(x); }
+template <> __device__ __forceinline__ float exp_op<__nv_bfloat16>(float x) { return __expf(x); }
+template <typename T> __device__ __forceinline__ float sigmoid_op(float x) { return sigmoid_f(x); }
+template <> __device__ __forceinline__ float sigmoid_op<__nv_bfloat16>(float x) { return __frcp_rn(1.0f + __expf(-x)); }
 
 // ---------------------------------------------------------------------------
 // Vector access helpers: N contiguous elements, 16-byte aligned.  Where the
@@ -237,7 +247,7 @@ struct EpiF1 {
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         float gv = v[k], uv = v[16 + k];
-        float sg = sigmoid_f(gv);
+        float sg = sigmoid_op<T>(gv);
         float silu = gv * sg;
         av[k] = silu * uv;
         fv[k] = uv * sg * (1.0f + gv * (1.0f - sg));
@@ -451,6 +461,7 @@ struct EpiB2 {
 // the logits (online softmax), and the target logit.  The logits stay on chip.
 // `part_index` (from the engine) numbers the column parts of a row.
 // ---------------------------------------------------------------------------
+template <typename T>
 struct EpiCEPartial {
   static constexpr bool kFixedHeadTile = true;
   static constexpr bool kPreload = false;
@@ -470,10 +481,10 @@ struct EpiCEPartial {
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 32; ++j) if (j < nv) mx = fmaxf(mx, v[j]);
-    if (mx > st.m) { st.s *= expf(st.m - mx); st.m = mx; }
+    if (mx > st.m) { st.s *= exp_op<T>(st.m - mx); st.m = mx; }
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) if (j < nv) acc += expf(v[j] - st.m);
+    for (int j = 0; j < 32; ++j) if (j < nv) acc += exp_op<T>(v[j] - st.m);
     st.s += acc;
     int k = st.y - c0;
     if (k >= 0 && k < nv) {
@@ -511,7 +522,7 @@ struct EpiCEGrad {
     const int k = y - slab0 - c0;
     float p[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) p[j] = expf(v[j] - l) - (j == k ? 1.0f : 0.0f);
+    for (int j = 0; j < 32; ++j) p[j] = exp_op<T>(v[j] - l) - (j == k ? 1.0f : 0.0f);
     if (nv == 32) vst<32>(o, p);
     else {
 #pragma unroll

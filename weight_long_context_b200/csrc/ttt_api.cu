@@ -448,7 +448,7 @@ static cudaError_t enqueue_head(ttt_handle* hd, const Plan& p, const int* tokens
     Operand A = opnd(z, d, 0, 1, n);
     Operand Be = opnd(E, d, 0, 1, V);
     LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-           TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
+           TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial<T>{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
   }
   LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + 16.0 * n,
          (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status)));
@@ -1223,7 +1223,7 @@ static cudaError_t enqueue_predict(ttt_handle* hd, const Plan& p, const float* h
       Operand A = opnd(z, d, 0, 1, n);
       Operand Be = opnd(E, d, 0, 1, V);
       LAUNCH(K_CE_LSE, 2.0 * n * V * d, e * ((double)n * d + (double)V * d) + 8.0 * n * p.ntn,
-             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
+             TRY((gemm<T, 1>(s, A, A, Be, EpiCEPartial<T>{part, tgt, tokens, tm, p.ntn}, st, status, ss))));
     }
     LAUNCH(K_CE_ROWS, 0, 8.0 * n * p.ntn + (token_loss ? 20.0 : 16.0) * n,
            (ce_rows_kernel<<<(n + 7) / 8, 256, 0, st>>>(part, tgt, p.ntn, tokens, tm, V, n, lse, ltok, status,
