@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <cstdlib>
+#include <utility>
 
 #include "../../include/ttt.h"
 
@@ -43,6 +45,36 @@ __device__ __forceinline__ void record_error(int* status, int code) {
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// 1: kernels are launched as programmatic dependents of the previous kernel
+// in their stream, so their launch and set-up overlap its tail (env
+// TTT_PDL=0 launches them the ordinary way, for A/B timing).
+inline int pdl_mode() {
+  static int m = -1;
+  if (m < 0) {
+    const char* e = getenv("TTT_PDL");
+    m = (e && e[0] == '0') ? 0 : 1;
+  }
+  return m;
+}
+
+// Launch `kernel` with the programmatic stream-serialisation attribute (see
+// grid_dependency_wait); the kernel must wait before its first global access.
+template <class... KArgs, class... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_mode() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // SwiGLU layout of the fused [gate; up] dimension inside the library:
 // 32-wide groups, gate columns j in [16g, 16g+16) at positions [32g, 32g+16),

@@ -1093,36 +1093,6 @@ inline int num_sms() {
   return n;
 }
 
-// 1: GEMMs are launched as programmatic dependents of the previous kernel in
-// their stream, so their launch and set-up overlap its tail (env TTT_PDL=0
-// launches them the ordinary way, for A/B timing).
-inline int pdl_mode() {
-  static int m = -1;
-  if (m < 0) {
-    const char* e = getenv("TTT_PDL");
-    m = (e && e[0] == '0') ? 0 : 1;
-  }
-  return m;
-}
-
-// Launch `kernel` with the programmatic stream-serialisation attribute (see
-// grid_dependency_wait); the kernel must wait before its first global access.
-template <class... KArgs, class... Args>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
-                             Args&&... args) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_mode() ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
 // 3-D map of a bf16 operand: dims (inner, outer, batch).  K-major: inner = K,
 // outer = MN rows; MN-major: inner = MN, outer = K rows.  Box: 64 inner
 // elements (128 bytes, 128-byte swizzle) by box_outer rows.
