@@ -408,10 +408,21 @@ def test_bounded_wait_times_out_cleanly(dev):
     h.close()
 
 
-def test_profiled_path_matches_graph_path(dev):
-    """ttt_prefill_profiled runs the same kernels eagerly with events: results
-    are bit-identical to the graph path and every launch is accounted for."""
-    w = I.Workload("prof", 128, 256, 544, 2, "swiglu", True, "bf16", 256, 64, 2, "e2ttt")
+PROF_CASES = [
+    I.Workload("prof", 128, 256, 544, 2, "swiglu", True, "bf16", 256, 64, 2, "e2ttt"),
+    # eight MLP levels: the backward reuses each of the three rotating dU and
+    # output-gradient buffers while the aggregation stream may still read it
+    I.Workload("prof_deep", 128, 256, 544, 4, "swiglu", True, "bf16", 256, 64, 2, "e2ttt"),
+    I.Workload("prof_deep_gelu", 96, 224, 416, 5, "gelu", False, "bf16", 192, 64, 1, "e2ttt"),
+]
+
+
+@pytest.mark.parametrize("w", PROF_CASES, ids=[c.name for c in PROF_CASES])
+def test_profiled_path_matches_graph_path(dev, w):
+    """ttt_prefill_profiled runs the same kernels eagerly and serially, with
+    events: results are bit-identical to the graph path, whose aggregations
+    run on a second stream beside the backward, and every launch is
+    accounted for."""
     x = I.make_inputs(w, seed=4, m0_scale=1e-3)
     Wa, Ma, La, st, h = H.run_gpu(w, x, dev, return_handle=True)
     t = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev, dt)
@@ -426,7 +437,8 @@ def test_profiled_path_matches_graph_path(dev):
     upd = next(s for s in stats if s["name"] == "agg_update")
     # two aggregation GEMMs per dynamic MLP per chunk, 2 x 2 x rows x cols x b x batch FLOPs
     assert upd["launches"] == 2 * w.n_blocks * w.n_chunks
-    assert upd["flops"] == pytest.approx(4.0 * 3 * w.hidden * w.d * w.b * w.batch * w.n_blocks * w.n_chunks)
+    m = 3 if w.mlp == "swiglu" else 2
+    assert upd["flops"] == pytest.approx(4.0 * m * w.hidden * w.d * w.b * w.batch * w.n_blocks * w.n_chunks)
     h.close()
 
 
