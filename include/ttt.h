@@ -35,7 +35,10 @@
  *     frozen-parameter copies a handle owns.
  *   - Enqueued work is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream).  Argument and shape errors are returned
- *     synchronously and launch nothing.
+ *     synchronously and launch nothing.  Inside a prefill the aggregation
+ *     GEMMs run on a second stream the handle owns, forked from and joined
+ *     back into `stream` with events, so the call's work is ordered on
+ *     `stream` as a whole.
  *   - Errors found on the device (token out of range, non-finite loss, a
  *     bounded wait that ran out) are recorded in the handle's device status
  *     word and read back with ttt_get_device_status().
