@@ -81,7 +81,9 @@ struct EpiStoreHeads {
 
 // Scores pass A: per (head, query) row and column part of the tile, the
 // online-softmax partial (max, sum exp) of scale * s over the keys inside the
-// window (empty parts give (-inf, 0)).  The scores never reach HBM.
+// window (empty parts give (-inf, 0)).  The scores never reach HBM.  The
+// exponential is exp_op<T>: with bf16 operands the hardware approximation.
+template <typename T>
 struct EpiScorePartial {
   static constexpr bool kFixedHeadTile = true;
   static constexpr bool kPreload = false;
@@ -95,20 +97,21 @@ struct EpiScorePartial {
   float scale;
   __device__ void row_begin(RowState& st, int, int) const { st.m = -INFINITY; st.s = 0.f; }
   __device__ void span(RowState& st, int, int r, int c0, const float* v, const float*, int nv) const {
-    const int64_t qpos = q0 + r;
+    // query position minus the span's first key position (|.| < 2^31)
+    const int base = (int)(q0 + r - (j0 + c0));
     float x[32];
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const int64_t dlt = qpos - (j0 + c0 + j);
-      x[j] = (j < nv && dlt >= 0 && dlt < window) ? v[j] * scale : -INFINITY;
+      const bool in = j < nv && (unsigned)(base - j) < (unsigned)window;
+      x[j] = in ? v[j] * scale : -INFINITY;
       mx = fmaxf(mx, x[j]);
     }
     if (mx == -INFINITY) return;
-    if (mx > st.m) { st.s *= expf(st.m - mx); st.m = mx; }
+    if (mx > st.m) { st.s *= exp_op<T>(st.m - mx); st.m = mx; }
     float acc = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc += expf(x[j] - st.m);
+    for (int j = 0; j < 32; ++j) acc += exp_op<T>(x[j] - st.m);
     st.s += acc;
   }
   __device__ void row_end(RowState& st, int z, int r, int part_index) const {
@@ -138,13 +141,10 @@ struct EpiScoreP {
   __device__ void span(RowState&, int z, int r, int c0, const float* v, const float*, int nv) const {
     const int64_t row = (int64_t)z * b + r;
     const float l = lse[row];
-    const int64_t qpos = q0 + r;
+    const int base = (int)(q0 + r - (j0 + c0));   // as in EpiScorePartial
     float x[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int64_t dlt = qpos - (j0 + c0 + j);
-      x[j] = (dlt >= 0 && dlt < window) ? expf(v[j] * scale - l) : 0.f;
-    }
+    for (int j = 0; j < 32; ++j) x[j] = (unsigned)(base - j) < (unsigned)window ? exp_op<T>(v[j] * scale - l) : 0.f;
     T* o = P + row * ldS + c0;
     if (nv == 32 && (ldS & 7) == 0 && (c0 & 7) == 0) {
       vst<32>(o, x);

@@ -784,7 +784,7 @@ static cudaError_t enqueue_prefill_swa(ttt_handle* hd, const Plan& p, const floa
           Operand Aq = opnd(qs, dh, (int64_t)b * dh, 1, b);
           Operand Bk = opnd(ks, dh, Tn * dh, 1, nk);
           LAUNCH(K_ATTN_SCORE, 2.0 * b * nk * dh * H, e * ((double)b + nk) * dh * H + 8.0 * H * b * ntn,
-                 TRY((gemm<T, 1>(g, Aq, Aq, Bk, EpiScorePartial{spart, b, ntn, q0, j0, p.window, scale}, st, status,
+                 TRY((gemm<T, 1>(g, Aq, Aq, Bk, EpiScorePartial<T>{spart, b, ntn, q0, j0, p.window, scale}, st, status,
                                  ss))));
           LAUNCH(K_ATTN_ROWS, 0, 8.0 * H * b * ntn + 4.0 * H * b,
                  (attn_lse_kernel<<<(H * b + 7) / 8, 256, 0, st>>>(spart, ntn, (int64_t)H * b, slse)));
