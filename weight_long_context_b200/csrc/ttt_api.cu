@@ -10,7 +10,8 @@
 //   per vocabulary slab: CE pass B (softmax - onehot) and dz += P E_slab ->
 //   RMSNorm backward -> per MLP, top down: B1 (dA, dU), B2 (dX) when a
 //   dynamic MLP lies below, and for dynamic MLPs the dual-accumulator
-//   aggregation whose epilogue writes W, M and the operand shadow in place.
+//   aggregation whose epilogue writes W, M and the operand shadow in place
+//   (on a second stream, beside the backward of the MLPs below).
 // The final prediction (ttt_predict) runs the same forward and CE pass A at
 // fixed weights, with no backward.  The whole sequence of launches of a call
 // is captured once into a CUDA graph on a private stream and replayed on the
