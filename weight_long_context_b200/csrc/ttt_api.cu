@@ -546,103 +546,113 @@ static cudaError_t enqueue_prefill(ttt_handle* hd, const Plan& p, const float* h
   const cudaStream_t ast = conc ? hd->agg : st;
   bool up_pend[3] = {false, false, false}, out_pend[3] = {false, false, false};
 
-  for (int c = 0; c < p.nchunks; ++c) {
-    TokenMap tm{b, p.T, c};
-    TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, true, KW, KM, ws, ss, st, prof));
+  auto chunks = [&]() -> cudaError_t {
+    for (int c = 0; c < p.nchunks; ++c) {
+      TokenMap tm{b, p.T, c};
+      TRY(enqueue_forward<T>(hd, p, hidden, Wsh, c, true, KW, KM, ws, ss, st, prof));
 
-    TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof, (p.nM - 1) % 3));
+      TRY(enqueue_head<T>(hd, p, tokens, chunk_loss, c, KW, KM, ws, ss, st, prof, (p.nM - 1) % 3));
 
-    // ---- backward, top down ----
-    for (int i = p.nM - 1; i >= i_min; --i) {
-      const bool dyn = is_dyn(i);
-      const int l = blk_of(i);
-      const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
-      const T* w2 = w1 + (int64_t)H2 * d;
-      const int64_t wstride = dyn ? seqW : 0;
-      const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
-      const bool need_dx = i > i_min;
-      T* fi = fac + (int64_t)i * n * H2;
-      const int k = i % 3;
-      T* dU = dUb[k];
-      if (up_pend[k]) {   // the aggregation of MLP i + 3 still reads dU[k]
-        TRY(cudaStreamWaitEvent(st, hd->ev_up[k], 0));
-        up_pend[k] = false;
+      // ---- backward, top down ----
+      for (int i = p.nM - 1; i >= i_min; --i) {
+        const bool dyn = is_dyn(i);
+        const int l = blk_of(i);
+        const T* w1 = dyn ? Wsh + l * blk : S + l * blk;
+        const T* w2 = w1 + (int64_t)H2 * d;
+        const int64_t wstride = dyn ? seqW : 0;
+        const int Bz = dyn ? B : 1, Mz = dyn ? b : n;
+        const bool need_dx = i > i_min;
+        T* fi = fac + (int64_t)i * n * H2;
+        const int k = i % 3;
+        T* dU = dUb[k];
+        if (up_pend[k]) {   // the aggregation of MLP i + 3 still reads dU[k]
+          TRY(cudaStreamWaitEvent(st, hd->ev_up[k], 0));
+          up_pend[k] = false;
+        }
+        {  // B1: dA = dOut W2 -> dU
+          GemmShape s{Mz, h, d, Bz};
+          Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
+          Operand Bw = opnd(w2, h, wstride, 0, d);
+          const double fl = 2.0 * Mz * h * d * Bz;
+          const double by = e * ((double)n * d + (double)d * h * Bz + 2.0 * n * H2);
+          if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, dU, h, Mz}, st, status, ss))));
+          else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, dU, h, Mz}, st, status, ss))));
+        }
+        if (need_dx) {  // B2: dout += dU W1
+          GemmShape s{Mz, d, H2, Bz};
+          Operand A = opnd(dU, H2, (int64_t)Mz * H2, 1, Mz);
+          Operand Bw = opnd(w1, d, wstride, 0, H2);
+          const bool below_dyn = is_dyn(i - 1);
+          const int ko = (i - 1) % 3;
+          if (below_dyn && out_pend[ko]) {   // the aggregation of MLP i + 2 still reads doutW/doutM[ko]
+            TRY(cudaStreamWaitEvent(st, hd->ev_out[ko], 0));
+            out_pend[ko] = false;
+          }
+          T* ow = below_dyn ? doutW[ko] : nullptr;
+          T* om = below_dyn ? doutM[ko] : nullptr;
+          LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
+                 e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
+                 TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status, ss))));
+        }
+        if (dyn) {
+          T* aout = act + (int64_t)i * n * h;
+          float* Wl = W + l * blk;
+          float* Ml = M + l * blk;
+          T* Sl = Wsh + l * blk;
+          // after this MLP's dA and dX, which read the shadow rows these update
+          if (conc) {
+            TRY(cudaEventRecord(hd->ev_fork, st));
+            TRY(cudaStreamWaitEvent(ast, hd->ev_fork, 0));
+          }
+          const cudaStream_t st = ast;
+          {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens:
+             // sum_t dU_t (x) (-K_t x_t), A = dU shared by both accumulators
+            GemmShape s{H2, d, b, B};
+            Operand A = opnd(dU, H2, (int64_t)b * H2, 0, b);
+            Operand B1 = opnd(aw + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+            Operand B2 = opnd(am + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
+            EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
+            LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B,
+                   (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
+                   TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
+          }
+          if (conc) {
+            TRY(cudaEventRecord(hd->ev_up[k], st));
+            up_pend[k] = true;
+          }
+          {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
+            GemmShape s{d, h, b, B};
+            Operand A = opnd(doutW[k], d, (int64_t)b * d, 0, b);
+            Operand A2 = opnd(doutM[k], d, (int64_t)b * d, 0, b);
+            Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
+            EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
+                            consts, c, p.nchunks, h, 0};
+            LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B,
+                   (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
+                   TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
+          }
+          if (conc) {
+            TRY(cudaEventRecord(hd->ev_out[k], st));
+            out_pend[k] = true;
+          }
+        }
       }
-      {  // B1: dA = dOut W2 -> dU
-        GemmShape s{Mz, h, d, Bz};
-        Operand A = opnd(dout_a, d, (int64_t)Mz * d, 1, Mz);
-        Operand Bw = opnd(w2, h, wstride, 0, d);
-        const double fl = 2.0 * Mz * h * d * Bz;
-        const double by = e * ((double)n * d + (double)d * h * Bz + 2.0 * n * H2);
-        if (sw) LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, true>{fi, dU, h, Mz}, st, status, ss))));
-        else LAUNCH(K_BWD_DA, fl, by, TRY((gemm<T, 1>(s, A, A, Bw, EpiB1<T, false>{fi, dU, h, Mz}, st, status, ss))));
-      }
-      if (need_dx) {  // B2: dout += dU W1
-        GemmShape s{Mz, d, H2, Bz};
-        Operand A = opnd(dU, H2, (int64_t)Mz * H2, 1, Mz);
-        Operand Bw = opnd(w1, d, wstride, 0, H2);
-        const bool below_dyn = is_dyn(i - 1);
-        const int ko = (i - 1) % 3;
-        if (below_dyn && out_pend[ko]) {   // the aggregation of MLP i + 2 still reads doutW/doutM[ko]
-          TRY(cudaStreamWaitEvent(st, hd->ev_out[ko], 0));
-          out_pend[ko] = false;
-        }
-        T* ow = below_dyn ? doutW[ko] : nullptr;
-        T* om = below_dyn ? doutM[ko] : nullptr;
-        LAUNCH(K_BWD_DX, 2.0 * Mz * d * H2 * Bz,
-               e * ((double)n * H2 + (double)H2 * d * Bz + (double)n * d * (ow ? 3 : 1)) + 8.0 * n * d,
-               TRY((gemm<T, 1>(s, A, A, Bw, EpiB2<T>{dout, dout_a, ow, om, KW, KM, p.kscale, tm, d, Mz}, st, status, ss))));
-      }
-      if (dyn) {
-        T* aout = act + (int64_t)i * n * h;
-        float* Wl = W + l * blk;
-        float* Ml = M + l * blk;
-        T* Sl = Wsh + l * blk;
-        // after this MLP's dA and dX, which read the shadow rows these update
-        if (conc) {
-          TRY(cudaEventRecord(hd->ev_fork, st));
-          TRY(cudaStreamWaitEvent(ast, hd->ev_fork, 0));
-        }
-        const cudaStream_t st = ast;
-        {  // rows of W1 (and W2 for SwiGLU): [H2, d], contraction over the b tokens:
-           // sum_t dU_t (x) (-K_t x_t), A = dU shared by both accumulators
-          GemmShape s{H2, d, b, B};
-          Operand A = opnd(dU, H2, (int64_t)b * H2, 0, b);
-          Operand B1 = opnd(aw + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
-          Operand B2 = opnd(am + (int64_t)i * n * d, d, (int64_t)b * d, 0, b);
-          EpiUpdate<T> ep{Wl, Ml, Sl, seqW, seqW, consts, c, p.nchunks, d, sw ? h : 0};
-          LAUNCH(K_AGG_UPDATE, 4.0 * H2 * d * b * B,
-                 (16.0 + e) * H2 * d * B + e * ((double)n * H2 + 2.0 * n * d),
-                 TRY((gemm_dualb<T>(s, A, B1, B2, ep, st, status))));
-        }
-        if (conc) {
-          TRY(cudaEventRecord(hd->ev_up[k], st));
-          up_pend[k] = true;
-        }
-        {  // the output matrix (W2 for GELU, W3 for SwiGLU): [d, h]
-          GemmShape s{d, h, b, B};
-          Operand A = opnd(doutW[k], d, (int64_t)b * d, 0, b);
-          Operand A2 = opnd(doutM[k], d, (int64_t)b * d, 0, b);
-          Operand Bx = opnd(aout, h, (int64_t)b * h, 0, b);
-          EpiUpdate<T> ep{Wl + (int64_t)H2 * d, Ml + (int64_t)H2 * d, Sl + (int64_t)H2 * d, seqW, seqW,
-                          consts, c, p.nchunks, h, 0};
-          LAUNCH(K_AGG_UPDATE, 4.0 * d * h * b * B,
-                 (16.0 + e) * d * h * B + e * ((double)n * d * 2 + (double)n * h),
-                 TRY((gemm<T, 2>(s, A, A2, Bx, ep, st, status))));
-        }
-        if (conc) {
-          TRY(cudaEventRecord(hd->ev_out[k], st));
-          out_pend[k] = true;
-        }
+      if (conc) {   // the next chunk's forward reads the updated shadow
+        TRY(cudaEventRecord(hd->ev_join, ast));
+        TRY(cudaStreamWaitEvent(st, hd->ev_join, 0));
+        for (int k = 0; k < 3; ++k) up_pend[k] = out_pend[k] = false;
       }
     }
-    if (conc) {   // the next chunk's forward reads the updated shadow
-      TRY(cudaEventRecord(hd->ev_join, ast));
-      TRY(cudaStreamWaitEvent(st, hd->ev_join, 0));
-      for (int k = 0; k < 3; ++k) up_pend[k] = out_pend[k] = false;
-    }
+    return cudaSuccess;
+  };
+  err = chunks();
+  // A failed launch leaves the call early: order what the aggregation stream
+  // already holds before anything the caller enqueues next (best effort).
+  if (err != cudaSuccess && conc) {
+    cudaEventRecord(hd->ev_join, ast);
+    cudaStreamWaitEvent(st, hd->ev_join, 0);
   }
-  return cudaSuccess;
+  return err;
 }
 
 // ---------------------------------------------------------------------------
